@@ -1,0 +1,149 @@
+// C ABI of the KDA library: argument checks on the host, then one launch on the
+// caller's stream.  Nothing here allocates, synchronizes or throws.
+#include <stdint.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+
+namespace {
+
+bool head_size_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool dtype_ok(kda_dtype t) { return t == KDA_F32 || t == KDA_BF16; }
+size_t dsize(kda_dtype t) { return t == KDA_BF16 ? 2 : 4; }
+bool aligned16(const void *p) { return p == nullptr || ((uintptr_t)p & 15u) == 0; }
+
+struct Range {
+    uintptr_t lo, hi;
+};
+Range range_of(const void *p, size_t bytes) { return Range{(uintptr_t)p, (uintptr_t)p + bytes}; }
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi && a.lo != a.hi && b.lo != b.hi; }
+
+// Common checks of the prefill-shaped entry points.  Sizes are in elements.
+kda_status check_forward(const void *q, const void *k, const void *v, const void *alpha,
+                         const void *beta, const float *s_in, const void *o, const float *s_out,
+                         int B, int T, int H, int dk, int dv, kda_dtype qkv, kda_dtype gate,
+                         kda_dtype out)
+{
+    if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return KDA_ERR_SHAPE;
+    if (!dtype_ok(qkv) || !dtype_ok(gate) || !dtype_ok(out)) return KDA_ERR_DTYPE;
+    if (!head_size_ok(dk) || !head_size_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    const unsigned long long tokens = (unsigned long long)B * T * H;
+    if (tokens * (unsigned long long)(dk > dv ? dk : dv) >= (1ull << 62)) return KDA_ERR_SHAPE;
+    if (B * (long long)H == 0) return KDA_OK;
+    if (T > 0 && (!q || !k || !v || !alpha || !beta || !o)) return KDA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(alpha) || !aligned16(beta) ||
+        !aligned16(s_in) || !aligned16(o) || !aligned16(s_out))
+        return KDA_ERR_ALIGN;
+    if (T > 0) {
+        const Range ro = range_of(o, tokens * dv * dsize(out));
+        const Range ins[] = {range_of(q, tokens * dk * dsize(qkv)), range_of(k, tokens * dk * dsize(qkv)),
+                             range_of(v, tokens * dv * dsize(qkv)), range_of(alpha, tokens * dk * dsize(gate)),
+                             range_of(beta, tokens * dsize(gate)),
+                             range_of(s_in, s_in ? (size_t)B * H * dk * dv * 4 : 0),
+                             range_of(s_out, s_out ? (size_t)B * H * dk * dv * 4 : 0)};
+        for (const Range &r : ins)
+            if (overlap(ro, r)) return KDA_ERR_ALIAS;
+    }
+    return KDA_OK;
+}
+
+// T = 0: the final state is the initial state (or zeros).
+kda_status empty_sequence(const float *s_in, float *s_out, int B, int H, int dk, int dv,
+                          cudaStream_t stream)
+{
+    if (!s_out || B * (long long)H == 0) return KDA_OK;
+    const size_t bytes = (size_t)B * H * dk * dv * sizeof(float);
+    cudaError_t err = cudaSuccess;
+    if (!s_in)
+        err = cudaMemsetAsync(s_out, 0, bytes, stream);
+    else if (s_in != s_out)
+        err = cudaMemcpyAsync(s_out, s_in, bytes, cudaMemcpyDeviceToDevice, stream);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *kda_status_string(kda_status s)
+{
+    switch (s) {
+    case KDA_OK: return "ok";
+    case KDA_ERR_NULL: return "a required pointer is NULL";
+    case KDA_ERR_SHAPE: return "a size is negative or too large";
+    case KDA_ERR_DTYPE: return "unknown dtype code";
+    case KDA_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case KDA_ERR_UNSUPPORTED: return "head size must be 16, 32, 64 or 128";
+    case KDA_ERR_WORKSPACE: return "workspace missing or too small";
+    case KDA_ERR_LAUNCH: return "CUDA launch failed";
+    case KDA_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+    case KDA_ERR_ALIAS: return "an output overlaps an input";
+    }
+    return "unknown status";
+}
+
+int kda_version(void) { return 100; }
+
+size_t kda_forward_workspace_bytes(int B, int T, int H, int d_k, int d_v)
+{
+    (void)B; (void)T; (void)H; (void)d_k; (void)d_v;
+    return 0;
+}
+
+kda_status kda_forward(const void *q, const void *k, const void *v, const void *alpha,
+                       const void *beta, const float *initial_state, void *o, float *final_state,
+                       int B, int T, int H, int d_k, int d_v, float scale, kda_dtype qkv_dtype,
+                       kda_dtype gate_dtype, kda_dtype out_dtype, void *workspace,
+                       size_t workspace_bytes, cudaStream_t stream)
+{
+    kda_status st = check_forward(q, k, v, alpha, beta, initial_state, o, final_state, B, T, H,
+                                  d_k, d_v, qkv_dtype, gate_dtype, out_dtype);
+    if (st != KDA_OK) return st;
+    const size_t need = kda_forward_workspace_bytes(B, T, H, d_k, d_v);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
+    if (B * (long long)H == 0) return KDA_OK;
+    if (T == 0) return empty_sequence(initial_state, final_state, B, H, d_k, d_v, stream);
+    kda::ChunkArgs a{q, k, v, alpha, beta, initial_state, final_state, o, B, T, H, scale,
+                     qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16};
+    cudaError_t err;
+    if (kda::chunk_tc_supported(d_k, d_v, qkv_dtype, gate_dtype))
+        err = kda::launch_chunk_tc(a, d_k, d_v, stream);
+    else
+        err = kda::launch_chunk_simt(a, d_k, d_v, stream);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+}
+
+kda_status kda_forward_sequential(const void *q, const void *k, const void *v, const void *alpha,
+                                  const void *beta, const float *initial_state, void *o,
+                                  float *final_state, int B, int T, int H, int d_k, int d_v,
+                                  float scale, kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                                  kda_dtype out_dtype, cudaStream_t stream)
+{
+    kda_status st = check_forward(q, k, v, alpha, beta, initial_state, o, final_state, B, T, H,
+                                  d_k, d_v, qkv_dtype, gate_dtype, out_dtype);
+    if (st != KDA_OK) return st;
+    if (B * (long long)H == 0) return KDA_OK;
+    if (T == 0) return empty_sequence(initial_state, final_state, B, H, d_k, d_v, stream);
+    kda::RecurrentArgs a{q, k, v, alpha, beta, initial_state, final_state, o, B, T, H, scale,
+                         qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16};
+    return kda::launch_recurrent(a, d_k, d_v, stream) == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+}
+
+kda_status kda_decode_step(const void *q, const void *k, const void *v, const void *alpha,
+                           const void *beta, float *state, void *o, int N, int H, int d_k,
+                           int d_v, float scale, kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                           kda_dtype out_dtype, cudaStream_t stream)
+{
+    if (N * (long long)H > 0 && !state) return KDA_ERR_NULL;
+    kda_status st = check_forward(q, k, v, alpha, beta, state, o, nullptr, N, 1, H, d_k, d_v,
+                                  qkv_dtype, gate_dtype, out_dtype);
+    if (st != KDA_OK) return st;
+    if (N * (long long)H == 0) return KDA_OK;
+    // the state is read and rewritten in place; one token per sequence
+    kda::RecurrentArgs a{q, k, v, alpha, beta, state, state, o, N, 1, H, scale,
+                         qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16};
+    return kda::launch_recurrent(a, d_k, d_v, stream) == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+}
+
+}  // extern "C"

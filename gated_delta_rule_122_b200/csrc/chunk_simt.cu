@@ -1,0 +1,237 @@
+// Chunkwise KDA on CUDA cores, fp32 throughout: the general path for every
+// supported head size and input dtype (the tensor-core kernel covers
+// d_k = d_v = 128 with bf16 q/k/v).
+//
+// One block per (sequence, head); chunks of C = 32 tokens are walked in order
+// with the state S [DK x DV] resident in shared memory.  For a chunk with
+// cumulative log-decay G[r] = sum_{t<=r} log alpha_t (per key channel):
+//   Akk[r][s] = beta_r sum_d k_rd k_sd exp(G_rd - G_sd)           s <  r
+//   Aqk[r][s] =        sum_d q_rd k_sd exp(G_rd - G_sd)           s <= r
+//   (I + Akk) W = Diag(beta) (K * exp(G)),  (I + Akk) U = Diag(beta) V
+//   E = U - W S                          (the true in-chunk errors)
+//   O = scale ((Q * exp(G)) S + Aqk E)
+//   S <- Diag(exp(G_end)) S + (K * exp(G_end - G))^T E
+// Every pairwise decay exp(G_r - G_s), s <= r, is formed directly, so no
+// factor ever exceeds 1 and no anchoring is needed on this path.
+// Algorithm: "Kimi Delta Attention (KDA)" (brain.bigb.es), "Two schedules for
+// the same recurrence"; "From Fast Weight Programmers to KDA"
+// (jonahsamost.bearblog.dev), section "Kimi Delta Attention".
+#include "common.cuh"
+#include "kernels.h"
+
+namespace kda {
+
+
+constexpr int kSimtChunk = 32;
+constexpr int kSimtThreads = 256;
+
+template <int DK, int DV>
+struct SimtLayout {
+    static constexpr int C = kSimtChunk;
+    static constexpr int PK = DK + 1, PV = DV + 1, PC = C + 1;
+    static constexpr int oQ = 0;
+    static constexpr int oK = oQ + C * PK;
+    static constexpr int oG = oK + C * PK;
+    static constexpr int oW = oG + C * PK;
+    static constexpr int oV = oW + C * PK;
+    static constexpr int oE = oV + C * PV;
+    static constexpr int oS = oE + C * PV;
+    static constexpr int oAkk = oS + DK * DV;
+    static constexpr int oAqk = oAkk + C * PC;
+    static constexpr int oBeta = oAqk + C * PC;
+    static constexpr int floats = oBeta + C;
+    static constexpr size_t bytes = sizeof(float) * (size_t)floats;
+};
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(kSimtThreads)
+kda_chunk_simt_kernel(ChunkArgs a)
+{
+    using Ly = SimtLayout<DK, DV>;
+    constexpr int C = Ly::C, PK = Ly::PK, PV = Ly::PV, PC = Ly::PC, NT = kSimtThreads;
+    constexpr int NRG = NT / DV;          // row groups for value-column loops
+    constexpr int RPT_C = C / NRG;        // chunk rows per thread
+    constexpr int RPT_K = DK / NRG;       // key rows per thread (state update)
+    static_assert(NT % DV == 0 && C % NRG == 0 && DK % NRG == 0, "thread mapping");
+
+    extern __shared__ float sm[];
+    float *Q = sm + Ly::oQ, *K = sm + Ly::oK, *G = sm + Ly::oG, *W = sm + Ly::oW;
+    float *V = sm + Ly::oV, *E = sm + Ly::oE, *S = sm + Ly::oS;
+    float *Akk = sm + Ly::oAkk, *Aqk = sm + Ly::oAqk, *Bt = sm + Ly::oBeta;
+
+    const int bh = blockIdx.x;
+    const int b = bh / a.H, h = bh % a.H;
+    const int tid = threadIdx.x;
+    const size_t tile = (size_t)bh * DK * DV;
+
+    for (int idx = tid; idx < DK * DV; idx += NT)
+        S[idx] = a.s_in ? a.s_in[tile + idx] : 0.f;
+
+    const int jcol = tid % DV, rgrp = tid / DV;
+
+    for (int t0 = 0; t0 < a.T; t0 += C) {
+        const int L = min(C, a.T - t0);
+        // 1. stage the chunk; rows >= L are identity steps (k = q = v = 0, alpha = 1, beta = 0)
+        for (int idx = tid; idx < C * DK; idx += NT) {
+            const int r = idx / DK, d = idx % DK;
+            float qv = 0.f, kv = 0.f, gv = 0.f;
+            if (r < L) {
+                const size_t row = ((size_t)b * a.T + t0 + r) * a.H + h;
+                qv = ld_elem(a.q, row * DK + d, a.qkv_bf16);
+                kv = ld_elem(a.k, row * DK + d, a.qkv_bf16);
+                gv = log_alpha(ld_elem(a.alpha, row * DK + d, a.gate_bf16));
+            }
+            Q[r * PK + d] = qv; K[r * PK + d] = kv; G[r * PK + d] = gv;
+        }
+        for (int idx = tid; idx < C * DV; idx += NT) {
+            const int r = idx / DV, j = idx % DV;
+            float vv = 0.f;
+            if (r < L) {
+                const size_t row = ((size_t)b * a.T + t0 + r) * a.H + h;
+                vv = ld_elem(a.v, row * DV + j, a.qkv_bf16);
+            }
+            V[r * PV + j] = vv;
+        }
+        for (int r = tid; r < C; r += NT) {
+            Bt[r] = (r < L) ? ld_elem(a.beta, ((size_t)b * a.T + t0 + r) * a.H + h, a.gate_bf16) : 0.f;
+        }
+        __syncthreads();
+
+        // 2. inclusive cumulative log-decay per key channel
+        for (int d = tid; d < DK; d += NT) {
+            float run = 0.f;
+            for (int r = 0; r < C; ++r) { run += G[r * PK + d]; G[r * PK + d] = run; }
+        }
+        __syncthreads();
+
+        // 3. interaction matrices and the right-hand sides of the triangular solves
+        for (int p = tid; p < C * C; p += NT) {
+            const int r = p / C, s = p % C;
+            float akk = 0.f, aqk = 0.f;
+            if (s <= r) {
+                for (int d = 0; d < DK; ++d) {
+                    const float ks = K[s * PK + d] * expf(G[r * PK + d] - G[s * PK + d]);
+                    akk = fmaf(K[r * PK + d], ks, akk);
+                    aqk = fmaf(Q[r * PK + d], ks, aqk);
+                }
+            }
+            Akk[r * PC + s] = (s < r) ? Bt[r] * akk : 0.f;
+            Aqk[r * PC + s] = aqk;
+        }
+        for (int idx = tid; idx < C * DK; idx += NT) {
+            const int r = idx / DK, d = idx % DK;
+            W[r * PK + d] = Bt[r] * K[r * PK + d] * expf(G[r * PK + d]);
+        }
+        for (int idx = tid; idx < C * DV; idx += NT) {
+            const int r = idx / DV, j = idx % DV;
+            V[r * PV + j] *= Bt[r];
+        }
+        __syncthreads();
+
+        // 4. forward substitution (I + Akk) X = RHS, one column per thread;
+        //    then the decay-scaled operands of the inter-chunk products
+        for (int col = tid; col < DK + DV; col += NT) {
+            float *X = (col < DK) ? (W + col) : (V + (col - DK));
+            const int stride = (col < DK) ? PK : PV;
+            float x[C];
+#pragma unroll
+            for (int i = 0; i < C; ++i) x[i] = X[i * stride];
+#pragma unroll
+            for (int i = 1; i < C; ++i) {
+                float acc = x[i];
+#pragma unroll
+                for (int j = 0; j < i; ++j) acc = fmaf(-Akk[i * PC + j], x[j], acc);
+                x[i] = acc;
+            }
+#pragma unroll
+            for (int i = 0; i < C; ++i) X[i * stride] = x[i];
+        }
+        __syncthreads();
+        for (int idx = tid; idx < C * DK; idx += NT) {
+            const int r = idx / DK, d = idx % DK;
+            const float g = G[r * PK + d];
+            Q[r * PK + d] *= expf(g);                              // q * gamma_r
+            K[r * PK + d] *= expf(G[(C - 1) * PK + d] - g);        // k * gamma_end / gamma_r
+        }
+        __syncthreads();
+
+        // 5. E = U - W S and the inter-chunk read (Q * gamma) S
+        float oacc[RPT_C];
+#pragma unroll
+        for (int m = 0; m < RPT_C; ++m) {
+            const int r = rgrp + NRG * m;
+            float e = V[r * PV + jcol], o = 0.f;
+            for (int d = 0; d < DK; ++d) {
+                const float sdj = S[d * DV + jcol];
+                e = fmaf(-W[r * PK + d], sdj, e);
+                o = fmaf(Q[r * PK + d], sdj, o);
+            }
+            E[r * PV + jcol] = e;
+            oacc[m] = o;
+        }
+        __syncthreads();
+
+        // 6. outputs: O = scale (inter + Aqk E)
+#pragma unroll
+        for (int m = 0; m < RPT_C; ++m) {
+            const int r = rgrp + NRG * m;
+            float o = oacc[m];
+            for (int s = 0; s <= r; ++s) o = fmaf(Aqk[r * PC + s], E[s * PV + jcol], o);
+            if (r < L) {
+                const size_t row = ((size_t)b * a.T + t0 + r) * a.H + h;
+                st_elem(a.o, row * DV + jcol, a.scale * o, a.out_bf16);
+            }
+        }
+        // 7. state fast-forward: S <- Diag(gamma_end) S + K_end^T E
+#pragma unroll 4
+        for (int m = 0; m < RPT_K; ++m) {
+            const int i = rgrp + NRG * m;
+            float s = S[i * DV + jcol] * expf(G[(C - 1) * PK + i]);
+            for (int r = 0; r < C; ++r) s = fmaf(K[r * PK + i], E[r * PV + jcol], s);
+            S[i * DV + jcol] = s;
+        }
+        __syncthreads();
+    }
+
+    if (a.s_out)
+        for (int idx = tid; idx < DK * DV; idx += NT) a.s_out[tile + idx] = S[idx];
+}
+
+template <int DK, int DV>
+static cudaError_t launch_chunk_simt_t(const ChunkArgs &a, cudaStream_t stream)
+{
+    using Ly = SimtLayout<DK, DV>;
+    const long long blocks = (long long)a.B * a.H;
+    if (blocks == 0) return cudaSuccess;
+    cudaError_t err = cudaFuncSetAttribute(kda_chunk_simt_kernel<DK, DV>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)Ly::bytes);
+    if (err != cudaSuccess) return err;
+    kda_chunk_simt_kernel<DK, DV><<<(unsigned)blocks, kSimtThreads, Ly::bytes, stream>>>(a);
+    return cudaGetLastError();
+}
+
+template <int DK>
+static cudaError_t launch_chunk_simt_dv(const ChunkArgs &a, int dv, cudaStream_t s)
+{
+    switch (dv) {
+    case 16: return launch_chunk_simt_t<DK, 16>(a, s);
+    case 32: return launch_chunk_simt_t<DK, 32>(a, s);
+    case 64: return launch_chunk_simt_t<DK, 64>(a, s);
+    case 128: return launch_chunk_simt_t<DK, 128>(a, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_chunk_simt(const ChunkArgs &a, int dk, int dv, cudaStream_t s)
+{
+    switch (dk) {
+    case 16: return launch_chunk_simt_dv<16>(a, dv, s);
+    case 32: return launch_chunk_simt_dv<32>(a, dv, s);
+    case 64: return launch_chunk_simt_dv<64>(a, dv, s);
+    case 128: return launch_chunk_simt_dv<128>(a, dv, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace kda

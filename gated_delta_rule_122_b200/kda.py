@@ -1,0 +1,228 @@
+"""Python binding of the KDA C ABI (include/kda.h): argument marshalling only.
+
+Every computation runs in the CUDA library ``libkda_b200.so`` built in-tree by
+``gated_delta_rule_122_b200.build``.  If the library is missing, calls raise;
+there is no fallback of any kind.  Tensors must be contiguous; device tensors
+are passed as raw pointers together with the current CUDA stream.  Host
+(CPU) tensors are accepted too: they are copied to the current device, the same
+C entry point runs, and the results are copied back (the end-to-end path).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = ["KDAError", "forward", "forward_sequential", "decode_step", "library", "library_path",
+           "status_string", "version", "EXPORTED_SYMBOLS"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libkda_b200.so")
+_lib = None
+_lock = threading.Lock()
+
+EXPORTED_SYMBOLS = ("kda_forward", "kda_forward_workspace_bytes", "kda_forward_sequential",
+                    "kda_decode_step", "kda_status_string", "kda_version")
+
+_DT = {torch.float32: 0, torch.bfloat16: 1}
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+
+
+class KDAError(RuntimeError):
+    """A non-OK status returned by the KDA C library."""
+
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {status_string(code)} (status {code})")
+        self.code = code
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def library() -> ctypes.CDLL:
+    """Load libkda_b200.so (once).  Raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError("the KDA CUDA library is not built (expected "
+                                   f"{_LIB_PATH}); run: python -m gated_delta_rule_122_b200.build")
+            lib = ctypes.CDLL(_LIB_PATH)
+            fwd_args = [_vp] * 8 + [_i] * 5 + [_f] + [_i] * 3
+            lib.kda_forward.argtypes = fwd_args + [_vp, ctypes.c_size_t, _vp]
+            lib.kda_forward.restype = _i
+            lib.kda_forward_sequential.argtypes = fwd_args + [_vp]
+            lib.kda_forward_sequential.restype = _i
+            lib.kda_forward_workspace_bytes.argtypes = [_i] * 5
+            lib.kda_forward_workspace_bytes.restype = ctypes.c_size_t
+            lib.kda_decode_step.argtypes = [_vp] * 7 + [_i] * 4 + [_f] + [_i] * 3 + [_vp]
+            lib.kda_decode_step.restype = _i
+            lib.kda_status_string.argtypes = [_i]
+            lib.kda_status_string.restype = ctypes.c_char_p
+            lib.kda_version.argtypes = []
+            lib.kda_version.restype = _i
+            _lib = lib
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return library().kda_status_string(int(code)).decode()
+
+
+def version() -> int:
+    return library().kda_version()
+
+
+def _ptr(t):
+    return None if t is None else _vp(t.data_ptr())
+
+
+def _dt(t: torch.Tensor, name: str) -> int:
+    if t.dtype not in _DT:
+        raise TypeError(f"{name}: dtype {t.dtype} not supported (float32 or bfloat16)")
+    return _DT[t.dtype]
+
+
+def _check(name, t, device):
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _stream_handle(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _to_device(tensors, device):
+    return [None if t is None else t.to(device, non_blocking=True) for t in tensors]
+
+
+def _prefill(fn_name, q, k, v, alpha, beta, initial_state, scale, output_final_state,
+             out_dtype, out, final_state):
+    host = q.device.type == "cpu"
+    host_out = host_state = None
+    if host:
+        # end-to-end path: host inputs are copied in (asynchronously when pinned),
+        # results are copied back into host tensors before returning
+        dev = torch.device("cuda", torch.cuda.current_device())
+        q, k, v, alpha, beta, initial_state = _to_device(
+            [q, k, v, alpha, beta, initial_state], dev)
+        host_out, host_state = out, final_state
+        out = None if out is None else torch.empty(out.shape, device=dev, dtype=out.dtype)
+        final_state = None if final_state is None else torch.empty(final_state.shape, device=dev,
+                                                                    dtype=final_state.dtype)
+    device = q.device
+    if device.type != "cuda":
+        raise ValueError("KDA runs on CUDA devices only")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for name, t in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta", beta)):
+        _check(name, t, device)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k and v must share a dtype")
+    if alpha.dtype != beta.dtype:
+        raise TypeError("alpha and beta must share a dtype")
+    if tuple(k.shape) != (B, T, H, dk) or tuple(alpha.shape) != (B, T, H, dk) \
+            or tuple(v.shape) != (B, T, H, dv) or tuple(beta.shape) != (B, T, H):
+        raise ValueError("shapes: q,k,alpha [B,T,H,dk], v [B,T,H,dv], beta [B,T,H]")
+    if initial_state is not None:
+        _check("initial_state", initial_state, device)
+        if initial_state.dtype != torch.float32 or tuple(initial_state.shape) != (B, H, dk, dv):
+            raise ValueError("initial_state must be float32 [B,H,dk,dv]")
+    if scale is None:
+        scale = dk ** -0.5
+    if out is None:
+        out = torch.empty((B, T, H, dv), device=device, dtype=out_dtype)
+    _check("out", out, device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((B, H, dk, dv), device=device, dtype=torch.float32)
+    if final_state is not None:
+        _check("final_state", final_state, device)
+    lib = library()
+    args = [_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(initial_state), _ptr(out),
+            _ptr(final_state), B, T, H, dk, dv, float(scale), _DT[q.dtype], _dt(alpha, "alpha"),
+            _dt(out, "out")]
+    with torch.cuda.device(device):
+        stream = _vp(_stream_handle(device))
+        if fn_name == "kda_forward":
+            ws_bytes = lib.kda_forward_workspace_bytes(B, T, H, dk, dv)
+            ws = torch.empty(ws_bytes, device=device, dtype=torch.uint8) if ws_bytes else None
+            code = lib.kda_forward(*args, _ptr(ws), ws_bytes, stream)
+        else:
+            code = lib.kda_forward_sequential(*args, stream)
+    if code != 0:
+        raise KDAError(fn_name, code)
+    if host:
+        with torch.cuda.device(device):
+            if host_out is None:
+                host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+            host_out.copy_(out, non_blocking=True)
+            if final_state is not None:
+                if host_state is None:
+                    host_state = torch.empty(final_state.shape, dtype=final_state.dtype,
+                                             pin_memory=True)
+                host_state.copy_(final_state, non_blocking=True)
+            torch.cuda.current_stream(device).synchronize()
+        return host_out, (host_state if final_state is not None else None)
+    return out, final_state
+
+
+def forward(q, k, v, alpha, beta, initial_state=None, scale=None, output_final_state=True,
+            out_dtype=torch.float32, out=None, final_state=None):
+    """Chunkwise KDA prefill (C entry point ``kda_forward``).
+
+    q, k, alpha: [B,T,H,dk]; v: [B,T,H,dv]; beta: [B,T,H] (q/k/v share a dtype,
+    alpha/beta share a dtype; float32 or bfloat16).  initial_state: float32
+    [B,H,dk,dv] or None.  Returns (o [B,T,H,dv] of out_dtype, final_state or None).
+    """
+    return _prefill("kda_forward", q, k, v, alpha, beta, initial_state, scale,
+                    output_final_state, out_dtype, out, final_state)
+
+
+def forward_sequential(q, k, v, alpha, beta, initial_state=None, scale=None,
+                       output_final_state=True, out_dtype=torch.float32, out=None,
+                       final_state=None):
+    """The token-by-token schedule (C entry point ``kda_forward_sequential``); same contract."""
+    return _prefill("kda_forward_sequential", q, k, v, alpha, beta, initial_state, scale,
+                    output_final_state, out_dtype, out, final_state)
+
+
+def decode_step(q, k, v, alpha, beta, state, scale=None, out_dtype=torch.float32, out=None):
+    """One token per sequence; ``state`` [N,H,dk,dv] float32 is updated in place.
+
+    q, k, alpha: [N,H,dk]; v: [N,H,dv]; beta: [N,H].  Returns o [N,H,dv].
+    """
+    device = state.device
+    if device.type != "cuda":
+        raise ValueError("decode_step needs the state on a CUDA device")
+    N, H, dk, dv = state.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta", beta),
+                    ("state", state)):
+        _check(name, t, device)
+    if state.dtype != torch.float32:
+        raise TypeError("state must be float32")
+    if tuple(q.shape) != (N, H, dk) or tuple(k.shape) != (N, H, dk) or \
+            tuple(alpha.shape) != (N, H, dk) or tuple(v.shape) != (N, H, dv) or \
+            tuple(beta.shape) != (N, H):
+        raise ValueError("shapes: q,k,alpha [N,H,dk], v [N,H,dv], beta [N,H], state [N,H,dk,dv]")
+    if k.dtype != q.dtype or v.dtype != q.dtype or alpha.dtype != beta.dtype:
+        raise TypeError("q/k/v and alpha/beta must each share a dtype")
+    if scale is None:
+        scale = dk ** -0.5
+    if out is None:
+        out = torch.empty((N, H, dv), device=device, dtype=out_dtype)
+    _check("out", out, device)
+    with torch.cuda.device(device):
+        code = library().kda_decode_step(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state), _ptr(out),
+            N, H, dk, dv, float(scale), _DT[q.dtype], _dt(alpha, "alpha"), _dt(out, "out"),
+            _vp(_stream_handle(device)))
+    if code != 0:
+        raise KDAError("kda_decode_step", code)
+    return out

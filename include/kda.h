@@ -1,0 +1,141 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) KDA library.
+ *
+ * KDA (Kimi Delta Attention) is the gated delta rule with one retention factor
+ * per key channel.  For each (sequence, head), with a state S in R^{d_k x d_v}
+ * (rows = key channels, columns = value channels) and per token t:
+ *
+ *   S~_t = Diag(alpha_t) S_{t-1}                 forget, per key channel
+ *   vh_t = S~_t^T k_t                            predict
+ *   e_t  = v_t - vh_t                            correct
+ *   S_t  = S~_t + beta_t k_t e_t^T               write
+ *   o_t  = S_t^T (scale q_t)                     read
+ *
+ * This is the five-step update of "Module 03 -- KDA I: The Delta-Rule
+ * Recurrence" (jared-hpc.com), section 2, in the d_k x d_v layout of the
+ * five-line recurrence in "Kimi Delta Attention (KDA)" (brain.bigb.es),
+ * section "KDA: one gate per key channel"; the scale multiplies q at the read
+ * only, as in that page's opening statement.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers, row-major and contiguous, owned
+ *    by the caller; the library allocates and frees nothing.
+ *  - Every pointer must be 16-byte aligned (KDA_ERR_ALIGN otherwise).
+ *  - Argument errors are detected on the host and returned before anything
+ *    is launched; nothing is written then.  Launch failures return
+ *    KDA_ERR_LAUNCH.  Calls are asynchronous on `stream` (0 = legacy default
+ *    stream); no call synchronizes.  No exception crosses the ABI.
+ *  - Supported head sizes: d_k, d_v in {16, 32, 64, 128}; otherwise
+ *    KDA_ERR_UNSUPPORTED.
+ *  - alpha is the linear retention factor in (0, 1] (alpha = 0 is accepted and
+ *    treated as a retention of e^-80 ~ 1.8e-35); beta is the write strength in
+ *    [0, 1]; neither is range-checked.
+ *  - Arithmetic and the state are fp32; bf16 inputs are read exactly.
+ */
+#ifndef KDA_B200_KDA_H
+#define KDA_B200_KDA_H
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element type of an input or output tensor. */
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_NULL = 1,        /* a required pointer is NULL */
+    KDA_ERR_SHAPE = 2,       /* a size is negative or a product overflows */
+    KDA_ERR_DTYPE = 3,       /* unknown dtype code */
+    KDA_ERR_ALIGN = 4,       /* a pointer is not 16-byte aligned */
+    KDA_ERR_UNSUPPORTED = 5, /* head size outside {16, 32, 64, 128} */
+    KDA_ERR_WORKSPACE = 6,   /* workspace too small or NULL when required */
+    KDA_ERR_LAUNCH = 7,      /* the CUDA launch reported an error */
+    KDA_ERR_TIMEOUT = 8,     /* a bounded device-side wait gave up */
+    KDA_ERR_ALIAS = 9        /* an output overlaps an input it must not alias */
+} kda_status;
+
+/*
+ * kda_forward -- prefill: run the recurrence over T tokens for B sequences and
+ * H heads with the chunkwise-parallel schedule.
+ *
+ * Defined by: "Kimi Delta Attention (KDA)" (brain.bigb.es), "Two schedules for
+ * the same recurrence" (provisional errors, the unit-lower-triangular
+ * correction, the one-shot state fast-forward and the diagonal-inclusive
+ * read), and "From Fast Weight Programmers to KDA" (jonahsamost.bearblog.dev),
+ * section "Kimi Delta Attention" (chunkwise WY/UT form with per-channel
+ * cumulative decay).  The result equals the sequential recurrence above up to
+ * rounding.
+ *
+ *   q, k, alpha   [B, T, H, d_k]   qkv_dtype (q, k) / gate_dtype (alpha)
+ *   v             [B, T, H, d_v]   qkv_dtype
+ *   beta          [B, T, H]        gate_dtype
+ *   initial_state [B, H, d_k, d_v] fp32, may be NULL (zero state)
+ *   o             [B, T, H, d_v]   out_dtype (written)
+ *   final_state   [B, H, d_k, d_v] fp32, may be NULL (not returned); may be
+ *                 the same pointer as initial_state (continuation in place)
+ *   scale         multiplies q at the read (callers usually pass d_k^-1/2)
+ *   workspace     device scratch of kda_forward_workspace_bytes() bytes; may be
+ *                 NULL when that size is 0
+ * T = 0 copies initial_state (or zeros) to final_state.  o must not overlap
+ * any input (KDA_ERR_ALIAS).  A last chunk shorter than the chunk size is
+ * handled exactly (no padding of the caller's buffers is needed).
+ */
+kda_status kda_forward(const void *q, const void *k, const void *v,
+                       const void *alpha, const void *beta,
+                       const float *initial_state, void *o, float *final_state,
+                       int B, int T, int H, int d_k, int d_v, float scale,
+                       kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                       kda_dtype out_dtype, void *workspace,
+                       size_t workspace_bytes, cudaStream_t stream);
+
+/* Bytes of device workspace kda_forward needs for these sizes (0 = none). */
+size_t kda_forward_workspace_bytes(int B, int T, int H, int d_k, int d_v);
+
+/*
+ * kda_forward_sequential -- the same operation and arguments as kda_forward
+ * (no workspace), computed with the token-by-token schedule ("fused
+ * recurrent" in "Two schedules for the same recurrence", brain.bigb.es): one
+ * block per (sequence, head) keeps its state on chip and walks the tokens in
+ * order.  It exists so the two schedules can be checked against each other on
+ * the GPU; it is not the fast path for long T.
+ */
+kda_status kda_forward_sequential(const void *q, const void *k, const void *v,
+                                  const void *alpha, const void *beta,
+                                  const float *initial_state, void *o,
+                                  float *final_state, int B, int T, int H,
+                                  int d_k, int d_v, float scale,
+                                  kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                                  kda_dtype out_dtype, cudaStream_t stream);
+
+/*
+ * kda_decode_step -- one token for each of N independent sequences, state
+ * updated in place: the five-step update of "Module 03", section 2, once.
+ * Each fp32 state tile is read from HBM once and written once; both
+ * reductions (S~^T k and S~^T q) come from the same read, using
+ * o = scale (S~^T q + e (k . q)) with e = beta (v - S~^T k).
+ *
+ *   q, k, alpha [N, H, d_k]  v [N, H, d_v]  beta [N, H]
+ *   state       [N, H, d_k, d_v] fp32, read and overwritten
+ *   o           [N, H, d_v] out_dtype (must not overlap state or inputs)
+ */
+kda_status kda_decode_step(const void *q, const void *k, const void *v,
+                           const void *alpha, const void *beta, float *state,
+                           void *o, int N, int H, int d_k, int d_v, float scale,
+                           kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                           kda_dtype out_dtype, cudaStream_t stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char *kda_status_string(kda_status status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_B200_KDA_H */
