@@ -92,7 +92,7 @@ class ClockSampler(threading.Thread):
         self.samples = []
         self.period = period_s
         self.err = None
-        self._stop = threading.Event()
+        self._halt = threading.Event()
         self.window = None
         self.max_mhz = None
         try:
@@ -116,7 +116,7 @@ class ClockSampler(threading.Thread):
     def run(self):
         if self.err:
             return
-        while not self._stop.is_set():
+        while not self._halt.is_set():
             try:
                 sm = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
                 rs = self._reasons(self.h)
@@ -130,7 +130,7 @@ class ClockSampler(threading.Thread):
         self.window = (t0, t1)
 
     def stop(self):
-        self._stop.set()
+        self._halt.set()
         self.join(timeout=2)
 
     def summary(self):

@@ -12,6 +12,7 @@ bool head_size_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 bool dtype_ok(kda_dtype t) { return t == KDA_F32 || t == KDA_BF16; }
 size_t dsize(kda_dtype t) { return t == KDA_BF16 ? 2 : 4; }
 bool aligned16(const void *p) { return p == nullptr || ((uintptr_t)p & 15u) == 0; }
+bool aligned_to(const void *p, size_t n) { return p == nullptr || ((uintptr_t)p % n) == 0; }
 
 struct Range {
     uintptr_t lo, hi;
@@ -32,8 +33,9 @@ kda_status check_forward(const void *q, const void *k, const void *v, const void
     if (tokens * (unsigned long long)(dk > dv ? dk : dv) >= (1ull << 62)) return KDA_ERR_SHAPE;
     if (B * (long long)H == 0) return KDA_OK;
     if (T > 0 && (!q || !k || !v || !alpha || !beta || !o)) return KDA_ERR_NULL;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(alpha) || !aligned16(beta) ||
-        !aligned16(s_in) || !aligned16(o) || !aligned16(s_out))
+    // vector tensors: 16-byte aligned rows; beta (one scalar per token): element-aligned
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(alpha) ||
+        !aligned_to(beta, dsize(gate)) || !aligned16(s_in) || !aligned16(o) || !aligned16(s_out))
         return KDA_ERR_ALIGN;
     if (T > 0) {
         const Range ro = range_of(o, tokens * dv * dsize(out));

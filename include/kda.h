@@ -20,7 +20,8 @@
  * Conventions for every entry point:
  *  - All tensor pointers are DEVICE pointers, row-major and contiguous, owned
  *    by the caller; the library allocates and frees nothing.
- *  - Every pointer must be 16-byte aligned (KDA_ERR_ALIGN otherwise).
+ *  - q, k, v, alpha, o and the state pointers must be 16-byte aligned; beta
+ *    only needs its element alignment (KDA_ERR_ALIGN otherwise).
  *  - Argument errors are detected on the host and returned before anything
  *    is launched; nothing is written then.  Launch failures return
  *    KDA_ERR_LAUNCH.  Calls are asynchronous on `stream` (0 = legacy default

@@ -73,8 +73,10 @@ def test_sequential_and_decode_reject_bad_arguments(lib):
              0, 0, 0, None) == ERR_NULL
     assert d(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 0x70000, 0x70000 + 16, 2, 2, 16, 16, 1.0,
              0, 0, 0, None) == ERR_ALIAS                    # o inside the state
-    assert d(0x10000, 0x20000, 0x30000, 0x40000, 0x50004, 0x70000, 0x60000, 2, 2, 16, 16, 1.0,
-             0, 0, 0, None) == ERR_ALIGN
+    assert d(0x10000, 0x20000, 0x30000, 0x40000, 0x50002, 0x70000, 0x60000, 2, 2, 16, 16, 1.0,
+             0, 0, 0, None) == ERR_ALIGN                    # fp32 beta, 2-byte offset
+    assert d(0x10000, 0x20000, 0x30000, 0x40008, 0x50004, 0x70000, 0x60000, 2, 2, 16, 16, 1.0,
+             0, 0, 0, None) == ERR_ALIGN                    # alpha rows need 16 bytes
 
 
 def test_workspace_query(lib):
