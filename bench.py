@@ -47,6 +47,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+                    help="run one kernel per step (for profiling); the JSON line is then partial")
     return ap.parse_args()
 
 
@@ -267,10 +269,14 @@ def main():
     od = torch.empty((wd.B, wd.H, wd.dv), device=device, dtype=torch.float32)
 
     def prefill():
+        if args.only == "decode":
+            return
         kda.forward(x["q"], x["k"], x["v"], x["alpha"], x["beta"], initial_state=x["s0"],
                     scale=x["scale"], out=o, final_state=S)
 
     def decode():
+        if args.only == "prefill":
+            return
         kda.decode_step(y["q"], y["k"], y["v"], y["alpha"], y["beta"], y["state"],
                         scale=y["scale"], out=od)
 
@@ -307,6 +313,7 @@ def main():
     pre_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
     dec_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / K
     step_ms, pre_ms, dec_ms = reduce_max(pg, [step_ms, pre_ms, dec_ms], device)
+    pre_ms, dec_ms = max(pre_ms, 1e-9), max(dec_ms, 1e-9)
 
     tokens = wp.B * wp.T
     value = world * tokens / (pre_ms * 1e-3) / 1e6
