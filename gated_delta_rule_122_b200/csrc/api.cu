@@ -8,6 +8,8 @@
 
 namespace {
 
+constexpr size_t kKdaWorkspaceBytes = 16;   // device status word (+ padding)
+
 bool head_size_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 bool dtype_ok(kda_dtype t) { return t == KDA_F32 || t == KDA_BF16; }
 size_t dsize(kda_dtype t) { return t == KDA_BF16 ? 2 : 4; }
@@ -90,7 +92,18 @@ int kda_version(void) { return 100; }
 size_t kda_forward_workspace_bytes(int B, int T, int H, int d_k, int d_v)
 {
     (void)B; (void)T; (void)H; (void)d_k; (void)d_v;
-    return 0;
+    return kKdaWorkspaceBytes;
+}
+
+kda_status kda_workspace_status(const void *workspace, cudaStream_t stream)
+{
+    if (!workspace) return KDA_ERR_NULL;
+    if (!aligned16(workspace)) return KDA_ERR_ALIGN;
+    unsigned int word = 0;
+    if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+        return KDA_ERR_LAUNCH;
+    return word ? KDA_ERR_TIMEOUT : KDA_OK;
 }
 
 kda_status kda_forward(const void *q, const void *k, const void *v, const void *alpha,
@@ -102,12 +115,15 @@ kda_status kda_forward(const void *q, const void *k, const void *v, const void *
     kda_status st = check_forward(q, k, v, alpha, beta, initial_state, o, final_state, B, T, H,
                                   d_k, d_v, qkv_dtype, gate_dtype, out_dtype);
     if (st != KDA_OK) return st;
-    const size_t need = kda_forward_workspace_bytes(B, T, H, d_k, d_v);
-    if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
     if (B * (long long)H == 0) return KDA_OK;
+    const size_t need = kda_forward_workspace_bytes(B, T, H, d_k, d_v);
+    if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return KDA_ERR_ALIGN;
+    if (cudaMemsetAsync(workspace, 0, need, stream) != cudaSuccess) return KDA_ERR_LAUNCH;
     if (T == 0) return empty_sequence(initial_state, final_state, B, H, d_k, d_v, stream);
     kda::ChunkArgs a{q, k, v, alpha, beta, initial_state, final_state, o, B, T, H, scale,
-                     qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16};
+                     qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16,
+                     static_cast<unsigned int *>(workspace)};
     cudaError_t err;
     if (kda::chunk_tc_supported(d_k, d_v, qkv_dtype, gate_dtype))
         err = kda::launch_chunk_tc(a, d_k, d_v, stream);
@@ -128,7 +144,8 @@ kda_status kda_forward_sequential(const void *q, const void *k, const void *v, c
     if (B * (long long)H == 0) return KDA_OK;
     if (T == 0) return empty_sequence(initial_state, final_state, B, H, d_k, d_v, stream);
     kda::RecurrentArgs a{q, k, v, alpha, beta, initial_state, final_state, o, B, T, H, scale,
-                         qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16};
+                         qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16,
+                         nullptr};
     return kda::launch_recurrent(a, d_k, d_v, stream) == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
 }
 
@@ -144,7 +161,8 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const vo
     if (N * (long long)H == 0) return KDA_OK;
     // the state is read and rewritten in place; one token per sequence
     kda::RecurrentArgs a{q, k, v, alpha, beta, state, state, o, N, 1, H, scale,
-                         qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16};
+                         qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16,
+                         nullptr};
     return kda::launch_recurrent(a, d_k, d_v, stream) == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
 }
 

@@ -16,6 +16,7 @@ struct ChunkArgs {
     int B, T, H;
     float scale;
     int qkv_bf16, gate_bf16, out_bf16;
+    unsigned int *status;   // device status word (bit 0: a bounded wait timed out) or null
 };
 using RecurrentArgs = ChunkArgs;
 

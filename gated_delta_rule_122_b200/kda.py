@@ -23,8 +23,8 @@ _LIB_PATH = os.path.join(_HERE, "libkda_b200.so")
 _lib = None
 _lock = threading.Lock()
 
-EXPORTED_SYMBOLS = ("kda_forward", "kda_forward_workspace_bytes", "kda_forward_sequential",
-                    "kda_decode_step", "kda_status_string", "kda_version")
+EXPORTED_SYMBOLS = ("kda_forward", "kda_forward_workspace_bytes", "kda_workspace_status",
+                    "kda_forward_sequential", "kda_decode_step", "kda_status_string", "kda_version")
 
 _DT = {torch.float32: 0, torch.bfloat16: 1}
 _vp = ctypes.c_void_p
@@ -60,6 +60,8 @@ def library() -> ctypes.CDLL:
             lib.kda_forward_sequential.restype = _i
             lib.kda_forward_workspace_bytes.argtypes = [_i] * 5
             lib.kda_forward_workspace_bytes.restype = ctypes.c_size_t
+            lib.kda_workspace_status.argtypes = [_vp, _vp]
+            lib.kda_workspace_status.restype = _i
             lib.kda_decode_step.argtypes = [_vp] * 7 + [_i] * 4 + [_f] + [_i] * 3 + [_vp]
             lib.kda_decode_step.restype = _i
             lib.kda_status_string.argtypes = [_i]
@@ -104,7 +106,7 @@ def _to_device(tensors, device):
 
 
 def _prefill(fn_name, q, k, v, alpha, beta, initial_state, scale, output_final_state,
-             out_dtype, out, final_state):
+             out_dtype, out, final_state, workspace=None, check_status=False):
     host = q.device.type == "cpu"
     host_out = host_state = None
     if host:
@@ -152,8 +154,12 @@ def _prefill(fn_name, q, k, v, alpha, beta, initial_state, scale, output_final_s
         stream = _vp(_stream_handle(device))
         if fn_name == "kda_forward":
             ws_bytes = lib.kda_forward_workspace_bytes(B, T, H, dk, dv)
-            ws = torch.empty(ws_bytes, device=device, dtype=torch.uint8) if ws_bytes else None
-            code = lib.kda_forward(*args, _ptr(ws), ws_bytes, stream)
+            ws = workspace
+            if ws is None or ws.numel() * ws.element_size() < ws_bytes:
+                ws = torch.empty(max(ws_bytes, 16), device=device, dtype=torch.uint8)
+            code = lib.kda_forward(*args, _ptr(ws), ws.numel() * ws.element_size(), stream)
+            if code == 0 and check_status:
+                code = lib.kda_workspace_status(_ptr(ws), stream)
         else:
             code = lib.kda_forward_sequential(*args, stream)
     if code != 0:
@@ -174,15 +180,19 @@ def _prefill(fn_name, q, k, v, alpha, beta, initial_state, scale, output_final_s
 
 
 def forward(q, k, v, alpha, beta, initial_state=None, scale=None, output_final_state=True,
-            out_dtype=torch.float32, out=None, final_state=None):
+            out_dtype=torch.float32, out=None, final_state=None, workspace=None,
+            check_status=False):
     """Chunkwise KDA prefill (C entry point ``kda_forward``).
 
     q, k, alpha: [B,T,H,dk]; v: [B,T,H,dv]; beta: [B,T,H] (q/k/v share a dtype,
     alpha/beta share a dtype; float32 or bfloat16).  initial_state: float32
-    [B,H,dk,dv] or None.  Returns (o [B,T,H,dv] of out_dtype, final_state or None).
+    [B,H,dk,dv] or None.  workspace: optional device uint8 tensor of at least
+    ``kda_forward_workspace_bytes`` bytes (allocated per call when omitted).
+    check_status=True synchronizes and raises KDAError if a bounded device wait
+    timed out.  Returns (o [B,T,H,dv] of out_dtype, final_state or None).
     """
     return _prefill("kda_forward", q, k, v, alpha, beta, initial_state, scale,
-                    output_final_state, out_dtype, out, final_state)
+                    output_final_state, out_dtype, out, final_state, workspace, check_status)
 
 
 def forward_sequential(q, k, v, alpha, beta, initial_state=None, scale=None,

@@ -79,8 +79,12 @@ typedef enum {
  *   final_state   [B, H, d_k, d_v] fp32, may be NULL (not returned); may be
  *                 the same pointer as initial_state (continuation in place)
  *   scale         multiplies q at the read (callers usually pass d_k^-1/2)
- *   workspace     device scratch of kda_forward_workspace_bytes() bytes; may be
- *                 NULL when that size is 0
+ *   workspace     device scratch of at least kda_forward_workspace_bytes()
+ *                 bytes, 16-byte aligned, owned by the caller.  The call
+ *                 zeroes it on `stream` and the kernel records there whether a
+ *                 bounded device-side wait gave up; read it with
+ *                 kda_workspace_status().  Calls that share a workspace must
+ *                 not overlap on the GPU.
  * T = 0 copies initial_state (or zeros) to final_state.  o must not overlap
  * any input (KDA_ERR_ALIAS).  A last chunk shorter than the chunk size is
  * handled exactly (no padding of the caller's buffers is needed).
@@ -93,8 +97,19 @@ kda_status kda_forward(const void *q, const void *k, const void *v,
                        kda_dtype out_dtype, void *workspace,
                        size_t workspace_bytes, cudaStream_t stream);
 
-/* Bytes of device workspace kda_forward needs for these sizes (0 = none). */
+/* Bytes of device workspace kda_forward needs for these sizes (currently 16:
+ * one status word and padding, independent of the sizes). */
 size_t kda_forward_workspace_bytes(int B, int T, int H, int d_k, int d_v);
+
+/*
+ * kda_workspace_status -- synchronize `stream`, then read the status word a
+ * kda_forward call left in `workspace`: KDA_OK, or KDA_ERR_TIMEOUT when one of
+ * the kernel's bounded waits on its own tensor-core completions gave up (the
+ * outputs of that call are then not valid).  KDA_ERR_LAUNCH if the copy or the
+ * synchronization fails.  Not part of the recurrence; the pages have no
+ * counterpart.
+ */
+kda_status kda_workspace_status(const void *workspace, cudaStream_t stream);
 
 /*
  * kda_forward_sequential -- the same operation and arguments as kda_forward

@@ -47,7 +47,7 @@ def test_status_strings(lib):
 
 
 def _fwd(lib, q=0x10000, k=0x20000, v=0x30000, a=0x40000, b=0x50000, s0=None, o=0x60000,
-         s1=None, B=1, T=4, H=1, dk=16, dv=16, qkv=0, gate=0, out=0, ws=None, wsb=0):
+         s1=None, B=1, T=4, H=1, dk=16, dv=16, qkv=0, gate=0, out=0, ws=0x90000, wsb=16):
     return lib.kda_forward(q, k, v, a, b, s0, o, s1, B, T, H, dk, dv, 1.0, qkv, gate, out, ws, wsb,
                            None)
 
@@ -61,7 +61,10 @@ def test_forward_rejects_bad_arguments_before_launch(lib):
     assert _fwd(lib, k=0x20008) == ERR_ALIGN
     assert _fwd(lib, o=0x10000 + 64) == ERR_ALIAS          # o overlaps q
     assert _fwd(lib, B=0) == OK                             # nothing to do, nothing launched
-    assert _fwd(lib, H=0) == OK
+    assert _fwd(lib, H=0, ws=None) == OK
+    assert _fwd(lib, ws=None) == ERR_WS
+    assert _fwd(lib, wsb=8) == ERR_WS
+    assert _fwd(lib, ws=0x90008) == ERR_ALIGN
 
 
 def test_sequential_and_decode_reject_bad_arguments(lib):
@@ -80,7 +83,9 @@ def test_sequential_and_decode_reject_bad_arguments(lib):
 
 
 def test_workspace_query(lib):
-    assert lib.kda_forward_workspace_bytes(2, 8192, 64, 128, 128) >= 0
+    assert lib.kda_forward_workspace_bytes(2, 8192, 64, 128, 128) == 16
+    assert lib.kda_workspace_status(None, None) == ERR_NULL
+    assert lib.kda_workspace_status(0x90004, None) == ERR_ALIGN
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
