@@ -172,11 +172,8 @@ def dist_setup(n_gpus):
 
 
 def reduce_max(pg, values, device):
-    import torch
-    t = torch.tensor(values, dtype=torch.float64, device=device)
-    if pg is not None:
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-    return t.tolist()
+    from gated_delta_rule_122_b200.shard import max_over_ranks
+    return max_over_ranks(values, device=device)
 
 
 def barrier(pg):
@@ -261,9 +258,14 @@ def main():
     torch.cuda.set_device(device)
     peaks, peak_kind = load_peaks()
 
+    from gated_delta_rule_122_b200.shard import shard_bounds
     wp, wd = workload("prefill"), workload("decode")
-    x = make_inputs(wp, device=device)
-    y = make_decode_inputs(wd, device=device)
+    # the global batch is world x the workload's sequences; this rank's block of them
+    p0, p1 = shard_bounds(world * wp.B, rank, world)
+    d0, d1 = shard_bounds(world * wd.B, rank, world)
+    wp, wd = wp.scaled(B=p1 - p0), wd.scaled(B=d1 - d0)
+    x = make_inputs(wp, device=device, seed=wp.seed + p0)
+    y = make_decode_inputs(wd, device=device, seed=wd.seed + d0)
     o = torch.empty((wp.B, wp.T, wp.H, wp.dv), device=device, dtype=torch.float32)
     S = torch.empty((wp.B, wp.H, wp.dk, wp.dv), device=device, dtype=torch.float32)
     od = torch.empty((wd.B, wd.H, wd.dv), device=device, dtype=torch.float32)
