@@ -24,7 +24,8 @@ _lib = None
 _lock = threading.Lock()
 
 EXPORTED_SYMBOLS = ("kda_forward", "kda_forward_workspace_bytes", "kda_workspace_status",
-                    "kda_forward_sequential", "kda_decode_step", "kda_status_string", "kda_version")
+                    "kda_forward_noalloc", "kda_forward_sequential", "kda_decode_step",
+                    "kda_status_string", "kda_version")
 
 _DT = {torch.float32: 0, torch.bfloat16: 1}
 _vp = ctypes.c_void_p
@@ -58,6 +59,8 @@ def library() -> ctypes.CDLL:
             lib.kda_forward.restype = _i
             lib.kda_forward_sequential.argtypes = fwd_args + [_vp]
             lib.kda_forward_sequential.restype = _i
+            lib.kda_forward_noalloc.argtypes = fwd_args + [_vp]
+            lib.kda_forward_noalloc.restype = _i
             lib.kda_forward_workspace_bytes.argtypes = [_i] * 5
             lib.kda_forward_workspace_bytes.restype = ctypes.c_size_t
             lib.kda_workspace_status.argtypes = [_vp, _vp]

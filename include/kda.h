@@ -112,6 +112,27 @@ size_t kda_forward_workspace_bytes(int B, int T, int H, int d_k, int d_v);
 kda_status kda_workspace_status(const void *workspace, cudaStream_t stream);
 
 /*
+ * kda_forward_noalloc -- kda_forward for callers that cannot allocate device
+ * memory (an allocator-less runtime, a plugin that must not touch its host's
+ * memory pool, code without an allocation API at hand).  Same arguments and
+ * results as kda_forward, without the workspace: the library uses its own
+ * fixed device array of 256 bytes (held on every GPU that loads the library
+ * until the process exits) and returns KDA_ERR_WORKSPACE if a call would need
+ * more than that.  Nothing is allocated or freed.  Every call shares that
+ * array and clears it at its start, so calls that overlap on the GPU race:
+ * serialize them.  The first call on a device looks up the array's address
+ * (once per device, with that device current); make it before any stream
+ * capture.  The pages have no counterpart of this entry point.
+ */
+kda_status kda_forward_noalloc(const void *q, const void *k, const void *v,
+                               const void *alpha, const void *beta,
+                               const float *initial_state, void *o,
+                               float *final_state, int B, int T, int H,
+                               int d_k, int d_v, float scale,
+                               kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                               kda_dtype out_dtype, cudaStream_t stream);
+
+/*
  * kda_forward_sequential -- the same operation and arguments as kda_forward
  * (no workspace), computed with the token-by-token schedule ("fused
  * recurrent" in "Two schedules for the same recurrence", brain.bigb.es): one
