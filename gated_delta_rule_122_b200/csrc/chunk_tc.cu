@@ -10,9 +10,9 @@
 // Per chunk, with G[r] = sum_{t<=r} log alpha_t (per key channel), an anchor
 // a = G[15] in the middle of the chunk and e_r = exp(G_r - a):
 //   Lk = K*e, Lq = scale*Q*e, R = K/e            (bf16 hi/lo operands)
-//   [A_kk; A_qk]  = [Lk; Lq] R^T                 (M=64 N=32 K=128)
+//   [A_kk; A_qk]  = [Lk; Lq] R^T                 (one M=128 product over both planes)
 //   A_kk <- strict lower * beta_r,  A_qk <- lower incl. diagonal
-//   T'   = (I + A_kk)^-1 Diag(beta)              (blocked substitution, fp32)
+//   T'   = (I + A_kk)^-1 Diag(beta)              (substitution in one warp, fp32)
 //   W'^T = Lk^T T'^T,   U^T = V^T T'^T
 // The state is carried pre-scaled, S' = Diag(exp(a)) S, which makes W S = W' S'
 // and (scale Q gamma) S = Lq S' with gamma_r = exp(G_r) the pages' in-chunk
@@ -23,19 +23,22 @@
 //   S_next = Diag(exp(G_end - a)) X,  S'_next = Diag(exp(a_next)) S_next
 // since K*gamma_end/gamma = R Diag(exp(G_end - a)) and gamma_end = exp(a) *
 // exp(G_end - a).  The anchor bounds every operand by exp(16 tokens of decay);
-// products are the exact pairwise decays.
+// products are the exact pairwise decays.  e and 1/e are running products of
+// alpha away from the anchor row (no logarithms), floored at 2^-125.
 //
-// Precision: operands that are not exact bf16 inputs are split x = hi + lo.
-// Each product runs as two MMAs per K step, A_hi x [B_hi | B_lo] and
-// A_lo x [B_hi | B_lo], the B planes concatenated along N, so the accumulator
-// holds (hi + lo)(hi + lo) in two column groups summed when read.  Operands are
-// "plane-interleaved": each 8-row block keeps its hi core matrices followed by
-// its lo core matrices, so one buffer serves as a single-plane operand, as the
-// two planes concatenated along N, and (swapping the descriptor strides) as
-// the transposed operand.  The state update and all accumulations are fp32.
+// Precision: operands that are not exact bf16 inputs are split x = hi + lo and
+// every product sums all four hi/lo cross terms: the planes are either
+// concatenated along M or N of one MMA (summed when the accumulator is read)
+// or issued as two MMAs into the same accumulator.  The state update and all
+// accumulations are fp32.
 //
-// The serial products are computed transposed: value channel j is the MMA's M
-// index and TMEM lane; the fp32 state lives in TMEM.
+// Layouts.  Lk, Lq, R and -W' are stored "d-major": 2 KB slabs of 8 rows
+// (tokens) x 128 key channels, each 16-byte core-matrix row holding 8
+// consecutive tokens of one channel.  The same slab is a K-major operand when
+// channels index M/N (W', X products) and an MN-major operand when tokens do
+// (A products, the O/E product), and one thread per channel writes it with
+// 16-byte stores.  The serial products are computed transposed: value channel j
+// is the MMA's M index and TMEM lane; the fp32 state lives in TMEM.
 //
 // Algorithm: "Kimi Delta Attention (KDA)" (brain.bigb.es), "Two schedules for
 // the same recurrence"; "From Fast Weight Programmers to KDA"
@@ -60,14 +63,32 @@ constexpr int kIssuerWarp = NCW + NPW;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per bounded wait
 constexpr int kChainBar = 1, kPrepBar = 2;         // named barriers of the two roles
 constexpr int kCstSlots = 4;                       // per-chunk constants kept in flight
+constexpr float kMinAlpha = 1.8048513e-35f;        // e^-80: per-token retention floor
+constexpr float kMinScale = 2.3509887e-38f;        // 2^-125: floor of the anchored decays
 
-// ---- plane-interleaved K-major operand layout ------------------------------------
-// Row-block (row/8) of an operand with K columns is K*32 bytes: the hi plane's
-// K/8 core matrices (128 B each), then the lo plane's.  Element (row, k, plane):
-__device__ __forceinline__ uint32_t ipl(int row, int k, int plane, int K)
+// ---- operand layouts ----------------------------------------------------------------
+// d-major slab (8 tokens x 128 channels, 2 KB): channel block d/8 at 128 B, channel
+// d%8 at 16 B, token r%8 at 2 B.
+constexpr int SLAB = 2048;
+__device__ __forceinline__ uint32_t dm(int slab, int d, int r)
 {
-    return (uint32_t)((row >> 3) * (K * 32) + plane * (K * 16) + (k >> 3) * 128 + (row & 7) * 16 +
-                      (k & 7) * 2);
+    return (uint32_t)(slab * SLAB + (d >> 3) * 128 + (d & 7) * 16 + (r & 7) * 2);
+}
+// Slabs of one operand stage.  M=128 A-product operand = slabs 0..15, O/E product
+// operand = slabs 8..23, R = slabs 24..31 (token block rb, plane pl at 24 + 2rb + pl).
+constexpr int SL_LK_LO = 0, SL_LK_HI = 4, SL_LQ_HI = 8, SL_LQ_LO = 12, SL_W_HI = 16, SL_W_LO = 20, SL_R = 24;
+
+// Plane-major K-major operand with N = 32 rows per plane and K = 32 (T', A_qk):
+// row block (pl*4 + r/8) at 512 B, K block s/8 at 128 B.
+__device__ __forceinline__ uint32_t pm(int pl, int r, int s)
+{
+    return (uint32_t)((pl * 4 + (r >> 3)) * 512 + (s >> 3) * 128 + (r & 7) * 16 + (s & 7) * 2);
+}
+// Plane-interleaved K-major layout with K = 32 (E^T: rows j, K = s): row block j/8
+// holds the hi plane's 4 core matrices, then the lo plane's.
+__device__ __forceinline__ uint32_t ipl(int row, int k, int plane)
+{
+    return (uint32_t)((row >> 3) * (C * 32) + plane * (C * 16) + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2);
 }
 // Plain MN-major layout (V): core matrices (mn/8, k/8) at (mn/8)*(K/8)*128 + (k/8)*128.
 __device__ __forceinline__ uint32_t mnmaj(int mn, int k, int K)
@@ -76,36 +97,43 @@ __device__ __forceinline__ uint32_t mnmaj(int mn, int k, int K)
 }
 
 // ---- shared-memory plan (bytes) ----------------------------------------------------
-constexpr int ROWB = 272;                              // staged row: 256 B + 16 B pad
+// Staged row r of q, k, alpha at r*256 + (r/8)*32: the 32 B step per 8-row block
+// keeps the per-channel column reads free of bank conflicts.
+__device__ __forceinline__ int stg_row(int r) { return r * 256 + (r >> 3) * 32; }
+constexpr int STG_T = C * 256 + (C / 8) * 32;          // one staged tensor
 constexpr int OFF_STG = 0;                             // staged q, k, alpha of one chunk
-constexpr int STG_Q = 0, STG_K = C * ROWB, STG_A = 2 * C * ROWB;
-constexpr int OFF_V = OFF_STG + 3 * C * ROWB;          // 2 x V (A of U^T: M=j, K=s, MN-major)
+constexpr int STG_Q = 0, STG_K = STG_T, STG_A = 2 * STG_T;
+constexpr int OFF_V = OFF_STG + 3 * STG_T;             // 2 x V (A of U^T: M=j, K=s, MN-major)
 constexpr int V_BYTES = D * C * 2;
 constexpr int OFF_CST = OFF_V + 2 * V_BYTES;           // kCstSlots x {exp(a), exp(G_end - a), f}[128]
 constexpr int CST_BYTES = 3 * D * 4;                   // f(n) = exp(a_n) exp(G_end,n-1 - a_n-1)
-constexpr int OFF_BETA = OFF_CST + kCstSlots * CST_BYTES;   // 2 x beta[32]
-constexpr int OFF_LQR = OFF_BETA + 2 * C * 4;          // 2 stages: [Lk; Lq; -W'] rows 0..95, then R
-constexpr int LQ_BYTES = 3 * C * D * 4;                // 96 rows x 128 x 2 planes x 2 B
-constexpr int R_OFF = LQ_BYTES;
-constexpr int LQR_BYTES = LQ_BYTES + C * D * 4;
-constexpr int OFF_ET = OFF_LQR + 2 * LQR_BYTES;        // E^T (A of O/dS: rows j, K = s)
-constexpr int OFF_TP = OFF_ET + D * C * 4;             // T'  (B of W'/U: rows r, K = s)
-constexpr int OFF_AQ = OFF_TP + C * C * 4;             // 2 x A_qk (B of O: rows r, K = s)
+constexpr int OFF_LQR = (OFF_CST + kCstSlots * CST_BYTES + 127) / 128 * 128;   // 2 operand stages
+constexpr int LQR_BYTES = 32 * SLAB;
+constexpr int OFF_ET = OFF_LQR + 2 * LQR_BYTES;        // E^T (A of the O and X products)
+constexpr int OFF_TP = OFF_ET + D * C * 4;             // T'  (B of W'/U: N = r, K = s)
+constexpr int OFF_AQ = OFF_TP + C * C * 4;             // 2 x A_qk (B of O: N = r, K = s)
 constexpr int AQ_BYTES = C * C * 4;
-constexpr int OFF_AKK = OFF_AQ + 2 * AQ_BYTES;         // A_kk fp32 [C][C+1]
-constexpr int OFF_TS = OFF_AKK + C * (C + 1) * 4;      // T fp32 [C][C+1]
-constexpr int NBARS = 9;
-constexpr int OFF_BAR = OFF_TS + C * (C + 1) * 4;
-constexpr int OFF_MISC = OFF_BAR + NBARS * 8;          // tmem base, error flag
+constexpr int P = C + 1;                               // fp32 [32][33] tiles
+constexpr int OFF_PK = OFF_AQ + 2 * AQ_BYTES;          // partial A_kk (lo-plane rows)
+constexpr int OFF_PQ = OFF_PK + C * P * 4;             // partial A_qk (hi-plane rows)
+constexpr int OFF_AKK = OFF_PQ + C * P * 4;            // A_kk^T fp32 [32][36]
+constexpr int OFF_TS = OFF_AKK + C * (C + 4) * 4;      // T fp32 [32][33]
+constexpr int OFF_BETA = OFF_TS + C * P * 4;           // beta of the chunk being solved
+constexpr int NBARS = 4;
+constexpr int OFF_BAR = (OFF_BETA + C * 4 + 7) / 8 * 8;
+constexpr int OFF_SIG = OFF_BAR + NBARS * 8;           // 6 readiness counters
+constexpr int OFF_MISC = OFF_SIG + 32;                 // tmem base, error flag
 constexpr int SMEM_BYTES = OFF_MISC + 16;
+static_assert(SMEM_BYTES <= 232448, "shared memory plan exceeds the per-block limit");
+static_assert(OFF_AKK % 16 == 0 && OFF_LQR % 128 == 0, "vector and operand alignment");
 
 // TMEM columns
-constexpr uint32_t TM_A = 0;      // [A_kk; A_qk] (M=64 layout, N=64)
+constexpr uint32_t TM_A = 0;      // [A_kk; A_qk] partial products (M=128: 4 row groups, N=64)
 constexpr uint32_t TM_O = 64;     // O^T (64 cols: hi/lo groups), directly followed by
 constexpr uint32_t TM_E = 128;    // E^T (64 cols) so that one N=128 MMA writes both
 constexpr uint32_t TM_S = 192;    // fp32 S'^T, accumulated into X^T by the E^T R product
 constexpr uint32_t TM_SP = 320;   // S'^T hi (64 cols) and lo (64 cols), the A operand of M3
-constexpr uint32_t TM_W = 448;    // W'^T (N=64)
+constexpr uint32_t TM_W = 448;    // W'^T (N=64: T' hi rows, then lo rows)
 constexpr uint32_t TM_COLS = 512;
 
 // x = hi + lo with hi = x truncated to bf16 (exact) and lo = bf16(x - hi); the
@@ -120,7 +148,7 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t &hw, uin
     lw = *reinterpret_cast<const uint32_t *>(&lp);
 }
 
-// Store 8 values (consecutive k) as hi and lo 16-byte chunks; lo sits plane_gap after hi.
+// Store 8 values as hi and lo 16-byte chunks; lo sits plane_gap bytes after hi.
 __device__ __forceinline__ void st_split8(uint8_t *p, int plane_gap, const float (&x)[8])
 {
     uint4 h, l;
@@ -132,15 +160,9 @@ __device__ __forceinline__ void st_split8(uint8_t *p, int plane_gap, const float
     *reinterpret_cast<uint4 *>(p + plane_gap) = l;
 }
 
-__device__ __forceinline__ void ld_bf16x8(const uint8_t *p, float (&x)[8])
+__device__ __forceinline__ float ld_bf16(const uint8_t *p)
 {
-    union {
-        uint4 u;
-        __nv_bfloat16 b[8];
-    } v;
-    v.u = *reinterpret_cast<const uint4 *>(p);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) x[i] = __bfloat162float(v.b[i]);
+    return __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t *>(p)) << 16);
 }
 
 __device__ __forceinline__ void chain_bar() { ptx::named_bar_sync(kChainBar, NCT); }
@@ -153,205 +175,256 @@ __device__ __forceinline__ float load_beta(const ChunkArgs &p, int b, int h, int
     return __bfloat162float(((const __nv_bfloat16 *)p.beta)[((size_t)b * p.T + t) * p.H + h]);
 }
 
-// Every warp of a role arrives once (barrier count = the role's warps).
-__device__ __forceinline__ void warp_arrive(uint32_t bar, int lane)
+// Every warp of a role adds 1 to a readiness counter once its writes are visible
+// (the counter of chunk n's step reaches (n + 1) x the role's warps).
+__device__ __forceinline__ void warp_signal(uint32_t cnt, int lane)
 {
     __syncwarp();
-    if (lane == 0) ptx::mbar_arrive(bar);
+    if (lane == 0) ptx::red_add_release(cnt, 1u);
 }
 
 struct Bars {
-    uint32_t a, w, e, s;      // issuer -> warps (tcgen05.commit)
-    uint32_t rc, rs, re;      // chain -> issuer: operands staged, S' written, E^T written
-    uint32_t rg, rj;          // prep -> issuer: T' and A_qk written, -W' written
+    uint32_t a, w, e, s;      // issuer -> warps (mbarriers, tcgen05.commit)
+    uint32_t rc, rs, re;      // chain -> issuer counters: operands staged, S' written, E^T written
+    uint32_t ra, rg, rj;      // prep -> issuer counters: A read, T' and A_qk written, -W' written
 };
 
 // ---- the MMA-issuer warp (lane 0) -------------------------------------------------
 // Four MMA groups per chunk: M1 (A-products) and M2 (W', U) depend only on the
-// prep warps, M3 (O, E) and M4 (O, X) on the chain warps.  The issuer polls the
-// readiness barriers and issues whichever group is ready next, so neither role
-// waits behind the other's group.
+// prep warps, M3 (O, E) and M4 (O, X) on the chain warps.  The tensor pipe runs
+// them in issue order.  The issuer polls the readiness counters (plain shared
+// loads) and issues the most urgent ready group: the chain's M3 and M4 first,
+// then M2, then M1.
+struct MmaIds {
+    uint32_t A, W, U, OE, O2, dS;
+};
+
+__device__ __forceinline__ void issue_m3(uint8_t *sm, uint32_t tmem, const Bars &bars, const MmaIds &id, int n3)
+{
+    ptx::tc_fence_after();
+    const uint32_t b0 = ptx::smem_u32(sm + OFF_LQR + (n3 & 1) * LQR_BYTES) + SL_LQ_HI * SLAB;
+    for (int ks = 0; ks < D / 16; ++ks)
+        for (int pl = 0; pl < 2; ++pl)
+            ptx::mma_bf16_ts(tmem + TM_O, tmem + TM_SP + 64 * pl + 8 * ks,
+                             ptx::smem_desc(b0 + 256 * ks, 128, SLAB), id.OE, 1);
+    ptx::mma_commit(bars.e);
+}
+
+__device__ __forceinline__ void issue_m4(uint8_t *sm, uint32_t tmem, const Bars &bars, const MmaIds &id, int n4)
+{
+    ptx::tc_fence_after();
+    const uint32_t et = ptx::smem_u32(sm + OFF_ET);
+    const uint32_t aq = ptx::smem_u32(sm + OFF_AQ + (n4 & 1) * AQ_BYTES);
+    const uint32_t rr = ptx::smem_u32(sm + OFF_LQR + (n4 & 1) * LQR_BYTES) + SL_R * SLAB;
+    for (int ks = 0; ks < C / 16; ++ks)
+        for (int pl = 0; pl < 2; ++pl)
+            ptx::mma_bf16(tmem + TM_O, ptx::smem_desc(et + C * 16 * pl + 256 * ks, 128, C * 32),
+                          ptx::smem_desc(aq + 256 * ks, 128, 512), id.O2, 1);
+    for (int ks = 0; ks < C / 16; ++ks)
+        for (int pa = 0; pa < 2; ++pa)
+            for (int pb = 0; pb < 2; ++pb)
+                // R as the K-major (N = d, K = s) operand: token blocks 2 slabs apart
+                ptx::mma_bf16(tmem + TM_S, ptx::smem_desc(et + C * 16 * pa + 256 * ks, 128, C * 32),
+                              ptx::smem_desc(rr + SLAB * pb + 4 * SLAB * ks, 2 * SLAB, 128), id.dS, 1);
+    ptx::mma_commit(bars.s);
+}
+
+__device__ __forceinline__ void issue_m1(uint8_t *sm, uint32_t tmem, const Bars &bars, const MmaIds &id, int n1)
+{
+    ptx::tc_fence_after();
+    const uint32_t base = ptx::smem_u32(sm + OFF_LQR + (n1 & 1) * LQR_BYTES);
+    for (int ks = 0; ks < D / 16; ++ks)
+        ptx::mma_bf16(tmem + TM_A, ptx::smem_desc(base + SL_LK_LO * SLAB + 256 * ks, 128, SLAB),
+                      ptx::smem_desc(base + SL_R * SLAB + 256 * ks, 128, SLAB), id.A, ks > 0);
+    ptx::mma_commit(bars.a);
+}
+
+__device__ __forceinline__ void issue_m2(uint8_t *sm, uint32_t tmem, const Bars &bars, const MmaIds &id, int n2)
+{
+    ptx::tc_fence_after();
+    const uint32_t base = ptx::smem_u32(sm + OFF_LQR + (n2 & 1) * LQR_BYTES);
+    const uint32_t tp = ptx::smem_u32(sm + OFF_TP);
+    const uint32_t vv = ptx::smem_u32(sm + OFF_V + (n2 & 1) * V_BYTES);
+    for (int ks = 0; ks < C / 16; ++ks)
+        for (int pl = 0; pl < 2; ++pl)
+            // Lk as the K-major (M = d, K = s) operand
+            ptx::mma_bf16(tmem + TM_W,
+                          ptx::smem_desc(base + (pl ? SL_LK_LO : SL_LK_HI) * SLAB + 2 * SLAB * ks, SLAB, 128),
+                          ptx::smem_desc(tp + 256 * ks, 128, 512), id.W, ks > 0 || pl > 0);
+    for (int ks = 0; ks < C / 16; ++ks)
+        ptx::mma_bf16(tmem + TM_E, ptx::smem_desc(vv + 256 * ks, 128, (C / 8) * 128),
+                      ptx::smem_desc(tp + 256 * ks, 128, 512), id.U, ks > 0);
+    ptx::mma_commit(bars.w);
+}
+
+// Readiness of each group: M1(n) needs Lk, Lq, R of chunk n (rc) and A(n-1) read
+// (ra); M2(n) needs T' and A_qk (rg; the prep warps signal it after reading
+// W'(n-1)) and M4(n-1) issued, since U goes into TM_E; M3(n) needs S'(n) (rs,
+// whose first count is the initial state) and -W'(n) (rj); M4(n) needs E^T(n) (re).
 __device__ void issuer(uint8_t *sm, uint32_t tmem, const Bars &bars, int nchunks, volatile int *err_flag)
 {
-    const uint32_t id_A = ptx::idesc_bf16(64, 64, 0, 0, 0);      // [Lk;Lq] x [R_hi|R_lo]
-    const uint32_t id_W = ptx::idesc_bf16(128, 64, 1, 0, 0);     // Lk^T (MN view) x T'
-    const uint32_t id_OE = ptx::idesc_bf16(128, 128, 0, 0, 0);   // S' x [Lq | -W']
-    const uint32_t id_O2 = ptx::idesc_bf16(128, 64, 0, 0, 0);    // E^T x A_qk
-    const uint32_t id_dS = ptx::idesc_bf16(128, 128, 0, 1, 0);   // E^T x R (MN view)
+    MmaIds id;
+    id.A = ptx::idesc_bf16(128, 64, 1, 1, 0);     // [Lk; Lq] (MN) x R (MN)
+    id.W = ptx::idesc_bf16(128, 64, 0, 0, 0);     // Lk (d x s) x T'
+    id.U = ptx::idesc_bf16(128, 64, 1, 0, 0);     // V (MN) x T'
+    id.OE = ptx::idesc_bf16(128, 128, 0, 1, 0);   // S' (TMEM) x [Lq | -W'] (MN)
+    id.O2 = ptx::idesc_bf16(128, 64, 0, 0, 0);    // E^T x A_qk
+    id.dS = ptx::idesc_bf16(128, 128, 0, 0, 0);   // E^T x R (d x s)
     int n1 = 0, n2 = 0, n3 = 0, n4 = 0;   // next chunk of each group
-    uint64_t t_idle = ptx::global_timer_ns();
+    uint32_t idle = 0;                     // polls since the last issue
+    uint64_t t_idle = 0;
     while (n4 < nchunks) {
-        bool issued = false;
-        // M3(n3): needs S'(n3) (rs), W'(n3) (rj, also implies Lq(n3)), U(n3) (M2 issued)
-        if (n3 < n2 && n3 <= n4 && ptx::mbar_test_wait(bars.rs, (uint32_t)(n3 & 1)) &&
-            ptx::mbar_test_wait(bars.rj, (uint32_t)(n3 & 1))) {
-            ptx::tc_fence_after();
-            const uint32_t b0 = ptx::smem_u32(sm + OFF_LQR + (n3 & 1) * LQR_BYTES) + 4 * D * 32;
-            for (int ks = 0; ks < D / 16; ++ks)
-                for (int pl = 0; pl < 2; ++pl)
-                    ptx::mma_bf16_ts(tmem + TM_O, tmem + TM_SP + 64 * pl + 8 * ks,
-                                     ptx::smem_desc(b0 + 256 * ks, 128, D * 16), id_OE, 1);
-            ptx::mma_commit(bars.e);
-            ++n3;
-            issued = true;
-        }
-        // M4(n4): needs E^T(n4) (re)
-        if (n4 < n3 && ptx::mbar_test_wait(bars.re, (uint32_t)(n4 & 1))) {
-            ptx::tc_fence_after();
-            const uint32_t et = ptx::smem_u32(sm + OFF_ET);
-            const uint32_t aq = ptx::smem_u32(sm + OFF_AQ + (n4 & 1) * AQ_BYTES);
-            const uint32_t rr = ptx::smem_u32(sm + OFF_LQR + (n4 & 1) * LQR_BYTES) + R_OFF;
-            for (int ks = 0; ks < C / 16; ++ks)
-                for (int pl = 0; pl < 2; ++pl)
-                    ptx::mma_bf16(tmem + TM_O, ptx::smem_desc(et + C * 16 * pl + 256 * ks, 128, C * 32),
-                                  ptx::smem_desc(aq + 256 * ks, 128, C * 16), id_O2, 1);
-            for (int ks = 0; ks < C / 16; ++ks)
-                for (int pa = 0; pa < 2; ++pa)
-                    for (int pb = 0; pb < 2; ++pb)
-                        // R as the MN-major (N = d, K = s) operand: d-blocks 128 B apart,
-                        // s-blocks (row-blocks) D*32 B apart
-                        ptx::mma_bf16(tmem + TM_S,
-                                      ptx::smem_desc(et + C * 16 * pa + 256 * ks, 128, C * 32),
-                                      ptx::smem_desc(rr + D * 16 * pb + 2 * D * 32 * ks, D * 32, 128),
-                                      id_dS, 1);
-            ptx::mma_commit(bars.s);
-            ++n4;
-            issued = true;
-        }
-        // M1(n1): needs Lk, Lq, R of chunk n1 (rc; the prep warps read A(n1-1) before that)
-        if (n1 < nchunks && n1 == n2 && ptx::mbar_test_wait(bars.rc, (uint32_t)(n1 & 1))) {
-            ptx::tc_fence_after();
-            const uint32_t lq = ptx::smem_u32(sm + OFF_LQR + (n1 & 1) * LQR_BYTES);
-            const uint32_t rr = lq + R_OFF;
-            uint32_t acc = 0;
-            for (int ks = 0; ks < D / 16; ++ks)
-                for (int pl = 0; pl < 2; ++pl) {
-                    ptx::mma_bf16(tmem + TM_A, ptx::smem_desc(lq + D * 16 * pl + 256 * ks, 128, D * 32),
-                                  ptx::smem_desc(rr + 256 * ks, 128, D * 16), id_A, acc);
-                    acc = 1;
-                }
-            ptx::mma_commit(bars.a);
-            ++n1;
-            issued = true;
-        }
-        // M2(n2): needs T', A_qk of chunk n2 (rg; the prep warps read W'(n2-1) before that);
-        // writes U into TM_E, so E(n2-1) must be consumed (M4(n2-1) issued)
-        if (n2 < n1 && n2 <= n4 && ptx::mbar_test_wait(bars.rg, (uint32_t)(n2 & 1))) {
-            ptx::tc_fence_after();
-            const uint32_t lk = ptx::smem_u32(sm + OFF_LQR + (n2 & 1) * LQR_BYTES);
-            const uint32_t tp = ptx::smem_u32(sm + OFF_TP);
-            const uint32_t vv = ptx::smem_u32(sm + OFF_V + (n2 & 1) * V_BYTES);
-            uint32_t acc = 0;
-            for (int ks = 0; ks < C / 16; ++ks)
-                for (int pl = 0; pl < 2; ++pl) {
-                    // Lk as the MN-major (M = d, K = s) operand
-                    ptx::mma_bf16(tmem + TM_W,
-                                  ptx::smem_desc(lk + D * 16 * pl + 2 * D * 32 * ks, D * 32, 128),
-                                  ptx::smem_desc(tp + 256 * ks, 128, C * 16), id_W, acc);
-                    acc = 1;
-                }
-            for (int ks = 0; ks < C / 16; ++ks)
-                ptx::mma_bf16(tmem + TM_E, ptx::smem_desc(vv + 256 * ks, 128, (C / 8) * 128),
-                              ptx::smem_desc(tp + 256 * ks, 128, C * 16), id_W, ks > 0);
-            ptx::mma_commit(bars.w);
-            ++n2;
-            issued = true;
-        }
-        if (issued) {
-            t_idle = ptx::global_timer_ns();
-        } else {
-            if (ptx::global_timer_ns() - t_idle > kWaitLimitNs || *err_flag) {
+        const uint32_t c_rs = ptx::ld_relaxed(bars.rs), c_rj = ptx::ld_relaxed(bars.rj);
+        const uint32_t c_re = ptx::ld_relaxed(bars.re), c_rg = ptx::ld_relaxed(bars.rg);
+        const uint32_t c_rc = ptx::ld_relaxed(bars.rc), c_ra = ptx::ld_relaxed(bars.ra);
+        int g = 0;
+        if (n3 < n2 && n3 <= n4 && c_rs >= (uint32_t)(NCW * (n3 + 1)) && c_rj >= (uint32_t)(NPW * (n3 + 1)))
+            g = 3;
+        else if (n4 < n3 && c_re >= (uint32_t)(NCW * (n4 + 1)))
+            g = 4;
+        else if (n2 < n1 && n2 <= n4 && c_rg >= (uint32_t)(NPW * (n2 + 1)))
+            g = 2;
+        else if (n1 < nchunks && c_ra >= (uint32_t)(NPW * n1) && c_rc >= (uint32_t)(NCW * (n1 + 1)))
+            g = 1;
+        if (g != 0) {
+            // acquire the producers' writes (the counters only grow)
+            if (g == 3) { (void)ptx::ld_acquire(bars.rs); (void)ptx::ld_acquire(bars.rj); }
+            else if (g == 4) (void)ptx::ld_acquire(bars.re);
+            else if (g == 2) (void)ptx::ld_acquire(bars.rg);
+            else { (void)ptx::ld_acquire(bars.ra); (void)ptx::ld_acquire(bars.rc); }
+            if (g == 3) issue_m3(sm, tmem, bars, id, n3++);
+            else if (g == 4) issue_m4(sm, tmem, bars, id, n4++);
+            else if (g == 2) issue_m2(sm, tmem, bars, id, n2++);
+            else issue_m1(sm, tmem, bars, id, n1++);
+            idle = 0;
+        } else if ((++idle & 1023u) == 0) {
+            // nothing ready for a while: check the time limit and the error flag
+            const uint64_t now = ptx::global_timer_ns();
+            if (idle == 1024u) t_idle = now;
+            if (now - t_idle > kWaitLimitNs || *err_flag) {
                 *err_flag = 1;
                 return;
             }
-            __nanosleep(32);   // nothing ready: leave the issue slots to the compute warps
+        } else {
+            __nanosleep(20);
         }
     }
 }
 
-// ---- T' = (I + A_kk)^-1 Diag(beta) in one warp ---------------------------------------
-// Lane c computes column c of T by right-looking forward substitution: once t_k
-// is final, every later row's partial sum takes its A[i][k] t_k term, so the
-// dependent chain is one FMA per row; A[i][k] are broadcast shared-memory reads.
-// The column is transposed through shared memory and written as the K-major
-// plane-interleaved B operand of M2 (rows r, K = s).
-__device__ void solve_warp(const float *A, float *Ts, const float *sbeta, uint8_t *tp, int lane)
+// ---- T' = (I + A_kk)^-1 Diag(beta), blocked over the four prep warps -------------
+// With A = [[A00, 0], [A10, A11]] in 16x16 blocks, (I + A)^-1 = [[T0, 0],
+// [-T1 A10 T0, T1]] with T0 = (I + A00)^-1 and T1 = (I + A11)^-1.  One warp
+// computes T0 (lanes 0-15) and T1 (lanes 16-31) at once, lane = column, by
+// right-looking forward substitution; A is stored transposed (At[k][i]) so a
+// column is read as broadcast 16-byte loads.  All four warps then form
+// X = A10 T0 and T10 = -T1 X, two entries per thread, and write T' = T Diag(beta)
+// as the plane-major K-major B operand of M2 (rows r, K = s).
+constexpr int PT = C + 4;   // row pitch of At (16-byte aligned rows)
+__device__ __forceinline__ void solve_diag_blocks(const float *At, float *Tm, int lane)
 {
-    constexpr int P = C + 1;
-    float t[C];
+    const int c = lane & 15, off = lane & 16;
+    float t[16];
 #pragma unroll
-    for (int i = 0; i < C; ++i) t[i] = (i == lane) ? 1.f : 0.f;
+    for (int i = 0; i < 16; ++i) t[i] = (i == c) ? 1.f : 0.f;
 #pragma unroll
-    for (int k = 0; k < C; ++k) {
+    for (int k = 0; k < 15; ++k) {
         const float tk = t[k];
 #pragma unroll
-        for (int i = k + 1; i < C; ++i) t[i] = fmaf(-A[i * P + k], tk, t[i]);
+        for (int i4 = (k + 1) / 4; i4 < 4; ++i4) {
+            const float4 a = *reinterpret_cast<const float4 *>(At + (off + k) * PT + off + 4 * i4);
+            if (4 * i4 + 0 > k) t[4 * i4 + 0] = fmaf(-a.x, tk, t[4 * i4 + 0]);
+            if (4 * i4 + 1 > k) t[4 * i4 + 1] = fmaf(-a.y, tk, t[4 * i4 + 1]);
+            if (4 * i4 + 2 > k) t[4 * i4 + 2] = fmaf(-a.z, tk, t[4 * i4 + 2]);
+            if (4 * i4 + 3 > k) t[4 * i4 + 3] = fmaf(-a.w, tk, t[4 * i4 + 3]);
+        }
     }
-    const float bc = sbeta[lane];
 #pragma unroll
-    for (int r = 0; r < C; ++r) Ts[r * P + lane] = t[r] * bc;
-    __syncwarp();
-#pragma unroll
-    for (int sc = 0; sc < 4; ++sc) {
-        float x[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) x[i] = Ts[lane * P + 8 * sc + i];
-        st_split8(tp + ipl(lane, 8 * sc, 0, C), C * 16, x);
-    }
+    for (int i = 0; i < 16; ++i) Tm[(off + i) * P + off + c] = t[i];
 }
 
-// ---- operand preparation of chunk n (chain warps, between two state updates) -------
-// Row r = lane, key channels 8g..8g+7 for g = warp, warp + 8: the prefix sum of
-// log2 alpha over the chunk (a warp scan over rows), the anchored decays, the
-// bf16 hi/lo operands Lk, Lq, R, and the chunk's per-channel constants.
-__device__ void stage_operands(const ChunkArgs &p, uint8_t *sm, int n, int warp, int lane)
+// ---- operand preparation of chunk n (chain warps) -----------------------------------
+// Thread (warp w, lane): token rows 8q..8q+7 with q = lane/8, key channels
+// 16w + lane%8 and 16w + lane%8 + 8.  Away from the anchor row 15 the decays are
+// running products of alpha: for r >= 16, e_r = prod_{16..r} alpha; for r < 16,
+// 1/e_r = prod_{r+1..15} alpha.  The four row quarters exchange their block
+// products with shuffles.  Part A writes Lk, Lq and the chunk constants and
+// returns 1/e; part B writes R = K/e.  Part A only touches slabs the A product
+// (M1), the W'/U product (M2) and the O/E product (M3) of the chunk two back have
+// finished with, so it can run while that chunk's state update (M4) still reads R.
+__device__ void stage_a(const ChunkArgs &p, uint8_t *sm, int n, int warp, int lane, float (&ie)[16])
 {
-    const int r = lane;
+    const int q = lane >> 3, dl = lane & 7;
     const int Lc = min(C, p.T - n * C);
     uint8_t *lqr = sm + OFF_LQR + (n & 1) * LQR_BYTES;
     float *cst = reinterpret_cast<float *>(sm + OFF_CST + (n % kCstSlots) * CST_BYTES);
     const float *cst_prev = reinterpret_cast<const float *>(sm + OFF_CST + ((n + kCstSlots - 1) % kCstSlots) * CST_BYTES);
-#pragma unroll 1
-    for (int gi = 0; gi < 2; ++gi) {
-        const int g = warp + NCW * gi;        // key channels 8g .. 8g+7
-        float q8[8], k8[8], x[8];
-        ld_bf16x8(sm + OFF_STG + STG_Q + r * ROWB + g * 16, q8);
-        ld_bf16x8(sm + OFF_STG + STG_K + r * ROWB + g * 16, k8);
-        ld_bf16x8(sm + OFF_STG + STG_A + r * ROWB + g * 16, x);
-        // base-2 log of the retention, floored at 2^-115.4 (= e^-80); rows past the
-        // end are identity steps
+    const uint8_t *stg = sm + OFF_STG;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) x[i] = (r < Lc) ? fmaxf(ptx::lg2(x[i]), -115.4f) : 0.f;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float y = __shfl_up_sync(0xffffffffu, x[i], off);
-                if (lane >= off) x[i] += y;
-            }
-        }
-        float lk[8], lq[8], rk[8], my_a = 0.f, my_gl = 0.f;
+    for (int ch = 0; ch < 2; ++ch) {
+        const int d = 16 * warp + 8 * ch + dl;
+        float al[8], pr[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const float a = __shfl_sync(0xffffffffu, x[i], 15);
-            const float gl = __shfl_sync(0xffffffffu, x[i], 31);
-            if (lane == i) { my_a = a; my_gl = gl; }
-            const float t = fminf(fmaxf(x[i] - a, -125.f), 125.f);
-            const float e = ptx::ex2(t), re = ptx::ex2(-t);
-            lk[i] = k8[i] * e;
-            lq[i] = p.scale * q8[i] * e;
-            rk[i] = k8[i] * re;
+            const int r = 8 * q + i;
+            const float x = ld_bf16(stg + STG_A + stg_row(r) + 2 * d);
+            al[i] = (r < Lc) ? fmaxf(x, kMinAlpha) : 1.f;   // rows past the end: identity steps
         }
-        if (lane < 8) {
-            const int d = 8 * g + lane;
-            const float aexp = ptx::ex2(fmaxf(my_a, -125.f));
-            cst[d] = aexp;                                                     // exp(a)
-            cst[D + d] = ptx::ex2(fminf(fmaxf(my_gl - my_a, -125.f), 125.f));  // exp(G_end - a)
-            cst[2 * D + d] = (n > 0) ? aexp * cst_prev[D + d] : 0.f;           // state-update factor
+        // within-quarter products: forward for rows >= 16, backward (exclusive) for rows < 16
+        float blk;
+        if (q >= 2) {
+            float acc = 1.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) { acc *= al[i]; pr[i] = acc; }
+            blk = acc;
+        } else {
+            float acc = 1.f;
+#pragma unroll
+            for (int i = 7; i >= 0; --i) { pr[i] = acc; acc *= al[i]; }
+            blk = acc;
         }
-        st_split8(lqr + ipl(r, 8 * g, 0, D), D * 16, lk);
-        st_split8(lqr + ipl(C + r, 8 * g, 0, D), D * 16, lq);
-        st_split8(lqr + R_OFF + ipl(r, 8 * g, 0, D), D * 16, rk);
+        const float blk_dn8 = __shfl_down_sync(0xffffffffu, blk, 8);    // quarter q+1
+        const float blk_up8 = __shfl_up_sync(0xffffffffu, blk, 8);      // quarter q-1
+        const float blk_dn16 = __shfl_down_sync(0xffffffffu, blk, 16);  // quarter q+2
+        const float blk_dn24 = __shfl_down_sync(0xffffffffu, blk, 24);  // quarter q+3
+        const float carry = (q == 0) ? blk_dn8 : (q == 3) ? blk_up8 : 1.f;
+        if (q == 0) {
+            // exp(a) = prod over rows 0..15, exp(G_end - a) = prod over rows 16..31
+            const float aexp = fmaxf(blk * blk_dn8, kMinScale);
+            const float cend = fmaxf(blk_dn16 * blk_dn24, kMinScale);
+            cst[d] = aexp;
+            cst[D + d] = cend;
+            cst[2 * D + d] = (n > 0) ? aexp * cst_prev[D + d] : 0.f;   // state-update factor
+        }
+        float lk[8], lq[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int r = 8 * q + i;
+            const float m = fminf(fmaxf(pr[i] * carry, kMinScale), 1.f / kMinScale);
+            const float rm = ptx::rcp(m);
+            const float e = (q >= 2) ? m : rm;
+            ie[8 * ch + i] = (q >= 2) ? rm : m;
+            const float kv = ld_bf16(stg + STG_K + stg_row(r) + 2 * d);
+            const float qv = ld_bf16(stg + STG_Q + stg_row(r) + 2 * d);
+            lk[i] = kv * e;
+            lq[i] = p.scale * qv * e;
+        }
+        st_split8(lqr + dm(SL_LK_HI + q, d, 0), (SL_LK_LO - SL_LK_HI) * SLAB, lk);
+        st_split8(lqr + dm(SL_LQ_HI + q, d, 0), (SL_LQ_LO - SL_LQ_HI) * SLAB, lq);
+    }
+}
+
+__device__ void stage_b(uint8_t *sm, int n, int warp, int lane, const float (&ie)[16])
+{
+    const int q = lane >> 3, dl = lane & 7;
+    uint8_t *lqr = sm + OFF_LQR + (n & 1) * LQR_BYTES;
+    const uint8_t *stg = sm + OFF_STG;
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch) {
+        const int d = 16 * warp + 8 * ch + dl;
+        float rk[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) rk[i] = ld_bf16(stg + STG_K + stg_row(8 * q + i) + 2 * d) * ie[8 * ch + i];
+        st_split8(lqr + dm(SL_R + 2 * q, d, 0), SLAB, rk);
     }
 }
 
@@ -373,7 +446,7 @@ __device__ void prefetch_qka(const ChunkArgs &p, uint8_t *sm, int b, int h, int 
         const void *src = tensor == 0 ? (const void *)((const __nv_bfloat16 *)p.q + g)
                         : tensor == 1 ? (const void *)((const __nv_bfloat16 *)p.k + g)
                                       : (const void *)((const __nv_bfloat16 *)p.alpha + g);
-        ptx::cp_async16(ptx::smem_u32(sm + OFF_STG + tensor * C * ROWB + r * ROWB + ch * 16), src, nbytes);
+        ptx::cp_async16(ptx::smem_u32(sm + OFF_STG + tensor * STG_T + stg_row(r) + ch * 16), src, nbytes);
     }
     ptx::cp_async_commit();
 }
@@ -398,98 +471,142 @@ __device__ void prefetch_v(const ChunkArgs &p, uint8_t *sm, int b, int h, int n,
 }
 
 // ---- the prep warps: A readout, the solve, W' readout, V loads ---------------------
+// The A product's four row groups (TMEM lane quadrants) are Lk_lo, Lk_hi, Lq_hi and
+// Lq_lo times R: warps 0 and 2 hand their partial sums to warps 1 and 3 through
+// shared memory; warp 1 forms A_kk and solves its diagonal blocks, warp 3 writes
+// A_qk, and all four finish the off-diagonal block of T and write T'.
 __device__ void prep_role(const ChunkArgs &p, uint8_t *sm, uint32_t tmem, const Bars &bars, int b, int h,
                           int nchunks, volatile int *err_flag)
 {
     const int pt = threadIdx.x - NCT;          // 0..127
     const int pw = pt >> 5, lane = pt & 31;    // warp = TMEM lane quadrant
     const uint32_t lane_base = (uint32_t)(pw * 32) << 16;
-    float *Akk = reinterpret_cast<float *>(sm + OFF_AKK);
-    float *Ts = reinterpret_cast<float *>(sm + OFF_TS);
-    float *sbeta_all = reinterpret_cast<float *>(sm + OFF_BETA);
+    float *PK = reinterpret_cast<float *>(sm + OFF_PK);
+    float *PQ = reinterpret_cast<float *>(sm + OFF_PQ);
+    float *At = reinterpret_cast<float *>(sm + OFF_AKK);   // A_kk transposed
+    float *Tm = reinterpret_cast<float *>(sm + OFF_TS);    // T = (I + A_kk)^-1
+    float *Xs = PK;                                        // A10 T0 (PK is consumed by then)
+    float *sbeta = reinterpret_cast<float *>(sm + OFF_BETA);
 
     prefetch_v(p, sm, b, h, 0, pt);
     if (nchunks > 1) prefetch_v(p, sm, b, h, 1, pt);
-    if (pw == 0) sbeta_all[lane] = load_beta(p, b, h, 0, lane);
-    prep_bar();
+    float beta = (pw == 1) ? load_beta(p, b, h, 0, lane) : 0.f;   // beta of row / column `lane`
 
     for (int cn = 0; cn < nchunks; ++cn) {
-        const float *sbeta = sbeta_all + (cn & 1) * C;
-        // beta of the next chunk, stored once this chunk's A readout is done (warp 0
-        // ran the solve of chunk cn-1 that read the same slot)
-        const float beta_next = (pw == 0 && cn + 1 < nchunks) ? load_beta(p, b, h, cn + 1, lane) : 0.f;
+        const float beta_next = (pw == 1 && cn + 1 < nchunks) ? load_beta(p, b, h, cn + 1, lane) : 0.f;
 
-        // ---- G(cn): A_kk / A_qk from TMEM; the solve in warp 0; T'
+        // ---- G(cn): A_kk / A_qk from TMEM; the solve; T'
         if (!ptx::mbar_wait(bars.a, (uint32_t)(cn & 1), kWaitLimitNs)) *err_flag = 1;
         ptx::tc_fence_after();
-#pragma unroll 1
+        float a32[32];   // this row group's products with R, summed over R's planes
+#pragma unroll
         for (int hs = 0; hs < 2; ++hs) {
             float v[32];
             ptx::tmem_ld32(tmem + lane_base + TM_A + 32 * hs, v);
             ptx::tmem_wait_ld();
-            if (lane < 16) {
-                const int row = 16 * pw + lane;   // M=64 rows sit in lanes 0-15 of each quadrant
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int sb = 2 * hs + u;       // s = 8sb .. 8sb+7
-                    if (row < C) {
-                        const float br = sbeta[row];
+            for (int u = 0; u < 2; ++u)
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const int s = 8 * sb + i;
-                            Akk[row * (C + 1) + s] = (s < row) ? br * (v[16 * u + i] + v[16 * u + 8 + i]) : 0.f;
-                        }
-                    } else {
-                        const int r = row - C;
-                        float x[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            x[i] = (8 * sb + i <= r) ? v[16 * u + i] + v[16 * u + 8 + i] : 0.f;
-                        st_split8(sm + OFF_AQ + (cn & 1) * AQ_BYTES + ipl(r, 8 * sb, 0, C), C * 16, x);
-                    }
-                }
-            }
+                for (int i = 0; i < 8; ++i) a32[16 * hs + 8 * u + i] = v[16 * u + i] + v[16 * u + 8 + i];
         }
-        if (pw == 0) sbeta_all[((cn + 1) & 1) * C + lane] = beta_next;
+        ptx::tc_fence_before();
+        warp_signal(bars.ra, lane);
+        if (pw == 0 || pw == 2) {
+            float *dst = (pw == 0 ? PK : PQ) + lane * P;
+#pragma unroll
+            for (int s = 0; s < C; ++s) dst[s] = a32[s];
+        }
         ptx::cp_async_wait_all();            // V(cn) (and V(cn+1)) have landed
         ptx::fence_proxy_async_smem();
-        ptx::tc_fence_before();
         prep_bar();
-        if (pw == 0) {
-            solve_warp(Akk, Ts, sbeta, sm + OFF_TP, lane);
+        if (pw == 1) {
+            // A_kk^T (row `lane` of A_kk scaled by beta_lane, strictly lower)
+            const float *src = PK + lane * P;
+#pragma unroll
+            for (int s = 0; s < C; ++s) At[s * PT + lane] = (s < lane) ? beta * (a32[s] + src[s]) : 0.f;
+            sbeta[lane] = beta;
+        } else if (pw == 3) {
+            const float *src = PQ + lane * P;
+            uint8_t *aq = sm + OFF_AQ + (cn & 1) * AQ_BYTES;
+#pragma unroll
+            for (int sb = 0; sb < 4; ++sb) {
+                float x[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int s = 8 * sb + i;
+                    x[i] = (s <= lane) ? a32[s] + src[s] : 0.f;
+                }
+                st_split8(aq + pm(0, lane, 8 * sb), 4 * 512, x);
+            }
             ptx::fence_proxy_async_smem();
-            warp_arrive(bars.rg, lane);
         }
+        prep_bar();
+        if (pw == 1) solve_diag_blocks(At, Tm, lane);
+        prep_bar();
+        {
+            // X = A10 T0 (rows 16..31 of A, columns 0..15), two columns per thread
+            const int i = pt >> 3, c0 = 2 * (pt & 7);
+            float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float a = At[k * PT + 16 + i];
+                x0 = fmaf(a, Tm[k * P + c0], x0);
+                x1 = fmaf(a, Tm[k * P + c0 + 1], x1);
+            }
+            Xs[i * P + c0] = x0;
+            Xs[i * P + c0 + 1] = x1;
+            prep_bar();
+            // T10 = -T1 X (T1 is lower triangular, stored with zeros above its diagonal)
+            float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float t1 = Tm[(16 + i) * P + 16 + k];
+                y0 = fmaf(t1, Xs[k * P + c0], y0);
+                y1 = fmaf(t1, Xs[k * P + c0 + 1], y1);
+            }
+            Tm[(16 + i) * P + c0] = -y0;
+            Tm[(16 + i) * P + c0 + 1] = -y1;
+        }
+        prep_bar();
+        {
+            // T' = T Diag(beta): row r, columns 8sc..8sc+7, as hi/lo planes
+            const int r = 8 * pw + (lane & 7), sc = lane >> 3;
+            float x[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int s = 8 * sc + i;
+                x[i] = (r < 16 && s >= 16) ? 0.f : Tm[r * P + s] * sbeta[s];
+            }
+            st_split8(sm + OFF_TP + pm(0, r, 8 * sc), 4 * 512, x);
+            ptx::fence_proxy_async_smem();
+        }
+        warp_signal(bars.rg, lane);
+        beta = beta_next;
 
-        // ---- J(cn): -W' from TMEM (lanes = key channel d) into rows 64..95 of the operand
+        // ---- J(cn): -W' from TMEM (lanes = key channel d) into the W' slabs
         if (!ptx::mbar_wait(bars.w, (uint32_t)(cn & 1), kWaitLimitNs)) *err_flag = 1;
         ptx::tc_fence_after();
         {
             uint8_t *lqr = sm + OFF_LQR + (cn & 1) * LQR_BYTES;
             const int d = 32 * pw + lane;
-#pragma unroll 1
+#pragma unroll
             for (int hs = 0; hs < 2; ++hs) {
-                float v[32];
-                ptx::tmem_ld32(tmem + lane_base + TM_W + 32 * hs, v);
+                float vh[16], vl[16];
+                ptx::tmem_ld16(tmem + lane_base + TM_W + 16 * hs, vh);        // T' hi rows
+                ptx::tmem_ld16(tmem + lane_base + TM_W + 32 + 16 * hs, vl);   // T' lo rows
                 ptx::tmem_wait_ld();
 #pragma unroll
-                for (int u = 0; u < 2; ++u)
+                for (int u = 0; u < 2; ++u) {
+                    float x[8];
 #pragma unroll
-                    for (int i = 0; i < 8; i += 2) {
-                        uint32_t hw, lw;
-                        split_pair(-(v[16 * u + i] + v[16 * u + 8 + i]), -(v[16 * u + i + 1] + v[16 * u + 9 + i]), hw, lw);
-                        const int r = 16 * hs + 8 * u + i;
-                        const uint32_t off0 = ipl(2 * C + r, d, 0, D), off1 = ipl(2 * C + r + 1, d, 0, D);
-                        *reinterpret_cast<uint16_t *>(lqr + off0) = (uint16_t)(hw & 0xFFFFu);
-                        *reinterpret_cast<uint16_t *>(lqr + off1) = (uint16_t)(hw >> 16);
-                        *reinterpret_cast<uint16_t *>(lqr + off0 + D * 16) = (uint16_t)(lw & 0xFFFFu);
-                        *reinterpret_cast<uint16_t *>(lqr + off1 + D * 16) = (uint16_t)(lw >> 16);
-                    }
+                    for (int i = 0; i < 8; ++i) x[i] = -(vh[8 * u + i] + vl[8 * u + i]);
+                    st_split8(lqr + dm(SL_W_HI + 2 * hs + u, d, 0), (SL_W_LO - SL_W_HI) * SLAB, x);
+                }
             }
         }
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
-        warp_arrive(bars.rj, lane);
+        warp_signal(bars.rj, lane);
         // M2(cn) has completed: its V buffer can take chunk cn+2
         if (cn + 2 < nchunks) prefetch_v(p, sm, b, h, cn + 2, pt);
         if (*err_flag) break;
@@ -516,16 +633,23 @@ __device__ __forceinline__ void write_state16(uint32_t tmem, uint32_t lane_base,
     ptx::tmem_st8(tmem + lane_base + TM_SP + 64 + d0 / 2, lw);
 }
 
-// Chain warps: stage chunk n's operands (staging must hold chunk n) and signal the
-// issuer; then start loading chunk n+1 into the staging rows.
-__device__ void chain_prepare(const ChunkArgs &p, uint8_t *sm, const Bars &bars, int b, int h, int n,
-                              int nchunks, int tid, int warp, int lane)
+// Chain warps, operands of chunk n (the staging rows must hold chunk n): part A,
+// then (later) part B, the signal to the issuer and the loads of chunk n+1.
+__device__ __forceinline__ void chain_stage_a(const ChunkArgs &p, uint8_t *sm, int n, int warp, int lane,
+                                              float (&ie)[16])
 {
     ptx::cp_async_wait_all();
-    chain_bar();
-    stage_operands(p, sm, n, warp, lane);
+    chain_bar();   // every thread's copies of chunk n have landed
+    stage_a(p, sm, n, warp, lane, ie);
+}
+
+__device__ __forceinline__ void chain_stage_b(const ChunkArgs &p, uint8_t *sm, const Bars &bars, int b, int h,
+                                              int n, int nchunks, int tid, int warp, int lane,
+                                              const float (&ie)[16])
+{
+    stage_b(sm, n, warp, lane, ie);
     ptx::fence_proxy_async_smem();
-    warp_arrive(bars.rc, lane);
+    warp_signal(bars.rc, lane);
     chain_bar();   // staging consumed, constants visible to every chain warp
     if (n + 1 < nchunks) prefetch_qka(p, sm, b, h, n + 1, tid);
 }
@@ -541,8 +665,10 @@ __device__ void chain_role(const ChunkArgs &p, uint8_t *sm, uint32_t tmem, const
     const int j = quad * 32 + lane;            // value channel = TMEM lane
     const size_t tile = (size_t)bh * D * D;
 
+    float ie[16];   // 1/e of the chunk being staged, carried from part A to part B
     prefetch_qka(p, sm, b, h, 0, tid);
-    chain_prepare(p, sm, bars, b, h, 0, nchunks, tid, warp, lane);
+    chain_stage_a(p, sm, 0, warp, lane, ie);
+    chain_stage_b(p, sm, bars, b, h, 0, nchunks, tid, warp, lane, ie);
 
     // S'_0 = Diag(exp(a_0)) S_0; cleared O accumulator
     {
@@ -555,52 +681,57 @@ __device__ void chain_role(const ChunkArgs &p, uint8_t *sm, uint32_t tmem, const
             for (int i = 0; i < 16; ++i) v[i] = p.s_in ? p.s_in[tile + (size_t)(d0 + i) * D + j] : 0.f;
             write_state16(tmem, lane_base, d0, v, cst0 + d0);
         }
-        ptx::tmem_st16_zero(tmem + lane_base + TM_O + 32 * half);
-        ptx::tmem_st16_zero(tmem + lane_base + TM_O + 32 * half + 16);
+        ptx::tmem_st16_zero(tmem + lane_base + TM_O + 16 * half);
+        ptx::tmem_st16_zero(tmem + lane_base + TM_O + 32 + 16 * half);
         ptx::tmem_wait_st();
     }
     ptx::tc_fence_before();
-    warp_arrive(bars.rs, lane);
-    if (nchunks > 1) chain_prepare(p, sm, bars, b, h, 1, nchunks, tid, warp, lane);
+    warp_signal(bars.rs, lane);
+    if (nchunks > 1) {
+        chain_stage_a(p, sm, 1, warp, lane, ie);
+        chain_stage_b(p, sm, bars, b, h, 1, nchunks, tid, warp, lane, ie);
+    }
 
     for (int c = 0; c < nchunks; ++c) {
-        // ---- E: E^T = U^T - S'^T W'^T (hi and lo groups) into the A operand of M4
+        // ---- E: E^T = U^T - S'^T W'^T (hi and lo column groups) into the A operand of M4
         if (!ptx::mbar_wait(bars.e, (uint32_t)(c & 1), kWaitLimitNs)) *err_flag = 1;
         ptx::tc_fence_after();
         {
-            float v[32];
-            ptx::tmem_ld32(tmem + lane_base + TM_E + 32 * half, v);
+            float vh[16], vl[16];
+            ptx::tmem_ld16(tmem + lane_base + TM_E + 16 * half, vh);
+            ptx::tmem_ld16(tmem + lane_base + TM_E + 32 + 16 * half, vl);
             ptx::tmem_wait_ld();
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 float e8[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) e8[i] = v[16 * u + i] + v[16 * u + 8 + i];
-                st_split8(sm + OFF_ET + ipl(j, 8 * (2 * half + u), 0, C), C * 16, e8);
+                for (int i = 0; i < 8; ++i) e8[i] = vh[8 * u + i] + vl[8 * u + i];
+                st_split8(sm + OFF_ET + ipl(j, 16 * half + 8 * u, 0), C * 16, e8);
             }
         }
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
-        warp_arrive(bars.re, lane);
+        warp_signal(bars.re, lane);
+        // Lk, Lq of chunk c+2 while the state update of chunk c runs
+        if (c + 2 < nchunks) chain_stage_a(p, sm, c + 2, warp, lane, ie);
 
         // ---- I: X = S' + E^T R -> the next S' (or the final state); outputs of chunk c
         if (!ptx::mbar_wait(bars.s, (uint32_t)(c & 1), kWaitLimitNs)) *err_flag = 1;
         ptx::tc_fence_after();
         float ov[16];
         {
-            float v[32];
-            ptx::tmem_ld32(tmem + lane_base + TM_O + 32 * half, v);
+            float vh[16], vl[16];
+            ptx::tmem_ld16(tmem + lane_base + TM_O + 16 * half, vh);
+            ptx::tmem_ld16(tmem + lane_base + TM_O + 32 + 16 * half, vl);
             ptx::tmem_wait_ld();
 #pragma unroll
-            for (int u = 0; u < 2; ++u)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) ov[8 * u + i] = v[16 * u + i] + v[16 * u + 8 + i];
+            for (int i = 0; i < 16; ++i) ov[i] = vh[i] + vl[i];
         }
         if (c + 1 < nchunks) {
             // f(c+1) = exp(a_{c+1}) exp(G_end,c - a_c), written when chunk c+1 was staged
             const float *f = reinterpret_cast<const float *>(sm + OFF_CST + ((c + 1) % kCstSlots) * CST_BYTES) + 2 * D;
-            ptx::tmem_st16_zero(tmem + lane_base + TM_O + 32 * half);
-            ptx::tmem_st16_zero(tmem + lane_base + TM_O + 32 * half + 16);
+            ptx::tmem_st16_zero(tmem + lane_base + TM_O + 16 * half);
+            ptx::tmem_st16_zero(tmem + lane_base + TM_O + 32 + 16 * half);
 #pragma unroll 1
             for (int part = 0; part < 4; ++part) {
                 const int d0 = 64 * half + 16 * part;
@@ -611,7 +742,7 @@ __device__ void chain_role(const ChunkArgs &p, uint8_t *sm, uint32_t tmem, const
             }
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
-            warp_arrive(bars.rs, lane);
+            warp_signal(bars.rs, lane);
         } else if (p.s_out) {
             const float *cend = reinterpret_cast<const float *>(sm + OFF_CST + (c % kCstSlots) * CST_BYTES) + D;
 #pragma unroll 1
@@ -624,6 +755,8 @@ __device__ void chain_role(const ChunkArgs &p, uint8_t *sm, uint32_t tmem, const
                 for (int i = 0; i < 16; ++i) p.s_out[tile + (size_t)(d0 + i) * D + j] = cend[d0 + i] * v[i];
             }
         }
+        // R of chunk c+2 (the update of chunk c has read R(c)), then the outputs of chunk c
+        if (c + 2 < nchunks) chain_stage_b(p, sm, bars, b, h, c + 2, nchunks, tid, warp, lane, ie);
         {
             const int t0 = c * C;
             const size_t step = (size_t)p.H * D;
@@ -632,8 +765,6 @@ __device__ void chain_role(const ChunkArgs &p, uint8_t *sm, uint32_t tmem, const
             for (int i = 0; i < 16; ++i, idx += step)
                 if (t0 + 16 * half + i < p.T) st_elem(p.o, idx, ov[i], p.out_bf16);
         }
-        // ---- operands of chunk c+2 (its operand stage held chunk c, whose MMAs are done)
-        if (c + 2 < nchunks) chain_prepare(p, sm, bars, b, h, c + 2, nchunks, tid, warp, lane);
         if (*err_flag) break;
     }
     ptx::cp_async_wait_all();
@@ -653,20 +784,18 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs p)
     const uint32_t bar0 = ptx::smem_u32(sm + OFF_BAR);
     Bars bars;
     bars.a = bar0; bars.w = bar0 + 8; bars.e = bar0 + 16; bars.s = bar0 + 24;
-    bars.rc = bar0 + 32; bars.rg = bar0 + 40; bars.rj = bar0 + 48;
-    bars.rs = bar0 + 56; bars.re = bar0 + 64;
+    const uint32_t sig0 = ptx::smem_u32(sm + OFF_SIG);
+    bars.rc = sig0; bars.rs = sig0 + 4; bars.re = sig0 + 8;
+    bars.ra = sig0 + 12; bars.rg = sig0 + 16; bars.rj = sig0 + 20;
 
     if (tid == 0) {
         ptx::mbar_init(bars.a, 1);
         ptx::mbar_init(bars.w, 1);
         ptx::mbar_init(bars.e, 1);
         ptx::mbar_init(bars.s, 1);
-        ptx::mbar_init(bars.rc, NCW);
-        ptx::mbar_init(bars.rg, 1);
-        ptx::mbar_init(bars.rj, NPW);
-        ptx::mbar_init(bars.rs, NCW);
-        ptx::mbar_init(bars.re, NCW);
         ptx::fence_mbar_init();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) reinterpret_cast<uint32_t *>(sm + OFF_SIG)[i] = 0u;
         *err_flag = 0;
     }
     if (warp == 0) {

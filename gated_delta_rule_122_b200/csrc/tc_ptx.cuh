@@ -58,17 +58,11 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
-// Hardware base-2 exponential and logarithm (approximate, flush-to-zero).
-__device__ __forceinline__ float ex2(float x)
+// Hardware reciprocal (approximate, flush-to-zero; about 1 ulp).
+__device__ __forceinline__ float rcp(float x)
 {
     float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-__device__ __forceinline__ float lg2(float x)
-{
-    float y;
-    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
 
@@ -103,6 +97,26 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
 __device__ __forceinline__ void mbar_arrive(uint32_t bar)
 {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Monotonic shared-memory counters as a cheap producer -> consumer signal: the
+// producer adds with release semantics; the consumer polls with relaxed loads and,
+// once it has seen the count it needs, re-reads that counter with acquire semantics.
+__device__ __forceinline__ void red_add_release(uint32_t addr, uint32_t v)
+{
+    asm volatile("red.release.cta.shared::cta.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_relaxed(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.relaxed.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_acquire(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
 }
 
 // Named barrier over the first `nthreads` threads of the block (id 1..15).
