@@ -43,7 +43,11 @@
 // Algorithm: "Kimi Delta Attention (KDA)" (brain.bigb.es), "Two schedules for
 // the same recurrence"; "From Fast Weight Programmers to KDA"
 // (jonahsamost.bearblog.dev), section "Kimi Delta Attention".
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -97,10 +101,9 @@ __device__ __forceinline__ uint32_t mnmaj(int mn, int k, int K)
 }
 
 // ---- shared-memory plan (bytes) ----------------------------------------------------
-// Staged row r of q, k, alpha at r*256 + (r/8)*32: the 32 B step per 8-row block
-// keeps the per-channel column reads free of bank conflicts.
-__device__ __forceinline__ int stg_row(int r) { return r * 256 + (r >> 3) * 32; }
-constexpr int STG_T = C * 256 + (C / 8) * 32;          // one staged tensor
+// q, k, alpha of one chunk are staged as dense 256-byte rows (one TMA box each).
+__device__ __forceinline__ int stg_row(int r) { return r * 256; }
+constexpr int STG_T = C * 256;                         // one staged tensor
 constexpr int OFF_STG = 0;                             // staged q, k, alpha of one chunk
 constexpr int STG_Q = 0, STG_K = STG_T, STG_A = 2 * STG_T;
 constexpr int OFF_V = OFF_STG + 3 * STG_T;             // 2 x V (A of U^T: M=j, K=s, MN-major)
@@ -119,7 +122,7 @@ constexpr int OFF_PQ = OFF_PK + C * P * 4;             // partial A_qk (hi-plane
 constexpr int OFF_AKK = OFF_PQ + C * P * 4;            // A_kk^T fp32 [32][36]
 constexpr int OFF_TS = OFF_AKK + C * (C + 4) * 4;      // T fp32 [32][33]
 constexpr int OFF_BETA = OFF_TS + C * P * 4;           // beta of the chunk being solved
-constexpr int NBARS = 4;
+constexpr int NBARS = 7;
 constexpr int OFF_BAR = (OFF_BETA + C * 4 + 7) / 8 * 8;
 constexpr int OFF_SIG = OFF_BAR + NBARS * 8;           // 6 readiness counters
 constexpr int OFF_MISC = OFF_SIG + 32;                 // tmem base, error flag
@@ -175,6 +178,13 @@ __device__ __forceinline__ float load_beta(const ChunkArgs &p, int b, int h, int
     return __bfloat162float(((const __nv_bfloat16 *)p.beta)[((size_t)b * p.T + t) * p.H + h]);
 }
 
+// TMA descriptors of one launch: q, k, alpha as [B][T][H][128] boxes of 32 token
+// rows; v as the 5-D view (j%8, t, j/8, h, b) whose 8 x 32 x 16 box lands in the
+// MN-major core-matrix layout of the U^T product.
+struct TcMaps {
+    CUtensorMap q, k, a, v;
+};
+
 // Every warp of a role adds 1 to a readiness counter once its writes are visible
 // (the counter of chunk n's step reaches (n + 1) x the role's warps).
 __device__ __forceinline__ void warp_signal(uint32_t cnt, int lane)
@@ -185,6 +195,7 @@ __device__ __forceinline__ void warp_signal(uint32_t cnt, int lane)
 
 struct Bars {
     uint32_t a, w, e, s;      // issuer -> warps (mbarriers, tcgen05.commit)
+    uint32_t stg, v;          // TMA fills: q/k/alpha staging; V buffers (v and v + 8)
     uint32_t rc, rs, re;      // chain -> issuer counters: operands staged, S' written, E^T written
     uint32_t ra, rg, rj;      // prep -> issuer counters: A read, T' and A_qk written, -W' written
 };
@@ -343,131 +354,94 @@ __device__ __forceinline__ void solve_diag_blocks(const float *At, float *Tm, in
 }
 
 // ---- operand preparation of chunk n (chain warps) -----------------------------------
-// Thread (warp w, lane): token rows 8q..8q+7 with q = lane/8, key channels
-// 16w + lane%8 and 16w + lane%8 + 8.  Away from the anchor row 15 the decays are
-// running products of alpha: for r >= 16, e_r = prod_{16..r} alpha; for r < 16,
-// 1/e_r = prod_{r+1..15} alpha.  The four row quarters exchange their block
-// products with shuffles.  Part A writes Lk, Lq and the chunk constants and
-// returns 1/e; part B writes R = K/e.  Part A only touches slabs the A product
-// (M1), the W'/U product (M2) and the O/E product (M3) of the chunk two back have
-// finished with, so it can run while that chunk's state update (M4) still reads R.
+// Thread (warp w, lane): key channel d = 32(w%4) + lane, token rows 16h..16h+15
+// with h = w/4.  Away from the anchor row 15 the decays are running products of
+// alpha: for r >= 16, e_r = prod_{16..r} alpha; for r < 16, 1/e_r =
+// prod_{r+1..15} alpha, so each half of the chunk is self-contained.  Part A
+// writes Lk, Lq and the chunk constants and returns 1/e; part B writes R = K/e.
+// Part A only touches slabs the A product (M1), the W'/U product (M2) and the O/E
+// product (M3) of the chunk two back have finished with, so it can run while that
+// chunk's state update (M4) still reads R.
 __device__ void stage_a(const ChunkArgs &p, uint8_t *sm, int n, int warp, int lane, float (&ie)[16])
 {
-    const int q = lane >> 3, dl = lane & 7;
+    const int hf = warp >> 2, d = 32 * (warp & 3) + lane;
     const int Lc = min(C, p.T - n * C);
     uint8_t *lqr = sm + OFF_LQR + (n & 1) * LQR_BYTES;
     float *cst = reinterpret_cast<float *>(sm + OFF_CST + (n % kCstSlots) * CST_BYTES);
     const float *cst_prev = reinterpret_cast<const float *>(sm + OFF_CST + ((n + kCstSlots - 1) % kCstSlots) * CST_BYTES);
     const uint8_t *stg = sm + OFF_STG;
+    float pr[16];
+    float acc = 1.f;
+    if (hf == 1) {
 #pragma unroll
-    for (int ch = 0; ch < 2; ++ch) {
-        const int d = 16 * warp + 8 * ch + dl;
-        float al[8], pr[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int r = 8 * q + i;
+        for (int i = 0; i < 16; ++i) {
+            const int r = 16 + i;
             const float x = ld_bf16(stg + STG_A + stg_row(r) + 2 * d);
-            al[i] = (r < Lc) ? fmaxf(x, kMinAlpha) : 1.f;   // rows past the end: identity steps
+            acc *= (r < Lc) ? fmaxf(x, kMinAlpha) : 1.f;   // rows past the end: identity steps
+            pr[i] = acc;                                     // e_r
         }
-        // within-quarter products: forward for rows >= 16, backward (exclusive) for rows < 16
-        float blk;
-        if (q >= 2) {
-            float acc = 1.f;
+        cst[D + d] = fmaxf(acc, kMinScale);                 // exp(G_end - a)
+    } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) { acc *= al[i]; pr[i] = acc; }
-            blk = acc;
-        } else {
-            float acc = 1.f;
+        for (int i = 15; i >= 0; --i) {
+            pr[i] = acc;                                     // 1/e_r
+            const float x = ld_bf16(stg + STG_A + stg_row(i) + 2 * d);
+            acc *= (i < Lc) ? fmaxf(x, kMinAlpha) : 1.f;
+        }
+        const float aexp = fmaxf(acc, kMinScale);           // exp(a)
+        cst[d] = aexp;
+        cst[2 * D + d] = (n > 0) ? aexp * cst_prev[D + d] : 0.f;   // state-update factor
+    }
 #pragma unroll
-            for (int i = 7; i >= 0; --i) { pr[i] = acc; acc *= al[i]; }
-            blk = acc;
-        }
-        const float blk_dn8 = __shfl_down_sync(0xffffffffu, blk, 8);    // quarter q+1
-        const float blk_up8 = __shfl_up_sync(0xffffffffu, blk, 8);      // quarter q-1
-        const float blk_dn16 = __shfl_down_sync(0xffffffffu, blk, 16);  // quarter q+2
-        const float blk_dn24 = __shfl_down_sync(0xffffffffu, blk, 24);  // quarter q+3
-        const float carry = (q == 0) ? blk_dn8 : (q == 3) ? blk_up8 : 1.f;
-        if (q == 0) {
-            // exp(a) = prod over rows 0..15, exp(G_end - a) = prod over rows 16..31
-            const float aexp = fmaxf(blk * blk_dn8, kMinScale);
-            const float cend = fmaxf(blk_dn16 * blk_dn24, kMinScale);
-            cst[d] = aexp;
-            cst[D + d] = cend;
-            cst[2 * D + d] = (n > 0) ? aexp * cst_prev[D + d] : 0.f;   // state-update factor
-        }
+    for (int u = 0; u < 2; ++u) {
         float lk[8], lq[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const int r = 8 * q + i;
-            const float m = fminf(fmaxf(pr[i] * carry, kMinScale), 1.f / kMinScale);
+            const int r = 16 * hf + 8 * u + i;
+            const float m = fminf(fmaxf(pr[8 * u + i], kMinScale), 1.f / kMinScale);
             const float rm = ptx::rcp(m);
-            const float e = (q >= 2) ? m : rm;
-            ie[8 * ch + i] = (q >= 2) ? rm : m;
+            const float e = hf ? m : rm;
+            ie[8 * u + i] = hf ? rm : m;
             const float kv = ld_bf16(stg + STG_K + stg_row(r) + 2 * d);
             const float qv = ld_bf16(stg + STG_Q + stg_row(r) + 2 * d);
             lk[i] = kv * e;
             lq[i] = p.scale * qv * e;
         }
-        st_split8(lqr + dm(SL_LK_HI + q, d, 0), (SL_LK_LO - SL_LK_HI) * SLAB, lk);
-        st_split8(lqr + dm(SL_LQ_HI + q, d, 0), (SL_LQ_LO - SL_LQ_HI) * SLAB, lq);
+        st_split8(lqr + dm(SL_LK_HI + 2 * hf + u, d, 0), (SL_LK_LO - SL_LK_HI) * SLAB, lk);
+        st_split8(lqr + dm(SL_LQ_HI + 2 * hf + u, d, 0), (SL_LQ_LO - SL_LQ_HI) * SLAB, lq);
     }
 }
 
 __device__ void stage_b(uint8_t *sm, int n, int warp, int lane, const float (&ie)[16])
 {
-    const int q = lane >> 3, dl = lane & 7;
+    const int hf = warp >> 2, d = 32 * (warp & 3) + lane;
     uint8_t *lqr = sm + OFF_LQR + (n & 1) * LQR_BYTES;
     const uint8_t *stg = sm + OFF_STG;
 #pragma unroll
-    for (int ch = 0; ch < 2; ++ch) {
-        const int d = 16 * warp + 8 * ch + dl;
+    for (int u = 0; u < 2; ++u) {
         float rk[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) rk[i] = ld_bf16(stg + STG_K + stg_row(8 * q + i) + 2 * d) * ie[8 * ch + i];
-        st_split8(lqr + dm(SL_R + 2 * q, d, 0), SLAB, rk);
+        for (int i = 0; i < 8; ++i) rk[i] = ld_bf16(stg + STG_K + stg_row(16 * hf + 8 * u + i) + 2 * d) * ie[8 * u + i];
+        st_split8(lqr + dm(SL_R + 2 * (2 * hf + u), d, 0), SLAB, rk);
     }
 }
 
-// cp.async copies of chunk n's q, k, alpha rows into the staging rows (chain warps).
-__device__ void prefetch_qka(const ChunkArgs &p, uint8_t *sm, int b, int h, int n, int ct)
+// TMA loads of chunk n's q, k, alpha rows into the staging rows (one thread).
+__device__ __forceinline__ void load_qka(const TcMaps &maps, uint8_t *sm, const Bars &bars, int b, int h, int n)
 {
-    const int t0 = n * C;
-    const int L = min(C, p.T - t0);
-    const size_t HD = (size_t)p.H * D;
-#pragma unroll
-    for (int it = 0; it < 6; ++it) {
-        const int idx = ct + it * NCT;          // 0..1535; tensor = it / 2
-        const int rem = idx & 511;
-        const int r = rem >> 4, ch = rem & 15;
-        const int rr = r < L ? r : 0;
-        const uint32_t nbytes = r < L ? 16u : 0u;
-        const size_t g = ((size_t)b * p.T + t0 + rr) * HD + (size_t)h * D + ch * 8;
-        const int tensor = it >> 1;
-        const void *src = tensor == 0 ? (const void *)((const __nv_bfloat16 *)p.q + g)
-                        : tensor == 1 ? (const void *)((const __nv_bfloat16 *)p.k + g)
-                                      : (const void *)((const __nv_bfloat16 *)p.alpha + g);
-        ptx::cp_async16(ptx::smem_u32(sm + OFF_STG + tensor * STG_T + stg_row(r) + ch * 16), src, nbytes);
-    }
-    ptx::cp_async_commit();
+    ptx::mbar_arrive_expect_tx(bars.stg, 3 * STG_T);
+    const uint32_t dst = ptx::smem_u32(sm + OFF_STG);
+    ptx::tma_load_4d(dst + STG_Q, &maps.q, bars.stg, 0, h, n * C, b);
+    ptx::tma_load_4d(dst + STG_K, &maps.k, bars.stg, 0, h, n * C, b);
+    ptx::tma_load_4d(dst + STG_A, &maps.a, bars.stg, 0, h, n * C, b);
 }
 
-// cp.async copies of chunk n's v rows into V buffer n&1, MN-major (prep warps).
-__device__ void prefetch_v(const ChunkArgs &p, uint8_t *sm, int b, int h, int n, int pt)
+// TMA load of chunk n's v rows into V buffer n&1 (one thread).
+__device__ __forceinline__ void load_v(const TcMaps &maps, uint8_t *sm, const Bars &bars, int b, int h, int n)
 {
-    const int t0 = n * C;
-    const int L = min(C, p.T - t0);
-    const size_t HD = (size_t)p.H * D;
-    uint8_t *vb = sm + OFF_V + (n & 1) * V_BYTES;
-#pragma unroll
-    for (int it = 0; it < 4; ++it) {
-        const int rem = pt + it * NPT;          // 0..511
-        const int r = rem >> 4, ch = rem & 15;
-        const int rr = r < L ? r : 0;
-        const size_t g = ((size_t)b * p.T + t0 + rr) * HD + (size_t)h * D + ch * 8;
-        ptx::cp_async16(ptx::smem_u32(vb + mnmaj(ch * 8, r, C)), (const __nv_bfloat16 *)p.v + g,
-                        r < L ? 16u : 0u);
-    }
-    ptx::cp_async_commit();
+    const uint32_t bar = bars.v + 8 * (n & 1);
+    ptx::mbar_arrive_expect_tx(bar, V_BYTES);
+    ptx::tma_load_5d(ptx::smem_u32(sm + OFF_V + (n & 1) * V_BYTES), &maps.v, bar, 0, n * C, 0, h, b);
 }
 
 // ---- the prep warps: A readout, the solve, W' readout, V loads ---------------------
@@ -475,8 +449,8 @@ __device__ void prefetch_v(const ChunkArgs &p, uint8_t *sm, int b, int h, int n,
 // Lq_lo times R: warps 0 and 2 hand their partial sums to warps 1 and 3 through
 // shared memory; warp 1 forms A_kk and solves its diagonal blocks, warp 3 writes
 // A_qk, and all four finish the off-diagonal block of T and write T'.
-__device__ void prep_role(const ChunkArgs &p, uint8_t *sm, uint32_t tmem, const Bars &bars, int b, int h,
-                          int nchunks, volatile int *err_flag)
+__device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, uint32_t tmem, const Bars &bars,
+                          int b, int h, int nchunks, volatile int *err_flag)
 {
     const int pt = threadIdx.x - NCT;          // 0..127
     const int pw = pt >> 5, lane = pt & 31;    // warp = TMEM lane quadrant
@@ -488,8 +462,12 @@ __device__ void prep_role(const ChunkArgs &p, uint8_t *sm, uint32_t tmem, const 
     float *Xs = PK;                                        // A10 T0 (PK is consumed by then)
     float *sbeta = reinterpret_cast<float *>(sm + OFF_BETA);
 
-    prefetch_v(p, sm, b, h, 0, pt);
-    if (nchunks > 1) prefetch_v(p, sm, b, h, 1, pt);
+    int v_loaded = 0, v_seen = 0;   // V loads issued (thread pt 0) and waited for
+    if (pt == 0) {
+        load_v(maps, sm, bars, b, h, 0);
+        if (nchunks > 1) load_v(maps, sm, bars, b, h, 1);
+    }
+    v_loaded = nchunks > 1 ? 2 : 1;
     float beta = (pw == 1) ? load_beta(p, b, h, 0, lane) : 0.f;   // beta of row / column `lane`
 
     for (int cn = 0; cn < nchunks; ++cn) {
@@ -516,8 +494,9 @@ __device__ void prep_role(const ChunkArgs &p, uint8_t *sm, uint32_t tmem, const 
 #pragma unroll
             for (int s = 0; s < C; ++s) dst[s] = a32[s];
         }
-        ptx::cp_async_wait_all();            // V(cn) (and V(cn+1)) have landed
-        ptx::fence_proxy_async_smem();
+        // V(cn) has landed (every warp observes it before it signals M2's readiness)
+        if (!ptx::mbar_wait(bars.v + 8 * (cn & 1), (uint32_t)((cn >> 1) & 1), kWaitLimitNs)) *err_flag = 1;
+        v_seen = cn + 1;
         prep_bar();
         if (pw == 1) {
             // A_kk^T (row `lane` of A_kk scaled by beta_lane, strictly lower)
@@ -608,10 +587,15 @@ __device__ void prep_role(const ChunkArgs &p, uint8_t *sm, uint32_t tmem, const 
         ptx::tc_fence_before();
         warp_signal(bars.rj, lane);
         // M2(cn) has completed: its V buffer can take chunk cn+2
-        if (cn + 2 < nchunks) prefetch_v(p, sm, b, h, cn + 2, pt);
+        if (cn + 2 < nchunks) {
+            if (pt == 0) load_v(maps, sm, bars, b, h, cn + 2);
+            v_loaded = cn + 3;
+        }
         if (*err_flag) break;
     }
-    ptx::cp_async_wait_all();
+    // on an early exit, let the V loads still in flight land before the block ends
+    for (int n = v_seen; n < v_loaded; ++n)
+        (void)ptx::mbar_wait(bars.v + 8 * (n & 1), (uint32_t)((n >> 1) & 1), kWaitLimitNs);
 }
 
 // 16 columns of S'^T in this thread's row j, starting at key channel d0: scale
@@ -635,15 +619,14 @@ __device__ __forceinline__ void write_state16(uint32_t tmem, uint32_t lane_base,
 
 // Chain warps, operands of chunk n (the staging rows must hold chunk n): part A,
 // then (later) part B, the signal to the issuer and the loads of chunk n+1.
-__device__ __forceinline__ void chain_stage_a(const ChunkArgs &p, uint8_t *sm, int n, int warp, int lane,
-                                              float (&ie)[16])
+__device__ __forceinline__ void chain_stage_a(const ChunkArgs &p, uint8_t *sm, const Bars &bars, int n, int warp,
+                                              int lane, float (&ie)[16], volatile int *err_flag)
 {
-    ptx::cp_async_wait_all();
-    chain_bar();   // every thread's copies of chunk n have landed
+    if (!ptx::mbar_wait(bars.stg, (uint32_t)(n & 1), kWaitLimitNs)) *err_flag = 1;   // chunk n's rows
     stage_a(p, sm, n, warp, lane, ie);
 }
 
-__device__ __forceinline__ void chain_stage_b(const ChunkArgs &p, uint8_t *sm, const Bars &bars, int b, int h,
+__device__ __forceinline__ void chain_stage_b(const TcMaps &maps, uint8_t *sm, const Bars &bars, int b, int h,
                                               int n, int nchunks, int tid, int warp, int lane,
                                               const float (&ie)[16])
 {
@@ -651,12 +634,12 @@ __device__ __forceinline__ void chain_stage_b(const ChunkArgs &p, uint8_t *sm, c
     ptx::fence_proxy_async_smem();
     warp_signal(bars.rc, lane);
     chain_bar();   // staging consumed, constants visible to every chain warp
-    if (n + 1 < nchunks) prefetch_qka(p, sm, b, h, n + 1, tid);
+    if (tid == 0 && n + 1 < nchunks) load_qka(maps, sm, bars, b, h, n + 1);
 }
 
 // ---- the chain warps: the serial recurrence over chunks --------------------------------
-__device__ void chain_role(const ChunkArgs &p, uint8_t *sm, uint32_t tmem, const Bars &bars, int b, int h,
-                           int bh, int nchunks, volatile int *err_flag)
+__device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, uint32_t tmem, const Bars &bars,
+                           int b, int h, int bh, int nchunks, volatile int *err_flag)
 {
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -666,9 +649,11 @@ __device__ void chain_role(const ChunkArgs &p, uint8_t *sm, uint32_t tmem, const
     const size_t tile = (size_t)bh * D * D;
 
     float ie[16];   // 1/e of the chunk being staged, carried from part A to part B
-    prefetch_qka(p, sm, b, h, 0, tid);
-    chain_stage_a(p, sm, 0, warp, lane, ie);
-    chain_stage_b(p, sm, bars, b, h, 0, nchunks, tid, warp, lane, ie);
+    if (tid == 0) load_qka(maps, sm, bars, b, h, 0);
+    int staged = 0;   // chunks whose rows have been waited for
+    chain_stage_a(p, sm, bars, 0, warp, lane, ie, err_flag);
+    staged = 1;
+    chain_stage_b(maps, sm, bars, b, h, 0, nchunks, tid, warp, lane, ie);
 
     // S'_0 = Diag(exp(a_0)) S_0; cleared O accumulator
     {
@@ -688,8 +673,9 @@ __device__ void chain_role(const ChunkArgs &p, uint8_t *sm, uint32_t tmem, const
     ptx::tc_fence_before();
     warp_signal(bars.rs, lane);
     if (nchunks > 1) {
-        chain_stage_a(p, sm, 1, warp, lane, ie);
-        chain_stage_b(p, sm, bars, b, h, 1, nchunks, tid, warp, lane, ie);
+        chain_stage_a(p, sm, bars, 1, warp, lane, ie, err_flag);
+        staged = 2;
+        chain_stage_b(maps, sm, bars, b, h, 1, nchunks, tid, warp, lane, ie);
     }
 
     for (int c = 0; c < nchunks; ++c) {
@@ -713,7 +699,10 @@ __device__ void chain_role(const ChunkArgs &p, uint8_t *sm, uint32_t tmem, const
         ptx::tc_fence_before();
         warp_signal(bars.re, lane);
         // Lk, Lq of chunk c+2 while the state update of chunk c runs
-        if (c + 2 < nchunks) chain_stage_a(p, sm, c + 2, warp, lane, ie);
+        if (c + 2 < nchunks) {
+            chain_stage_a(p, sm, bars, c + 2, warp, lane, ie, err_flag);
+            staged = c + 3;
+        }
 
         // ---- I: X = S' + E^T R -> the next S' (or the final state); outputs of chunk c
         if (!ptx::mbar_wait(bars.s, (uint32_t)(c & 1), kWaitLimitNs)) *err_flag = 1;
@@ -756,7 +745,7 @@ __device__ void chain_role(const ChunkArgs &p, uint8_t *sm, uint32_t tmem, const
             }
         }
         // R of chunk c+2 (the update of chunk c has read R(c)), then the outputs of chunk c
-        if (c + 2 < nchunks) chain_stage_b(p, sm, bars, b, h, c + 2, nchunks, tid, warp, lane, ie);
+        if (c + 2 < nchunks) chain_stage_b(maps, sm, bars, b, h, c + 2, nchunks, tid, warp, lane, ie);
         {
             const int t0 = c * C;
             const size_t step = (size_t)p.H * D;
@@ -767,10 +756,12 @@ __device__ void chain_role(const ChunkArgs &p, uint8_t *sm, uint32_t tmem, const
         }
         if (*err_flag) break;
     }
-    ptx::cp_async_wait_all();
+    // on an early exit, let a staging load still in flight land before the block ends
+    if (staged < nchunks && staged > 0)
+        (void)ptx::mbar_wait(bars.stg, (uint32_t)(staged & 1), kWaitLimitNs);
 }
 
-__global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs p)
+__global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs p, const __grid_constant__ TcMaps maps)
 {
     extern __shared__ __align__(1024) uint8_t sm[];
     const int tid = threadIdx.x;
@@ -784,6 +775,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs p)
     const uint32_t bar0 = ptx::smem_u32(sm + OFF_BAR);
     Bars bars;
     bars.a = bar0; bars.w = bar0 + 8; bars.e = bar0 + 16; bars.s = bar0 + 24;
+    bars.stg = bar0 + 32; bars.v = bar0 + 40;   // v and v + 8
     const uint32_t sig0 = ptx::smem_u32(sm + OFF_SIG);
     bars.rc = sig0; bars.rs = sig0 + 4; bars.re = sig0 + 8;
     bars.ra = sig0 + 12; bars.rg = sig0 + 16; bars.rj = sig0 + 20;
@@ -793,6 +785,9 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs p)
         ptx::mbar_init(bars.w, 1);
         ptx::mbar_init(bars.e, 1);
         ptx::mbar_init(bars.s, 1);
+        ptx::mbar_init(bars.stg, 1);
+        ptx::mbar_init(bars.v, 1);
+        ptx::mbar_init(bars.v + 8, 1);
         ptx::fence_mbar_init();
 #pragma unroll
         for (int i = 0; i < 8; ++i) reinterpret_cast<uint32_t *>(sm + OFF_SIG)[i] = 0u;
@@ -810,9 +805,9 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs p)
     if (warp == kIssuerWarp) {
         if (lane == 0) issuer(sm, tmem, bars, nchunks, err_flag);
     } else if (warp >= NCW) {
-        prep_role(p, sm, tmem, bars, b, h, nchunks, err_flag);
+        prep_role(p, maps, sm, tmem, bars, b, h, nchunks, err_flag);
     } else {
-        chain_role(p, sm, tmem, bars, b, h, bh, nchunks, err_flag);
+        chain_role(p, maps, sm, tmem, bars, b, h, bh, nchunks, err_flag);
     }
     if (*err_flag && tid == 0 && p.status) atomicOr(p.status, 1u);
     ptx::tc_fence_before();
@@ -830,15 +825,67 @@ bool chunk_tc_supported(int dk, int dv, kda_dtype qkv, kda_dtype gate)
     return dk == tc::D && dv == tc::D && qkv == KDA_BF16 && gate == KDA_BF16;
 }
 
+namespace {
+
+// cuTensorMapEncodeTiled, looked up once through the runtime (no link-time
+// dependency on the driver library).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// q, k, alpha [B][T][H][128] bf16: dims (d, h, t, b), box (128, 1, 32, 1).
+bool encode_rows(CUtensorMap *m, const void *base, int B, int T, int H)
+{
+    const cuuint64_t dims[4] = {(cuuint64_t)tc::D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)tc::D * 2, (cuuint64_t)H * tc::D * 2,
+                                   (cuuint64_t)T * H * tc::D * 2};
+    const cuuint32_t box[4] = {(cuuint32_t)tc::D, 1, (cuuint32_t)tc::C, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// v [B][T][H][128] bf16 as (j%8, t, j/8, h, b), box (8, 32, 16, 1, 1): the box lands
+// as j/8-major, token-minor 16-byte rows, the MN-major core matrices of V^T.
+bool encode_v(CUtensorMap *m, const void *base, int B, int T, int H)
+{
+    const cuuint64_t dims[5] = {8, (cuuint64_t)T, (cuuint64_t)tc::D / 8, (cuuint64_t)H, (cuuint64_t)B};
+    const cuuint64_t strides[4] = {(cuuint64_t)H * tc::D * 2, 16, (cuuint64_t)tc::D * 2,
+                                   (cuuint64_t)T * H * tc::D * 2};
+    const cuuint32_t box[5] = {8, (cuuint32_t)tc::C, (cuuint32_t)tc::D / 8, 1, 1};
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
 cudaError_t launch_chunk_tc(const ChunkArgs &a, int dk, int dv, cudaStream_t stream)
 {
     (void)dk; (void)dv;
     const long long blocks = (long long)a.B * a.H;
     if (blocks == 0) return cudaSuccess;
+    if (encode_fn() == nullptr) return cudaErrorNotSupported;
+    tc::TcMaps maps;
+    if (!encode_rows(&maps.q, a.q, a.B, a.T, a.H) || !encode_rows(&maps.k, a.k, a.B, a.T, a.H) ||
+        !encode_rows(&maps.a, a.alpha, a.B, a.T, a.H) || !encode_v(&maps.v, a.v, a.B, a.T, a.H))
+        return cudaErrorInvalidValue;
     cudaError_t err = cudaFuncSetAttribute(tc::kda_chunk_tc_kernel,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
     if (err != cudaSuccess) return err;
-    tc::kda_chunk_tc_kernel<<<(unsigned)blocks, tc::NT, tc::SMEM_BYTES, stream>>>(a);
+    tc::kda_chunk_tc_kernel<<<(unsigned)blocks, tc::NT, tc::SMEM_BYTES, stream>>>(a, maps);
     return cudaGetLastError();
 }
 
