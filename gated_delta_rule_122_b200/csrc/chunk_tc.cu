@@ -78,18 +78,15 @@ __device__ __forceinline__ uint32_t dm(int slab, int d, int r)
 {
     return (uint32_t)(slab * SLAB + (d >> 3) * 128 + (d & 7) * 16 + (r & 7) * 2);
 }
-// Slabs of one operand stage.  M=128 A-product operand = slabs 0..15, O/E product
-// operand = slabs 8..23, R = slabs 24..31 (token block rb, plane pl at 24 + 2rb + pl).
-constexpr int SL_LK_LO = 0, SL_LK_HI = 4, SL_LQ_HI = 8, SL_LQ_LO = 12, SL_W_HI = 16, SL_W_LO = 20, SL_R = 24;
+// Slabs of one operand stage: every operand keeps token block rb's hi plane in slab
+// base + 2rb and its lo plane in base + 2rb + 1.  M=128 A-product operand = slabs
+// 0..15 (Lk, Lq), O/E product operand = slabs 8..23 (Lq, -W'), R = slabs 24..31.
+constexpr int SL_LK = 0, SL_LQ = 8, SL_W = 16, SL_R = 24;
 
-// Plane-major K-major operand with N = 32 rows per plane and K = 32 (T', A_qk):
-// row block (pl*4 + r/8) at 512 B, K block s/8 at 128 B.
-__device__ __forceinline__ uint32_t pm(int pl, int r, int s)
-{
-    return (uint32_t)((pl * 4 + (r >> 3)) * 512 + (s >> 3) * 128 + (r & 7) * 16 + (s & 7) * 2);
-}
-// Plane-interleaved K-major layout with K = 32 (E^T: rows j, K = s): row block j/8
-// holds the hi plane's 4 core matrices, then the lo plane's.
+// Plane-interleaved K-major layout with K = 32 (E^T: rows j; T', A_qk: rows r;
+// K = s): row block row/8 holds the hi plane's 4 core matrices, then the lo
+// plane's, so the N = 64 operand [rows 0-7 hi, rows 0-7 lo, rows 8-15 hi, ...]
+// has uniform 512-byte row-block strides.
 __device__ __forceinline__ uint32_t ipl(int row, int k, int plane)
 {
     return (uint32_t)((row >> 3) * (C * 32) + plane * (C * 16) + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2);
@@ -117,9 +114,8 @@ constexpr int OFF_TP = OFF_ET + D * C * 4;             // T'  (B of W'/U: N = r,
 constexpr int OFF_AQ = OFF_TP + C * C * 4;             // 2 x A_qk (B of O: N = r, K = s)
 constexpr int AQ_BYTES = C * C * 4;
 constexpr int P = C + 1;                               // fp32 [32][33] tiles
-constexpr int OFF_PK = OFF_AQ + 2 * AQ_BYTES;          // partial A_kk (lo-plane rows)
-constexpr int OFF_PQ = OFF_PK + C * P * 4;             // partial A_qk (hi-plane rows)
-constexpr int OFF_AKK = OFF_PQ + C * P * 4;            // A_kk^T fp32 [32][36]
+constexpr int OFF_XS = OFF_AQ + 2 * AQ_BYTES;          // A10 T0 of the solve fp32 [16][33]
+constexpr int OFF_AKK = OFF_XS + C * P * 4;            // A_kk^T fp32 [32][36]
 constexpr int OFF_TS = OFF_AKK + C * (C + 4) * 4;      // T fp32 [32][33]
 constexpr int OFF_BETA = OFF_TS + C * P * 4;           // beta of the chunk being solved
 constexpr int NBARS = 7;
@@ -131,7 +127,7 @@ static_assert(SMEM_BYTES <= 232448, "shared memory plan exceeds the per-block li
 static_assert(OFF_AKK % 16 == 0 && OFF_LQR % 128 == 0, "vector and operand alignment");
 
 // TMEM columns
-constexpr uint32_t TM_A = 0;      // [A_kk; A_qk] partial products (M=128: 4 row groups, N=64)
+constexpr uint32_t TM_A = 0;      // [A_kk; A_qk] per plane of Lk, Lq (M=128, N=64)
 constexpr uint32_t TM_O = 64;     // O^T (64 cols: hi/lo groups), directly followed by
 constexpr uint32_t TM_E = 128;    // E^T (64 cols) so that one N=128 MMA writes both
 constexpr uint32_t TM_S = 192;    // fp32 S'^T, accumulated into X^T by the E^T R product
@@ -170,6 +166,17 @@ __device__ __forceinline__ float ld_bf16(const uint8_t *p)
 
 __device__ __forceinline__ void chain_bar() { ptx::named_bar_sync(kChainBar, NCT); }
 __device__ __forceinline__ void prep_bar() { ptx::named_bar_sync(kPrepBar, NPT); }
+// The same barriers, returning whether any thread of the role has seen the error
+// flag: a role leaves its loop only on this common answer, so no thread is left
+// waiting at a named barrier (which has no time limit).
+__device__ __forceinline__ bool chain_bar_err(volatile int *err_flag)
+{
+    return ptx::named_bar_sync_or(kChainBar, NCT, *err_flag != 0);
+}
+__device__ __forceinline__ bool prep_bar_err(volatile int *err_flag)
+{
+    return ptx::named_bar_sync_or(kPrepBar, NPT, *err_flag != 0);
+}
 
 __device__ __forceinline__ float load_beta(const ChunkArgs &p, int b, int h, int n, int r)
 {
@@ -180,9 +187,9 @@ __device__ __forceinline__ float load_beta(const ChunkArgs &p, int b, int h, int
 
 // TMA descriptors of one launch: q, k, alpha as [B][T][H][128] boxes of 32 token
 // rows; v as the 5-D view (j%8, t, j/8, h, b) whose 8 x 32 x 16 box lands in the
-// MN-major core-matrix layout of the U^T product.
+// MN-major core-matrix layout of the U^T product; o as boxes of 16 token rows.
 struct TcMaps {
-    CUtensorMap q, k, a, v;
+    CUtensorMap q, k, a, v, o;
 };
 
 // Every warp of a role adds 1 to a readiness counter once its writes are visible
@@ -213,7 +220,7 @@ struct MmaIds {
 __device__ __forceinline__ void issue_m3(uint8_t *sm, uint32_t tmem, const Bars &bars, const MmaIds &id, int n3)
 {
     ptx::tc_fence_after();
-    const uint32_t b0 = ptx::smem_u32(sm + OFF_LQR + (n3 & 1) * LQR_BYTES) + SL_LQ_HI * SLAB;
+    const uint32_t b0 = ptx::smem_u32(sm + OFF_LQR + (n3 & 1) * LQR_BYTES) + SL_LQ * SLAB;
     for (int ks = 0; ks < D / 16; ++ks)
         for (int pl = 0; pl < 2; ++pl)
             ptx::mma_bf16_ts(tmem + TM_O, tmem + TM_SP + 64 * pl + 8 * ks,
@@ -245,7 +252,7 @@ __device__ __forceinline__ void issue_m1(uint8_t *sm, uint32_t tmem, const Bars 
     ptx::tc_fence_after();
     const uint32_t base = ptx::smem_u32(sm + OFF_LQR + (n1 & 1) * LQR_BYTES);
     for (int ks = 0; ks < D / 16; ++ks)
-        ptx::mma_bf16(tmem + TM_A, ptx::smem_desc(base + SL_LK_LO * SLAB + 256 * ks, 128, SLAB),
+        ptx::mma_bf16(tmem + TM_A, ptx::smem_desc(base + SL_LK * SLAB + 256 * ks, 128, SLAB),
                       ptx::smem_desc(base + SL_R * SLAB + 256 * ks, 128, SLAB), id.A, ks > 0);
     ptx::mma_commit(bars.a);
 }
@@ -258,9 +265,9 @@ __device__ __forceinline__ void issue_m2(uint8_t *sm, uint32_t tmem, const Bars 
     const uint32_t vv = ptx::smem_u32(sm + OFF_V + (n2 & 1) * V_BYTES);
     for (int ks = 0; ks < C / 16; ++ks)
         for (int pl = 0; pl < 2; ++pl)
-            // Lk as the K-major (M = d, K = s) operand
+            // Lk plane pl as the K-major (M = d, K = s) operand: token blocks 2 slabs apart
             ptx::mma_bf16(tmem + TM_W,
-                          ptx::smem_desc(base + (pl ? SL_LK_LO : SL_LK_HI) * SLAB + 2 * SLAB * ks, SLAB, 128),
+                          ptx::smem_desc(base + (SL_LK + pl) * SLAB + 4 * SLAB * ks, 2 * SLAB, 128),
                           ptx::smem_desc(tp + 256 * ks, 128, 512), id.W, ks > 0 || pl > 0);
     for (int ks = 0; ks < C / 16; ++ks)
         ptx::mma_bf16(tmem + TM_E, ptx::smem_desc(vv + 256 * ks, 128, (C / 8) * 128),
@@ -268,8 +275,9 @@ __device__ __forceinline__ void issue_m2(uint8_t *sm, uint32_t tmem, const Bars 
     ptx::mma_commit(bars.w);
 }
 
-// Readiness of each group: M1(n) needs Lk, Lq, R of chunk n (rc) and A(n-1) read
-// (ra); M2(n) needs T' and A_qk (rg; the prep warps signal it after reading
+// Readiness of each group: M1(n) needs Lk, Lq, R of chunk n (rc), A(n-1) read (ra)
+// and M2(n-1) issued (an M1 issued ahead of a ready M2 would hold the prep warps
+// up for its whole issue time); M2(n) needs T' and A_qk (rg; the prep warps signal it after reading
 // W'(n-1)) and M4(n-1) issued, since U goes into TM_E; M3(n) needs S'(n) (rs,
 // whose first count is the initial state) and -W'(n) (rj); M4(n) needs E^T(n) (re).
 __device__ void issuer(uint8_t *sm, uint32_t tmem, const Bars &bars, int nchunks, volatile int *err_flag)
@@ -295,7 +303,7 @@ __device__ void issuer(uint8_t *sm, uint32_t tmem, const Bars &bars, int nchunks
             g = 4;
         else if (n2 < n1 && n2 <= n4 && c_rg >= (uint32_t)(NPW * (n2 + 1)))
             g = 2;
-        else if (n1 < nchunks && c_ra >= (uint32_t)(NPW * n1) && c_rc >= (uint32_t)(NCW * (n1 + 1)))
+        else if (n1 < nchunks && n1 == n2 && c_ra >= (uint32_t)(NPW * n1) && c_rc >= (uint32_t)(NCW * (n1 + 1)))
             g = 1;
         if (g != 0) {
             // acquire the producers' writes (the counters only grow)
@@ -407,8 +415,8 @@ __device__ void stage_a(const ChunkArgs &p, uint8_t *sm, int n, int warp, int la
             lk[i] = kv * e;
             lq[i] = p.scale * qv * e;
         }
-        st_split8(lqr + dm(SL_LK_HI + 2 * hf + u, d, 0), (SL_LK_LO - SL_LK_HI) * SLAB, lk);
-        st_split8(lqr + dm(SL_LQ_HI + 2 * hf + u, d, 0), (SL_LQ_LO - SL_LQ_HI) * SLAB, lq);
+        st_split8(lqr + dm(SL_LK + 2 * (2 * hf + u), d, 0), SLAB, lk);
+        st_split8(lqr + dm(SL_LQ + 2 * (2 * hf + u), d, 0), SLAB, lq);
     }
 }
 
@@ -455,12 +463,15 @@ __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, u
     const int pt = threadIdx.x - NCT;          // 0..127
     const int pw = pt >> 5, lane = pt & 31;    // warp = TMEM lane quadrant
     const uint32_t lane_base = (uint32_t)(pw * 32) << 16;
-    float *PK = reinterpret_cast<float *>(sm + OFF_PK);
-    float *PQ = reinterpret_cast<float *>(sm + OFF_PQ);
     float *At = reinterpret_cast<float *>(sm + OFF_AKK);   // A_kk transposed
     float *Tm = reinterpret_cast<float *>(sm + OFF_TS);    // T = (I + A_kk)^-1
-    float *Xs = PK;                                        // A10 T0 (PK is consumed by then)
+    float *Xs = reinterpret_cast<float *>(sm + OFF_XS);    // A10 T0
     float *sbeta = reinterpret_cast<float *>(sm + OFF_BETA);
+    // This lane's row of the A product: lane quadrant pw holds token blocks 2(pw&1)
+    // and 2(pw&1)+1 of Lk (pw < 2) or Lq (pw >= 2), hi plane in lanes 0-7 / 16-23,
+    // lo plane in lanes 8-15 / 24-31.
+    const int pl = (lane >> 3) & 1;
+    const int r = 16 * (pw & 1) + 8 * (lane >> 4) + (lane & 7);
 
     int v_loaded = 0, v_seen = 0;   // V loads issued (thread pt 0) and waited for
     if (pt == 0) {
@@ -468,15 +479,15 @@ __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, u
         if (nchunks > 1) load_v(maps, sm, bars, b, h, 1);
     }
     v_loaded = nchunks > 1 ? 2 : 1;
-    float beta = (pw == 1) ? load_beta(p, b, h, 0, lane) : 0.f;   // beta of row / column `lane`
+    float beta = (pw < 2) ? load_beta(p, b, h, 0, r) : 0.f;   // beta of row r
 
     for (int cn = 0; cn < nchunks; ++cn) {
-        const float beta_next = (pw == 1 && cn + 1 < nchunks) ? load_beta(p, b, h, cn + 1, lane) : 0.f;
+        const float beta_next = (pw < 2 && cn + 1 < nchunks) ? load_beta(p, b, h, cn + 1, r) : 0.f;
 
         // ---- G(cn): A_kk / A_qk from TMEM; the solve; T'
         if (!ptx::mbar_wait(bars.a, (uint32_t)(cn & 1), kWaitLimitNs)) *err_flag = 1;
         ptx::tc_fence_after();
-        float a32[32];   // this row group's products with R, summed over R's planes
+        float a32[32];   // this plane's row r times R, summed over R's planes
 #pragma unroll
         for (int hs = 0; hs < 2; ++hs) {
             float v[32];
@@ -489,33 +500,34 @@ __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, u
         }
         ptx::tc_fence_before();
         warp_signal(bars.ra, lane);
-        if (pw == 0 || pw == 2) {
-            float *dst = (pw == 0 ? PK : PQ) + lane * P;
+        // add the other plane's row (lane ^ 8): this lane keeps columns s = 16 pl .. 16 pl + 15
+        float ar[16];
 #pragma unroll
-            for (int s = 0; s < C; ++s) dst[s] = a32[s];
+        for (int i = 0; i < 16; ++i) {
+            const float send = pl ? a32[i] : a32[16 + i];
+            const float keep = pl ? a32[16 + i] : a32[i];
+            ar[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
         }
         // V(cn) has landed (every warp observes it before it signals M2's readiness)
         if (!ptx::mbar_wait(bars.v + 8 * (cn & 1), (uint32_t)((cn >> 1) & 1), kWaitLimitNs)) *err_flag = 1;
         v_seen = cn + 1;
-        prep_bar();
-        if (pw == 1) {
-            // A_kk^T (row `lane` of A_kk scaled by beta_lane, strictly lower)
-            const float *src = PK + lane * P;
+        if (pw < 2) {
+            // A_kk^T: row r of A_kk scaled by beta_r, strictly lower
 #pragma unroll
-            for (int s = 0; s < C; ++s) At[s * PT + lane] = (s < lane) ? beta * (a32[s] + src[s]) : 0.f;
-            sbeta[lane] = beta;
-        } else if (pw == 3) {
-            const float *src = PQ + lane * P;
+            for (int i = 0; i < 16; ++i) {
+                const int s = 16 * pl + i;
+                At[s * PT + r] = (s < r) ? beta * ar[i] : 0.f;
+            }
+            if (pl == 0) sbeta[r] = beta;
+        } else {
+            // A_qk row r, lower triangle including the diagonal
             uint8_t *aq = sm + OFF_AQ + (cn & 1) * AQ_BYTES;
 #pragma unroll
-            for (int sb = 0; sb < 4; ++sb) {
+            for (int u = 0; u < 2; ++u) {
                 float x[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int s = 8 * sb + i;
-                    x[i] = (s <= lane) ? a32[s] + src[s] : 0.f;
-                }
-                st_split8(aq + pm(0, lane, 8 * sb), 4 * 512, x);
+                for (int i = 0; i < 8; ++i) x[i] = (16 * pl + 8 * u + i <= r) ? ar[8 * u + i] : 0.f;
+                st_split8(aq + ipl(r, 16 * pl + 8 * u, 0), C * 16, x);
             }
             ptx::fence_proxy_async_smem();
         }
@@ -546,17 +558,17 @@ __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, u
             Tm[(16 + i) * P + c0] = -y0;
             Tm[(16 + i) * P + c0 + 1] = -y1;
         }
-        prep_bar();
+        const bool stop = prep_bar_err(err_flag);
         {
-            // T' = T Diag(beta): row r, columns 8sc..8sc+7, as hi/lo planes
-            const int r = 8 * pw + (lane & 7), sc = lane >> 3;
+            // T' = T Diag(beta): row rt, columns 8sc..8sc+7, as hi/lo planes
+            const int rt = 8 * pw + (lane & 7), sc = lane >> 3;
             float x[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int s = 8 * sc + i;
-                x[i] = (r < 16 && s >= 16) ? 0.f : Tm[r * P + s] * sbeta[s];
+                x[i] = (rt < 16 && s >= 16) ? 0.f : Tm[rt * P + s] * sbeta[s];
             }
-            st_split8(sm + OFF_TP + pm(0, r, 8 * sc), 4 * 512, x);
+            st_split8(sm + OFF_TP + ipl(rt, 8 * sc, 0), C * 16, x);
             ptx::fence_proxy_async_smem();
         }
         warp_signal(bars.rg, lane);
@@ -570,17 +582,18 @@ __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, u
             const int d = 32 * pw + lane;
 #pragma unroll
             for (int hs = 0; hs < 2; ++hs) {
-                float vh[16], vl[16];
-                ptx::tmem_ld16(tmem + lane_base + TM_W + 16 * hs, vh);        // T' hi rows
-                ptx::tmem_ld16(tmem + lane_base + TM_W + 32 + 16 * hs, vl);   // T' lo rows
+                float v0[16], v1[16];   // token blocks 2hs and 2hs+1: T' hi rows, then lo rows
+                ptx::tmem_ld16(tmem + lane_base + TM_W + 32 * hs, v0);
+                ptx::tmem_ld16(tmem + lane_base + TM_W + 32 * hs + 16, v1);
                 ptx::tmem_wait_ld();
+                float x0[8], x1[8];
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    float x[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) x[i] = -(vh[8 * u + i] + vl[8 * u + i]);
-                    st_split8(lqr + dm(SL_W_HI + 2 * hs + u, d, 0), (SL_W_LO - SL_W_HI) * SLAB, x);
+                for (int i = 0; i < 8; ++i) {
+                    x0[i] = -(v0[i] + v0[8 + i]);
+                    x1[i] = -(v1[i] + v1[8 + i]);
                 }
+                st_split8(lqr + dm(SL_W + 2 * (2 * hs), d, 0), SLAB, x0);
+                st_split8(lqr + dm(SL_W + 2 * (2 * hs + 1), d, 0), SLAB, x1);
             }
         }
         ptx::fence_proxy_async_smem();
@@ -591,7 +604,7 @@ __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, u
             if (pt == 0) load_v(maps, sm, bars, b, h, cn + 2);
             v_loaded = cn + 3;
         }
-        if (*err_flag) break;
+        if (stop) break;
     }
     // on an early exit, let the V loads still in flight land before the block ends
     for (int n = v_seen; n < v_loaded; ++n)
@@ -637,6 +650,12 @@ __device__ __forceinline__ void chain_stage_b(const TcMaps &maps, uint8_t *sm, c
     if (tid == 0 && n + 1 < nchunks) load_qka(maps, sm, bars, b, h, n + 1);
 }
 
+__device__ __forceinline__ void warp_signal_after_stage(const Bars &bars, int lane)
+{
+    ptx::fence_proxy_async_smem();
+    warp_signal(bars.rc, lane);
+}
+
 // ---- the chain warps: the serial recurrence over chunks --------------------------------
 __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, uint32_t tmem, const Bars &bars,
                            int b, int h, int bh, int nchunks, volatile int *err_flag)
@@ -666,8 +685,8 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
             for (int i = 0; i < 16; ++i) v[i] = p.s_in ? p.s_in[tile + (size_t)(d0 + i) * D + j] : 0.f;
             write_state16(tmem, lane_base, d0, v, cst0 + d0);
         }
-        ptx::tmem_st16_zero(tmem + lane_base + TM_O + 16 * half);
-        ptx::tmem_st16_zero(tmem + lane_base + TM_O + 32 + 16 * half);
+        ptx::tmem_st16_zero(tmem + lane_base + TM_O + 32 * half);
+        ptx::tmem_st16_zero(tmem + lane_base + TM_O + 32 * half + 16);
         ptx::tmem_wait_st();
     }
     ptx::tc_fence_before();
@@ -683,17 +702,19 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
         if (!ptx::mbar_wait(bars.e, (uint32_t)(c & 1), kWaitLimitNs)) *err_flag = 1;
         ptx::tc_fence_after();
         {
-            float vh[16], vl[16];
-            ptx::tmem_ld16(tmem + lane_base + TM_E + 16 * half, vh);
-            ptx::tmem_ld16(tmem + lane_base + TM_E + 32 + 16 * half, vl);
+            // token blocks 2 half and 2 half + 1, each as [hi 8 | lo 8] columns
+            float v0[16], v1[16];
+            ptx::tmem_ld16(tmem + lane_base + TM_E + 32 * half, v0);
+            ptx::tmem_ld16(tmem + lane_base + TM_E + 32 * half + 16, v1);
             ptx::tmem_wait_ld();
+            float e0[8], e1[8];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                float e8[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) e8[i] = vh[8 * u + i] + vl[8 * u + i];
-                st_split8(sm + OFF_ET + ipl(j, 16 * half + 8 * u, 0), C * 16, e8);
+            for (int i = 0; i < 8; ++i) {
+                e0[i] = v0[i] + v0[8 + i];
+                e1[i] = v1[i] + v1[8 + i];
             }
+            st_split8(sm + OFF_ET + ipl(j, 16 * half, 0), C * 16, e0);
+            st_split8(sm + OFF_ET + ipl(j, 16 * half + 8, 0), C * 16, e1);
         }
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
@@ -709,25 +730,42 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
         ptx::tc_fence_after();
         float ov[16];
         {
-            float vh[16], vl[16];
-            ptx::tmem_ld16(tmem + lane_base + TM_O + 16 * half, vh);
-            ptx::tmem_ld16(tmem + lane_base + TM_O + 32 + 16 * half, vl);
+            float v0[16], v1[16];
+            ptx::tmem_ld16(tmem + lane_base + TM_O + 32 * half, v0);
+            ptx::tmem_ld16(tmem + lane_base + TM_O + 32 * half + 16, v1);
             ptx::tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) ov[i] = vh[i] + vl[i];
+            for (int i = 0; i < 8; ++i) {
+                ov[i] = v0[i] + v0[8 + i];
+                ov[8 + i] = v1[i] + v1[8 + i];
+            }
         }
         if (c + 1 < nchunks) {
             // f(c+1) = exp(a_{c+1}) exp(G_end,c - a_c), written when chunk c+1 was staged
             const float *f = reinterpret_cast<const float *>(sm + OFF_CST + ((c + 1) % kCstSlots) * CST_BYTES) + 2 * D;
-            ptx::tmem_st16_zero(tmem + lane_base + TM_O + 16 * half);
-            ptx::tmem_st16_zero(tmem + lane_base + TM_O + 32 + 16 * half);
+            ptx::tmem_st16_zero(tmem + lane_base + TM_O + 32 * half);
+            ptx::tmem_st16_zero(tmem + lane_base + TM_O + 32 * half + 16);
 #pragma unroll 1
-            for (int part = 0; part < 4; ++part) {
-                const int d0 = 64 * half + 16 * part;
-                float v[16];
-                ptx::tmem_ld16(tmem + lane_base + TM_S + d0, v);
+            for (int q2 = 0; q2 < 2; ++q2) {
+                const int d0 = 64 * half + 32 * q2;
+                float v[32];
+                ptx::tmem_ld32(tmem + lane_base + TM_S + d0, v);
                 ptx::tmem_wait_ld();
-                write_state16(tmem, lane_base, d0, v, f + d0);
+                const float4 *f4 = reinterpret_cast<const float4 *>(f + d0);
+#pragma unroll
+                for (int i4 = 0; i4 < 8; ++i4) {
+                    const float4 ff = f4[i4];
+                    v[4 * i4 + 0] *= ff.x;
+                    v[4 * i4 + 1] *= ff.y;
+                    v[4 * i4 + 2] *= ff.z;
+                    v[4 * i4 + 3] *= ff.w;
+                }
+                ptx::tmem_st32(tmem + lane_base + TM_S + d0, v);
+                uint32_t hw[16], lw[16];
+#pragma unroll
+                for (int m = 0; m < 16; ++m) split_pair(v[2 * m], v[2 * m + 1], hw[m], lw[m]);
+                ptx::tmem_st16(tmem + lane_base + TM_SP + d0 / 2, hw);
+                ptx::tmem_st16(tmem + lane_base + TM_SP + 64 + d0 / 2, lw);
             }
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
@@ -744,21 +782,48 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
                 for (int i = 0; i < 16; ++i) p.s_out[tile + (size_t)(d0 + i) * D + j] = cend[d0 + i] * v[i];
             }
         }
-        // R of chunk c+2 (the update of chunk c has read R(c)), then the outputs of chunk c
-        if (c + 2 < nchunks) chain_stage_b(maps, sm, bars, b, h, c + 2, nchunks, tid, warp, lane, ie);
-        {
-            const int t0 = c * C;
-            const size_t step = (size_t)p.H * D;
-            size_t idx = (((size_t)b * p.T + t0 + 16 * half) * p.H + h) * D + j;
-#pragma unroll
-            for (int i = 0; i < 16; ++i, idx += step)
-                if (t0 + 16 * half + i < p.T) st_elem(p.o, idx, ov[i], p.out_bf16);
+        // outputs of chunk c into the staging rows q and alpha have left (rows 16h..16h+15
+        // into the q rows for h = 0, the alpha rows for h = 1), as one TMA box each.
+        // The previous chunk's output store must have read those rows: a staging fill
+        // orders that (thread 0 issues it after the read); without one, sync here.
+        if (c > 0 && c + 2 >= nchunks) {
+            if (tid == 0) ptx::bulk_wait_read();
+            chain_bar();
         }
-        if (*err_flag) break;
+        {
+            const int esz = p.out_bf16 ? 2 : 4;
+            uint8_t *tile = sm + OFF_STG + (half ? STG_A : STG_Q) + j * esz;
+            if (p.out_bf16) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    *reinterpret_cast<__nv_bfloat16 *>(tile + i * D * 2) = __float2bfloat16_rn(ov[i]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) *reinterpret_cast<float *>(tile + i * D * 4) = ov[i];
+            }
+        }
+        // R of chunk c+2 (the update of chunk c has read R(c))
+        if (c + 2 < nchunks) {
+            stage_b(sm, c + 2, warp, lane, ie);
+            warp_signal_after_stage(bars, lane);
+        }
+        ptx::fence_proxy_async_smem();
+        const bool stop = chain_bar_err(err_flag);   // output tile written, staging rows consumed
+        if (tid == 0) {
+            ptx::tma_store_4d(&maps.o, ptx::smem_u32(sm + OFF_STG + STG_Q), 0, h, c * C, b);
+            if (c * C + 16 < p.T) ptx::tma_store_4d(&maps.o, ptx::smem_u32(sm + OFF_STG + STG_A), 0, h, c * C + 16, b);
+            ptx::bulk_commit();
+            if (c + 3 < nchunks) {
+                ptx::bulk_wait_read();   // the tile has been read: the staging rows can be refilled
+                load_qka(maps, sm, bars, b, h, c + 3);
+            }
+        }
+        if (stop) break;
     }
     // on an early exit, let a staging load still in flight land before the block ends
     if (staged < nchunks && staged > 0)
         (void)ptx::mbar_wait(bars.stg, (uint32_t)(staged & 1), kWaitLimitNs);
+    if (tid == 0) ptx::bulk_wait();   // the output stores are complete
 }
 
 __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs p, const __grid_constant__ TcMaps maps)
@@ -870,6 +935,19 @@ bool encode_v(CUtensorMap *m, const void *base, int B, int T, int H)
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// o [B][T][H][128] fp32 or bf16: dims (j, h, t, b), box (128, 1, 16, 1).
+bool encode_out(CUtensorMap *m, void *base, int B, int T, int H, int bf16)
+{
+    const cuuint64_t es = bf16 ? 2 : 4;
+    const cuuint64_t dims[4] = {(cuuint64_t)tc::D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)tc::D * es, (cuuint64_t)H * tc::D * es, (cuuint64_t)T * H * tc::D * es};
+    const cuuint32_t box[4] = {(cuuint32_t)tc::D, 1, 16, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return encode_fn()(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims,
+                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                       CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 cudaError_t launch_chunk_tc(const ChunkArgs &a, int dk, int dv, cudaStream_t stream)
@@ -880,7 +958,8 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, int dk, int dv, cudaStream_t str
     if (encode_fn() == nullptr) return cudaErrorNotSupported;
     tc::TcMaps maps;
     if (!encode_rows(&maps.q, a.q, a.B, a.T, a.H) || !encode_rows(&maps.k, a.k, a.B, a.T, a.H) ||
-        !encode_rows(&maps.a, a.alpha, a.B, a.T, a.H) || !encode_v(&maps.v, a.v, a.B, a.T, a.H))
+        !encode_rows(&maps.a, a.alpha, a.B, a.T, a.H) || !encode_v(&maps.v, a.v, a.B, a.T, a.H) ||
+        !encode_out(&maps.o, a.o, a.B, a.T, a.H, a.out_bf16))
         return cudaErrorInvalidValue;
     cudaError_t err = cudaFuncSetAttribute(tc::kda_chunk_tc_kernel,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);

@@ -129,6 +129,23 @@ __device__ __forceinline__ void tma_load_5d(uint32_t dst, const void *tmap, uint
         : "memory");
 }
 
+// TMA tiled store of a box from shared memory (bulk-group completion).  The
+// box must start at a non-negative coordinate; rows past the tensor's end are
+// not written.
+__device__ __forceinline__ void tma_store_4d(const void *tmap, uint32_t src, int c0, int c1, int c2, int c3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(tmap)),
+        "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until the committed bulk stores have read their shared-memory source.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Wait until the committed bulk stores are complete.
+__device__ __forceinline__ void bulk_wait() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Monotonic shared-memory counters as a cheap producer -> consumer signal: the
 // producer adds with release semantics; the consumer polls with relaxed loads and,
 // once it has seen the count it needs, re-reads that counter with acquire semantics.
@@ -153,6 +170,22 @@ __device__ __forceinline__ uint32_t ld_acquire(uint32_t addr)
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Named barrier that also ORs a predicate over the participating threads: every
+// thread gets the same answer (used to leave a loop together).
+__device__ __forceinline__ bool named_bar_sync_or(int id, int nthreads, bool pred)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.cta.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
 }
 
 // ---- proxies and tcgen05 ordering -------------------------------------------
