@@ -49,6 +49,11 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="run one kernel per step (for profiling); the JSON line is then partial")
+    ap.add_argument("--prefill-seqs", type=int, default=None,
+                    help="sequences per rank of the prefill workload (profiling a smaller case; "
+                         "the JSON line then describes that case, not the headline workload)")
+    ap.add_argument("--prefill-len", type=int, default=None,
+                    help="tokens per sequence of the prefill workload (profiling a smaller case)")
     return ap.parse_args()
 
 
@@ -264,8 +269,13 @@ def main():
     p0, p1 = shard_bounds(world * wp.B, rank, world)
     d0, d1 = shard_bounds(world * wd.B, rank, world)
     wp, wd = wp.scaled(B=p1 - p0), wd.scaled(B=d1 - d0)
+    if args.prefill_seqs is not None:
+        wp = wp.scaled(B=args.prefill_seqs)
+    if args.prefill_len is not None:
+        wp = wp.scaled(T=args.prefill_len)
     x = make_inputs(wp, device=device, seed=wp.seed + p0)
-    y = make_decode_inputs(wd, device=device, seed=wd.seed + d0)
+    # the decode state (2.2 GB) is only allocated when the decode step runs
+    y = make_decode_inputs(wd, device=device, seed=wd.seed + d0) if args.only != "prefill" else None
     o = torch.empty((wp.B, wp.T, wp.H, wp.dv), device=device, dtype=torch.float32)
     S = torch.empty((wp.B, wp.H, wp.dk, wp.dv), device=device, dtype=torch.float32)
     od = torch.empty((wd.B, wd.H, wd.dv), device=device, dtype=torch.float32)
@@ -356,13 +366,17 @@ def main():
     clocks = sampler.summary()
     if rank != 0:
         return
-    traffic = PREFILL_TRAFFIC_BYTES
+    headline = args.prefill_seqs is None and args.prefill_len is None
+    traffic = PREFILL_TRAFFIC_BYTES if headline else None
+    workload_desc = (f"prefill B={wp.B * world} H={wp.H} T={wp.T} d_k=d_v={wp.dk} bf16 q/k/v/alpha/beta, "
+                     "fp32 o and state")
+    if args.only != "prefill":
+        workload_desc += f" (+ decode step N={wd.B * world} H={wd.H} d={wd.dk} in the same step)"
     line = {
         "metric": METRIC, "value": value, "unit": "Mtokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": "prefill B=2 H=64 T=8192 d_k=d_v=128 bf16 q/k/v/alpha/beta, fp32 o and "
-                               "state (+ decode step N=256 H=64 d=128 in the same step)",
+        "config": {"workload": workload_desc,
                    "global_batch": wp.B * world, "seq_len": wp.T, "heads": wp.H, "d": wp.dk,
                    "parallelism": f"dp{world}" if world > 1 else "single",
                    "l2": "inputs larger than L2 (126 MB), no flush",
@@ -371,10 +385,10 @@ def main():
         "roofline": {"bound": "hbm", "achieved": pre_gbs, "peak": hbm, "unit": "GB/s",
                      "frac": pre_gbs / hbm, "traffic": traffic,
                      "algorithmic_bytes": pb, "peak_source": f"{peak_kind} hbm_gbs (copy)"},
-        "decode": {"value": dec_gbs, "unit": "GB/s", "us_per_step": dec_ms * 1e3,
-                   "algorithmic_bytes": db, "frac_of_measured_hbm": dec_gbs / hbm,
-                   "frac_of_8TBs": dec_gbs / 8000.0},
-        "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": 2 * K, "clocks": clocks,
+        "decode": None if args.only == "prefill" else {
+            "value": dec_gbs, "unit": "GB/s", "us_per_step": dec_ms * 1e3, "algorithmic_bytes": db,
+            "frac_of_measured_hbm": dec_gbs / hbm, "frac_of_8TBs": dec_gbs / 8000.0},
+        "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": (1 if args.only else 2) * K, "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
 

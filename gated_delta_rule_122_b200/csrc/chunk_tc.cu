@@ -140,8 +140,9 @@ constexpr uint32_t TM_COLS = 512;
 __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t &hw, uint32_t &lw)
 {
     const uint32_t u0 = __float_as_uint(x0), u1 = __float_as_uint(x1);
-    const float l0 = x0 - __uint_as_float(u0 & 0xFFFF0000u);
-    const float l1 = x1 - __uint_as_float(u1 & 0xFFFF0000u);
+    float l0, l1;
+    ptx::upk2(ptx::sub2(ptx::pk2(x0, x1), ptx::pk2(__uint_as_float(u0 & 0xFFFF0000u), __uint_as_float(u1 & 0xFFFF0000u))),
+              l0, l1);
     hw = __byte_perm(u0, u1, 0x7632);            // upper halves of u0 (low) and u1 (high)
     const __nv_bfloat162 lp = __floats2bfloat162_rn(l0, l1);
     lw = *reinterpret_cast<const uint32_t *>(&lp);
@@ -403,17 +404,23 @@ __device__ void stage_a(const ChunkArgs &p, uint8_t *sm, int n, int warp, int la
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
         float lk[8], lq[8];
+        const uint64_t scale2 = ptx::pk2(p.scale, p.scale);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int r = 16 * hf + 8 * u + i;
-            const float m = fminf(fmaxf(pr[8 * u + i], kMinScale), 1.f / kMinScale);
-            const float rm = ptx::rcp(m);
-            const float e = hf ? m : rm;
-            ie[8 * u + i] = hf ? rm : m;
-            const float kv = ld_bf16(stg + STG_K + stg_row(r) + 2 * d);
-            const float qv = ld_bf16(stg + STG_Q + stg_row(r) + 2 * d);
-            lk[i] = kv * e;
-            lq[i] = p.scale * qv * e;
+        for (int i = 0; i < 8; i += 2) {
+            float e[2], kv[2], qv[2];
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const int r = 16 * hf + 8 * u + i + t;
+                const float m = fminf(fmaxf(pr[8 * u + i + t], kMinScale), 1.f / kMinScale);
+                const float rm = ptx::rcp(m);
+                e[t] = hf ? m : rm;
+                ie[8 * u + i + t] = hf ? rm : m;
+                kv[t] = ld_bf16(stg + STG_K + stg_row(r) + 2 * d);
+                qv[t] = ld_bf16(stg + STG_Q + stg_row(r) + 2 * d);
+            }
+            const uint64_t e2 = ptx::pk2(e[0], e[1]);
+            ptx::upk2(ptx::mul2(ptx::pk2(kv[0], kv[1]), e2), lk[i], lk[i + 1]);
+            ptx::upk2(ptx::mul2(ptx::mul2(ptx::pk2(qv[0], qv[1]), scale2), e2), lq[i], lq[i + 1]);
         }
         st_split8(lqr + dm(SL_LK + 2 * (2 * hf + u), d, 0), SLAB, lk);
         st_split8(lqr + dm(SL_LQ + 2 * (2 * hf + u), d, 0), SLAB, lq);
@@ -755,10 +762,10 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
 #pragma unroll
                 for (int i4 = 0; i4 < 8; ++i4) {
                     const float4 ff = f4[i4];
-                    v[4 * i4 + 0] *= ff.x;
-                    v[4 * i4 + 1] *= ff.y;
-                    v[4 * i4 + 2] *= ff.z;
-                    v[4 * i4 + 3] *= ff.w;
+                    ptx::upk2(ptx::mul2(ptx::pk2(v[4 * i4], v[4 * i4 + 1]), ptx::pk2(ff.x, ff.y)), v[4 * i4],
+                              v[4 * i4 + 1]);
+                    ptx::upk2(ptx::mul2(ptx::pk2(v[4 * i4 + 2], v[4 * i4 + 3]), ptx::pk2(ff.z, ff.w)), v[4 * i4 + 2],
+                              v[4 * i4 + 3]);
                 }
                 ptx::tmem_st32(tmem + lane_base + TM_S + d0, v);
                 uint32_t hw[16], lw[16];
