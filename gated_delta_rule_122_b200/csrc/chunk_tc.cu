@@ -276,9 +276,8 @@ __device__ __forceinline__ void issue_m2(uint8_t *sm, uint32_t tmem, const Bars 
     ptx::mma_commit(bars.w);
 }
 
-// Readiness of each group: M1(n) needs Lk, Lq, R of chunk n (rc), A(n-1) read (ra)
-// and M2(n-1) issued (an M1 issued ahead of a ready M2 would hold the prep warps
-// up for its whole issue time); M2(n) needs T' and A_qk (rg; the prep warps signal it after reading
+// Readiness of each group: M1(n) needs Lk, Lq, R of chunk n (rc) and A(n-1) read
+// (ra), so it runs while the prep warps solve chunk n-1; M2(n) needs T' and A_qk (rg; the prep warps signal it after reading
 // W'(n-1)) and M4(n-1) issued, since U goes into TM_E; M3(n) needs S'(n) (rs,
 // whose first count is the initial state) and -W'(n) (rj); M4(n) needs E^T(n) (re).
 __device__ void issuer(uint8_t *sm, uint32_t tmem, const Bars &bars, int nchunks, volatile int *err_flag)
@@ -304,7 +303,7 @@ __device__ void issuer(uint8_t *sm, uint32_t tmem, const Bars &bars, int nchunks
             g = 4;
         else if (n2 < n1 && n2 <= n4 && c_rg >= (uint32_t)(NPW * (n2 + 1)))
             g = 2;
-        else if (n1 < nchunks && n1 == n2 && c_ra >= (uint32_t)(NPW * n1) && c_rc >= (uint32_t)(NCW * (n1 + 1)))
+        else if (n1 < nchunks && c_ra >= (uint32_t)(NPW * n1) && c_rc >= (uint32_t)(NCW * (n1 + 1)))
             g = 1;
         if (g != 0) {
             // acquire the producers' writes (the counters only grow)
@@ -735,6 +734,12 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
         // ---- I: X = S' + E^T R -> the next S' (or the final state); outputs of chunk c
         if (!ptx::mbar_wait(bars.s, (uint32_t)(c & 1), kWaitLimitNs)) *err_flag = 1;
         ptx::tc_fence_after();
+        // R of chunk c+2 first (the update of chunk c has read R(c)): the A product of
+        // chunk c+2 can then start while the state is rewritten
+        if (c + 2 < nchunks) {
+            stage_b(sm, c + 2, warp, lane, ie);
+            warp_signal_after_stage(bars, lane);
+        }
         float ov[16];
         {
             float v0[16], v1[16];
@@ -808,11 +813,6 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
 #pragma unroll
                 for (int i = 0; i < 16; ++i) *reinterpret_cast<float *>(tile + i * D * 4) = ov[i];
             }
-        }
-        // R of chunk c+2 (the update of chunk c has read R(c))
-        if (c + 2 < nchunks) {
-            stage_b(sm, c + 2, warp, lane, ie);
-            warp_signal_after_stage(bars, lane);
         }
         ptx::fence_proxy_async_smem();
         const bool stop = chain_bar_err(err_flag);   // output tile written, staging rows consumed
