@@ -34,9 +34,21 @@ if ROOT not in sys.path:
 METRIC = "KDA prefill Mtokens/s (H=64,d=128); decode-step HBM GB/s vs ~8 TB/s peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of the prefill
-# kernel, from the capture summarised under profiles/ (None until taken for the
-# kernel as it stands).
-PREFILL_TRAFFIC_BYTES = None
+# kernel (1.08 GB read + 0.509 GB written), from the capture summarised under
+# profiles/, with the hash of the kernel sources it was taken for: once the
+# sources change, the line reports traffic as null until it is captured again.
+PREFILL_TRAFFIC_BYTES = 1_589_000_000
+PREFILL_TRAFFIC_SOURCES = "8b257c2abe040c77"
+
+
+def kernel_sources_hash() -> str:
+    import hashlib
+    csrc = os.path.join(ROOT, "gated_delta_rule_122_b200", "csrc")
+    h = hashlib.sha256()
+    for name in ("chunk_tc.cu", "tc_ptx.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def parse_args():
@@ -367,7 +379,7 @@ def main():
     if rank != 0:
         return
     headline = args.prefill_seqs is None and args.prefill_len is None
-    traffic = PREFILL_TRAFFIC_BYTES if headline else None
+    traffic = PREFILL_TRAFFIC_BYTES if headline and kernel_sources_hash() == PREFILL_TRAFFIC_SOURCES else None
     workload_desc = (f"prefill B={wp.B * world} H={wp.H} T={wp.T} d_k=d_v={wp.dk} bf16 q/k/v/alpha/beta, "
                      "fp32 o and state")
     if args.only != "prefill":
