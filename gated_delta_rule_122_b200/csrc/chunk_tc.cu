@@ -370,7 +370,7 @@ __device__ __forceinline__ void solve_diag_blocks(const float *At, float *Tm, in
 // Part A only touches slabs the A product (M1), the W'/U product (M2) and the O/E
 // product (M3) of the chunk two back have finished with, so it can run while that
 // chunk's state update (M4) still reads R.
-__device__ void stage_a(const ChunkArgs &p, uint8_t *sm, int n, int warp, int lane, float (&ie)[16])
+__device__ void stage_a(const ChunkArgs &p, uint8_t *sm, int n, int warp, int lane, uint32_t (&rw)[16])
 {
     const int hf = warp >> 2, d = 32 * (warp & 3) + lane;
     const int Lc = min(C, p.T - n * C);
@@ -402,7 +402,7 @@ __device__ void stage_a(const ChunkArgs &p, uint8_t *sm, int n, int warp, int la
     }
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-        float lk[8], lq[8];
+        float lk[8], lq[8], ie[8];
         const uint64_t scale2 = ptx::pk2(p.scale, p.scale);
 #pragma unroll
         for (int i = 0; i < 8; i += 2) {
@@ -413,30 +413,32 @@ __device__ void stage_a(const ChunkArgs &p, uint8_t *sm, int n, int warp, int la
                 const float m = fminf(fmaxf(pr[8 * u + i + t], kMinScale), 1.f / kMinScale);
                 const float rm = ptx::rcp(m);
                 e[t] = hf ? m : rm;
-                ie[8 * u + i + t] = hf ? rm : m;
+                ie[i + t] = hf ? rm : m;
                 kv[t] = ld_bf16(stg + STG_K + stg_row(r) + 2 * d);
                 qv[t] = ld_bf16(stg + STG_Q + stg_row(r) + 2 * d);
             }
             const uint64_t e2 = ptx::pk2(e[0], e[1]);
             ptx::upk2(ptx::mul2(ptx::pk2(kv[0], kv[1]), e2), lk[i], lk[i + 1]);
             ptx::upk2(ptx::mul2(ptx::mul2(ptx::pk2(qv[0], qv[1]), scale2), e2), lq[i], lq[i + 1]);
+            // R = K/e, kept split (hi words, lo words) until its slabs are free
+            float r0, r1;
+            ptx::upk2(ptx::mul2(ptx::pk2(kv[0], kv[1]), ptx::pk2(ie[i], ie[i + 1])), r0, r1);
+            split_pair(r0, r1, rw[8 * u + i / 2], rw[8 * u + 4 + i / 2]);
         }
         st_split8(lqr + dm(SL_LK + 2 * (2 * hf + u), d, 0), SLAB, lk);
         st_split8(lqr + dm(SL_LQ + 2 * (2 * hf + u), d, 0), SLAB, lq);
     }
 }
 
-__device__ void stage_b(uint8_t *sm, int n, int warp, int lane, const float (&ie)[16])
+__device__ void stage_b(uint8_t *sm, int n, int warp, int lane, const uint32_t (&rw)[16])
 {
     const int hf = warp >> 2, d = 32 * (warp & 3) + lane;
     uint8_t *lqr = sm + OFF_LQR + (n & 1) * LQR_BYTES;
-    const uint8_t *stg = sm + OFF_STG;
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-        float rk[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) rk[i] = ld_bf16(stg + STG_K + stg_row(16 * hf + 8 * u + i) + 2 * d) * ie[8 * u + i];
-        st_split8(lqr + dm(SL_R + 2 * (2 * hf + u), d, 0), SLAB, rk);
+        uint8_t *dst = lqr + dm(SL_R + 2 * (2 * hf + u), d, 0);
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(rw[8 * u], rw[8 * u + 1], rw[8 * u + 2], rw[8 * u + 3]);
+        *reinterpret_cast<uint4 *>(dst + SLAB) = make_uint4(rw[8 * u + 4], rw[8 * u + 5], rw[8 * u + 6], rw[8 * u + 7]);
     }
 }
 
@@ -639,7 +641,7 @@ __device__ __forceinline__ void write_state16(uint32_t tmem, uint32_t lane_base,
 // Chain warps, operands of chunk n (the staging rows must hold chunk n): part A,
 // then (later) part B, the signal to the issuer and the loads of chunk n+1.
 __device__ __forceinline__ void chain_stage_a(const ChunkArgs &p, uint8_t *sm, const Bars &bars, int n, int warp,
-                                              int lane, float (&ie)[16], volatile int *err_flag)
+                                              int lane, uint32_t (&ie)[16], volatile int *err_flag)
 {
     if (!ptx::mbar_wait(bars.stg, (uint32_t)(n & 1), kWaitLimitNs)) *err_flag = 1;   // chunk n's rows
     stage_a(p, sm, n, warp, lane, ie);
@@ -647,7 +649,7 @@ __device__ __forceinline__ void chain_stage_a(const ChunkArgs &p, uint8_t *sm, c
 
 __device__ __forceinline__ void chain_stage_b(const TcMaps &maps, uint8_t *sm, const Bars &bars, int b, int h,
                                               int n, int nchunks, int tid, int warp, int lane,
-                                              const float (&ie)[16])
+                                              const uint32_t (&ie)[16])
 {
     stage_b(sm, n, warp, lane, ie);
     ptx::fence_proxy_async_smem();
@@ -673,7 +675,7 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
     const int j = quad * 32 + lane;            // value channel = TMEM lane
     const size_t tile = (size_t)bh * D * D;
 
-    float ie[16];   // 1/e of the chunk being staged, carried from part A to part B
+    uint32_t ie[16];   // R of the chunk being staged (split words), carried from part A to part B
     if (tid == 0) load_qka(maps, sm, bars, b, h, 0);
     int staged = 0;   // chunks whose rows have been waited for
     chain_stage_a(p, sm, bars, 0, warp, lane, ie, err_flag);
