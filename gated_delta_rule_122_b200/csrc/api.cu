@@ -103,6 +103,7 @@ kda_status kda_workspace_status(const void *workspace, cudaStream_t stream)
     if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
         cudaStreamSynchronize(stream) != cudaSuccess)
         return KDA_ERR_LAUNCH;
+    if (word & 2u) return KDA_ERR_SHAPE;     // invalid sequence offsets (packed layout)
     return word ? KDA_ERR_TIMEOUT : KDA_OK;
 }
 
@@ -124,6 +125,48 @@ kda_status kda_forward(const void *q, const void *k, const void *v, const void *
     kda::ChunkArgs a{q, k, v, alpha, beta, initial_state, final_state, o, B, T, H, scale,
                      qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16,
                      static_cast<unsigned int *>(workspace)};
+    cudaError_t err;
+    if (kda::chunk_tc_supported(d_k, d_v, qkv_dtype, gate_dtype))
+        err = kda::launch_chunk_tc(a, d_k, d_v, stream);
+    else
+        err = kda::launch_chunk_simt(a, d_k, d_v, stream);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+}
+
+kda_status kda_forward_varlen(const void *q, const void *k, const void *v, const void *alpha,
+                              const void *beta, const int *cu_seqlens, const float *initial_state,
+                              void *o, float *final_state, int N, int total_T, int H, int d_k,
+                              int d_v, float scale, kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                              kda_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                              cudaStream_t stream)
+{
+    if (N < 0) return KDA_ERR_SHAPE;
+    // the token tensors are one [1, total_T, H, d] batch; the states are per sequence
+    kda_status st = check_forward(q, k, v, alpha, beta, nullptr, o, nullptr, 1, total_T, H, d_k, d_v,
+                                  qkv_dtype, gate_dtype, out_dtype);
+    if (st != KDA_OK) return st;
+    if (N * (long long)H == 0) return KDA_OK;
+    if (!cu_seqlens) return KDA_ERR_NULL;
+    if (!aligned_to(cu_seqlens, sizeof(int)) || !aligned16(initial_state) || !aligned16(final_state))
+        return KDA_ERR_ALIGN;
+    if ((unsigned long long)N * H * d_k * d_v >= (1ull << 60)) return KDA_ERR_SHAPE;
+    if (total_T > 0) {
+        const size_t state_bytes = (size_t)N * H * d_k * d_v * 4;
+        const Range ro = range_of(o, (size_t)total_T * H * d_v * dsize(out_dtype));
+        if (overlap(ro, range_of(initial_state, initial_state ? state_bytes : 0)) ||
+            overlap(ro, range_of(final_state, final_state ? state_bytes : 0)) ||
+            overlap(ro, range_of(cu_seqlens, (size_t)(N + 1) * sizeof(int))))
+            return KDA_ERR_ALIAS;
+    }
+    const size_t need = kda_forward_workspace_bytes(N, total_T, H, d_k, d_v);
+    if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return KDA_ERR_ALIGN;
+    if (cudaMemsetAsync(workspace, 0, need, stream) != cudaSuccess) return KDA_ERR_LAUNCH;
+    // no tokens at all: every sequence is empty (the offsets are all zero)
+    if (total_T == 0) return empty_sequence(initial_state, final_state, N, H, d_k, d_v, stream);
+    kda::ChunkArgs a{q, k, v, alpha, beta, initial_state, final_state, o, N, total_T, H, scale,
+                     qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16,
+                     static_cast<unsigned int *>(workspace), cu_seqlens};
     cudaError_t err;
     if (kda::chunk_tc_supported(d_k, d_v, qkv_dtype, gate_dtype))
         err = kda::launch_chunk_tc(a, d_k, d_v, stream);

@@ -45,7 +45,7 @@ struct SimtLayout {
 
 template <int DK, int DV>
 __global__ void __launch_bounds__(kSimtThreads)
-kda_chunk_simt_kernel(ChunkArgs a)
+kda_chunk_simt_kernel(ChunkArgs ain)
 {
     using Ly = SimtLayout<DK, DV>;
     constexpr int C = Ly::C, PK = Ly::PK, PV = Ly::PV, PC = Ly::PC, NT = kSimtThreads;
@@ -59,10 +59,17 @@ kda_chunk_simt_kernel(ChunkArgs a)
     float *V = sm + Ly::oV, *E = sm + Ly::oE, *S = sm + Ly::oS;
     float *Akk = sm + Ly::oAkk, *Aqk = sm + Ly::oAqk, *Bt = sm + Ly::oBeta;
 
-    const int bh = blockIdx.x;
-    const int b = bh / a.H, h = bh % a.H;
+    const int bh = blockIdx.x;                 // sequence * H + head (state tile)
+    const int h = bh % ain.H;
     const int tid = threadIdx.x;
     const size_t tile = (size_t)bh * DK * DV;
+    // the sequence's own rows (packed layout) as a batch of one
+    ChunkArgs a;
+    int b, row0;
+    if (!sequence_view(ain, bh / ain.H, DK, DV, a, b, row0)) {
+        if (tid == 0 && ain.status) atomicOr(ain.status, 2u);
+        return;
+    }
 
     for (int idx = tid; idx < DK * DV; idx += NT)
         S[idx] = a.s_in ? a.s_in[tile + idx] : 0.f;

@@ -414,8 +414,9 @@ __device__ void stage_a(const ChunkArgs &p, uint8_t *sm, int n, int warp, int la
                 const float rm = ptx::rcp(m);
                 e[t] = hf ? m : rm;
                 ie[i + t] = hf ? rm : m;
-                kv[t] = ld_bf16(stg + STG_K + stg_row(r) + 2 * d);
-                qv[t] = ld_bf16(stg + STG_Q + stg_row(r) + 2 * d);
+                // rows past the sequence's end: zero (the staging may hold another sequence's rows)
+                kv[t] = (r < Lc) ? ld_bf16(stg + STG_K + stg_row(r) + 2 * d) : 0.f;
+                qv[t] = (r < Lc) ? ld_bf16(stg + STG_Q + stg_row(r) + 2 * d) : 0.f;
             }
             const uint64_t e2 = ptx::pk2(e[0], e[1]);
             ptx::upk2(ptx::mul2(ptx::pk2(kv[0], kv[1]), e2), lk[i], lk[i + 1]);
@@ -442,22 +443,29 @@ __device__ void stage_b(uint8_t *sm, int n, int warp, int lane, const uint32_t (
     }
 }
 
-// TMA loads of chunk n's q, k, alpha rows into the staging rows (one thread).
-__device__ __forceinline__ void load_qka(const TcMaps &maps, uint8_t *sm, const Bars &bars, int b, int h, int n)
+// Where a sequence's rows sit in the tensor maps: batch coordinate b and first token
+// t0 (b = sequence, t0 = 0 for the dense layout; b = 0, t0 = its offset when packed).
+struct TmaPos {
+    int b, h, t0;
+};
+
+// TMA loads of chunk n's q, k, alpha rows into the staging rows (one thread).  Rows
+// past the sequence's end are masked where they are used.
+__device__ __forceinline__ void load_qka(const TcMaps &maps, uint8_t *sm, const Bars &bars, const TmaPos &tp, int n)
 {
     ptx::mbar_arrive_expect_tx(bars.stg, 3 * STG_T);
     const uint32_t dst = ptx::smem_u32(sm + OFF_STG);
-    ptx::tma_load_4d(dst + STG_Q, &maps.q, bars.stg, 0, h, n * C, b);
-    ptx::tma_load_4d(dst + STG_K, &maps.k, bars.stg, 0, h, n * C, b);
-    ptx::tma_load_4d(dst + STG_A, &maps.a, bars.stg, 0, h, n * C, b);
+    ptx::tma_load_4d(dst + STG_Q, &maps.q, bars.stg, 0, tp.h, tp.t0 + n * C, tp.b);
+    ptx::tma_load_4d(dst + STG_K, &maps.k, bars.stg, 0, tp.h, tp.t0 + n * C, tp.b);
+    ptx::tma_load_4d(dst + STG_A, &maps.a, bars.stg, 0, tp.h, tp.t0 + n * C, tp.b);
 }
 
 // TMA load of chunk n's v rows into V buffer n&1 (one thread).
-__device__ __forceinline__ void load_v(const TcMaps &maps, uint8_t *sm, const Bars &bars, int b, int h, int n)
+__device__ __forceinline__ void load_v(const TcMaps &maps, uint8_t *sm, const Bars &bars, const TmaPos &tp, int n)
 {
     const uint32_t bar = bars.v + 8 * (n & 1);
     ptx::mbar_arrive_expect_tx(bar, V_BYTES);
-    ptx::tma_load_5d(ptx::smem_u32(sm + OFF_V + (n & 1) * V_BYTES), &maps.v, bar, 0, n * C, 0, h, b);
+    ptx::tma_load_5d(ptx::smem_u32(sm + OFF_V + (n & 1) * V_BYTES), &maps.v, bar, 0, tp.t0 + n * C, 0, tp.h, tp.b);
 }
 
 // ---- the prep warps: A readout, the solve, W' readout, V loads ---------------------
@@ -466,7 +474,7 @@ __device__ __forceinline__ void load_v(const TcMaps &maps, uint8_t *sm, const Ba
 // shared memory; warp 1 forms A_kk and solves its diagonal blocks, warp 3 writes
 // A_qk, and all four finish the off-diagonal block of T and write T'.
 __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, uint32_t tmem, const Bars &bars,
-                          int b, int h, int nchunks, volatile int *err_flag)
+                          const TmaPos &tp, int b, int h, int nchunks, volatile int *err_flag)
 {
     const int pt = threadIdx.x - NCT;          // 0..127
     const int pw = pt >> 5, lane = pt & 31;    // warp = TMEM lane quadrant
@@ -483,8 +491,8 @@ __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, u
 
     int v_loaded = 0, v_seen = 0;   // V loads issued (thread pt 0) and waited for
     if (pt == 0) {
-        load_v(maps, sm, bars, b, h, 0);
-        if (nchunks > 1) load_v(maps, sm, bars, b, h, 1);
+        load_v(maps, sm, bars, tp, 0);
+        if (nchunks > 1) load_v(maps, sm, bars, tp, 1);
     }
     v_loaded = nchunks > 1 ? 2 : 1;
     float beta = (pw < 2) ? load_beta(p, b, h, 0, r) : 0.f;   // beta of row r
@@ -519,6 +527,17 @@ __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, u
         // V(cn) has landed (every warp observes it before it signals M2's readiness)
         if (!ptx::mbar_wait(bars.v + 8 * (cn & 1), (uint32_t)((cn >> 1) & 1), kWaitLimitNs)) *err_flag = 1;
         v_seen = cn + 1;
+        if (p.T - cn * C < C) {
+            // rows past the sequence's end hold zeros (dense layout) or the next
+            // sequence's tokens (packed): clear them, T' does not see them anyway
+            const int Lc = p.T - cn * C;
+            uint8_t *vb = sm + OFF_V + (cn & 1) * V_BYTES;
+            for (int i = pt; i < (C - Lc) * (D / 8); i += NPT) {
+                const int r = Lc + i / (D / 8), jb = i % (D / 8);
+                *reinterpret_cast<uint4 *>(vb + mnmaj(8 * jb, r, C)) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            ptx::fence_proxy_async_smem();
+        }
         if (pw < 2) {
             // A_kk^T: row r of A_kk scaled by beta_r, strictly lower
 #pragma unroll
@@ -609,7 +628,7 @@ __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, u
         warp_signal(bars.rj, lane);
         // M2(cn) has completed: its V buffer can take chunk cn+2
         if (cn + 2 < nchunks) {
-            if (pt == 0) load_v(maps, sm, bars, b, h, cn + 2);
+            if (pt == 0) load_v(maps, sm, bars, tp, cn + 2);
             v_loaded = cn + 3;
         }
         if (stop) break;
@@ -647,7 +666,7 @@ __device__ __forceinline__ void chain_stage_a(const ChunkArgs &p, uint8_t *sm, c
     stage_a(p, sm, n, warp, lane, ie);
 }
 
-__device__ __forceinline__ void chain_stage_b(const TcMaps &maps, uint8_t *sm, const Bars &bars, int b, int h,
+__device__ __forceinline__ void chain_stage_b(const TcMaps &maps, uint8_t *sm, const Bars &bars, const TmaPos &tp,
                                               int n, int nchunks, int tid, int warp, int lane,
                                               const uint32_t (&ie)[16])
 {
@@ -655,7 +674,7 @@ __device__ __forceinline__ void chain_stage_b(const TcMaps &maps, uint8_t *sm, c
     ptx::fence_proxy_async_smem();
     warp_signal(bars.rc, lane);
     chain_bar();   // staging consumed, constants visible to every chain warp
-    if (tid == 0 && n + 1 < nchunks) load_qka(maps, sm, bars, b, h, n + 1);
+    if (tid == 0 && n + 1 < nchunks) load_qka(maps, sm, bars, tp, n + 1);
 }
 
 __device__ __forceinline__ void warp_signal_after_stage(const Bars &bars, int lane)
@@ -666,7 +685,7 @@ __device__ __forceinline__ void warp_signal_after_stage(const Bars &bars, int la
 
 // ---- the chain warps: the serial recurrence over chunks --------------------------------
 __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, uint32_t tmem, const Bars &bars,
-                           int b, int h, int bh, int nchunks, volatile int *err_flag)
+                           const TmaPos &tp, int b, int h, int bh, int nchunks, volatile int *err_flag)
 {
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -676,11 +695,11 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
     const size_t tile = (size_t)bh * D * D;
 
     uint32_t ie[16];   // R of the chunk being staged (split words), carried from part A to part B
-    if (tid == 0) load_qka(maps, sm, bars, b, h, 0);
+    if (tid == 0) load_qka(maps, sm, bars, tp, 0);
     int staged = 0;   // chunks whose rows have been waited for
     chain_stage_a(p, sm, bars, 0, warp, lane, ie, err_flag);
     staged = 1;
-    chain_stage_b(maps, sm, bars, b, h, 0, nchunks, tid, warp, lane, ie);
+    chain_stage_b(maps, sm, bars, tp, 0, nchunks, tid, warp, lane, ie);
 
     // S'_0 = Diag(exp(a_0)) S_0; cleared O accumulator
     {
@@ -702,7 +721,7 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
     if (nchunks > 1) {
         chain_stage_a(p, sm, bars, 1, warp, lane, ie, err_flag);
         staged = 2;
-        chain_stage_b(maps, sm, bars, b, h, 1, nchunks, tid, warp, lane, ie);
+        chain_stage_b(maps, sm, bars, tp, 1, nchunks, tid, warp, lane, ie);
     }
 
     for (int c = 0; c < nchunks; ++c) {
@@ -804,7 +823,8 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
             if (tid == 0) ptx::bulk_wait_read();
             chain_bar();
         }
-        {
+        const bool full = (c + 1) * C <= p.T;
+        if (full) {
             const int esz = p.out_bf16 ? 2 : 4;
             uint8_t *tile = sm + OFF_STG + (half ? STG_A : STG_Q) + j * esz;
             if (p.out_bf16) {
@@ -815,16 +835,26 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
 #pragma unroll
                 for (int i = 0; i < 16; ++i) *reinterpret_cast<float *>(tile + i * D * 4) = ov[i];
             }
+        } else {
+            // the sequence's last, partial chunk: only its own rows, one element per row
+            // (a TMA box would also cover rows that belong to the next sequence)
+            const size_t step = (size_t)p.H * D;
+            size_t idx = (((size_t)b * p.T + c * C + 16 * half) * p.H + h) * D + j;
+#pragma unroll
+            for (int i = 0; i < 16; ++i, idx += step)
+                if (c * C + 16 * half + i < p.T) st_elem(p.o, idx, ov[i], p.out_bf16);
         }
         ptx::fence_proxy_async_smem();
         const bool stop = chain_bar_err(err_flag);   // output tile written, staging rows consumed
         if (tid == 0) {
-            ptx::tma_store_4d(&maps.o, ptx::smem_u32(sm + OFF_STG + STG_Q), 0, h, c * C, b);
-            if (c * C + 16 < p.T) ptx::tma_store_4d(&maps.o, ptx::smem_u32(sm + OFF_STG + STG_A), 0, h, c * C + 16, b);
+            if (full) {
+                ptx::tma_store_4d(&maps.o, ptx::smem_u32(sm + OFF_STG + STG_Q), 0, h, tp.t0 + c * C, tp.b);
+                ptx::tma_store_4d(&maps.o, ptx::smem_u32(sm + OFF_STG + STG_A), 0, h, tp.t0 + c * C + 16, tp.b);
+            }
             ptx::bulk_commit();
             if (c + 3 < nchunks) {
                 ptx::bulk_wait_read();   // the tile has been read: the staging rows can be refilled
-                load_qka(maps, sm, bars, b, h, c + 3);
+                load_qka(maps, sm, bars, tp, c + 3);
             }
         }
         if (stop) break;
@@ -835,14 +865,29 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
     if (tid == 0) ptx::bulk_wait();   // the output stores are complete
 }
 
-__global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs p, const __grid_constant__ TcMaps maps)
+__global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs pa, const __grid_constant__ TcMaps maps)
 {
     extern __shared__ __align__(1024) uint8_t sm[];
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.x;
-    const int b = bh / p.H, h = bh % p.H;
+    const int bh = blockIdx.x;                 // sequence * H + head (state tile)
+    const int h = bh % pa.H;
+    ChunkArgs p;
+    int b, row0;                               // batch index within the view, first token row
+    if (!sequence_view(pa, bh / pa.H, D, D, p, b, row0)) {
+        if (tid == 0 && pa.status) atomicOr(pa.status, 2u);
+        return;
+    }
+    const TmaPos tp{pa.cu_seqlens ? 0 : b, h, row0};
     const int nchunks = (p.T + C - 1) / C;
+    if (nchunks == 0) {
+        // an empty sequence: the final state is the initial one (or zeros)
+        if (p.s_out) {
+            const size_t tile = (size_t)bh * D * D;
+            for (int i = tid; i < D * D; i += NT) p.s_out[tile + i] = p.s_in ? p.s_in[tile + i] : 0.f;
+        }
+        return;
+    }
 
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC);
     volatile int *err_flag = reinterpret_cast<volatile int *>(sm + OFF_MISC + 4);
@@ -879,9 +924,9 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs p, const 
     if (warp == kIssuerWarp) {
         if (lane == 0) issuer(sm, tmem, bars, nchunks, err_flag);
     } else if (warp >= NCW) {
-        prep_role(p, maps, sm, tmem, bars, b, h, nchunks, err_flag);
+        prep_role(p, maps, sm, tmem, bars, tp, b, h, nchunks, err_flag);
     } else {
-        chain_role(p, maps, sm, tmem, bars, b, h, bh, nchunks, err_flag);
+        chain_role(p, maps, sm, tmem, bars, tp, b, h, bh, nchunks, err_flag);
     }
     if (*err_flag && tid == 0 && p.status) atomicOr(p.status, 1u);
     ptx::tc_fence_before();
@@ -966,9 +1011,10 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, int dk, int dv, cudaStream_t str
     if (blocks == 0) return cudaSuccess;
     if (encode_fn() == nullptr) return cudaErrorNotSupported;
     tc::TcMaps maps;
-    if (!encode_rows(&maps.q, a.q, a.B, a.T, a.H) || !encode_rows(&maps.k, a.k, a.B, a.T, a.H) ||
-        !encode_rows(&maps.a, a.alpha, a.B, a.T, a.H) || !encode_v(&maps.v, a.v, a.B, a.T, a.H) ||
-        !encode_out(&maps.o, a.o, a.B, a.T, a.H, a.out_bf16))
+    const int mb = a.cu_seqlens ? 1 : a.B;   // packed sequences: one [1, T, H, d] tensor
+    if (!encode_rows(&maps.q, a.q, mb, a.T, a.H) || !encode_rows(&maps.k, a.k, mb, a.T, a.H) ||
+        !encode_rows(&maps.a, a.alpha, mb, a.T, a.H) || !encode_v(&maps.v, a.v, mb, a.T, a.H) ||
+        !encode_out(&maps.o, a.o, mb, a.T, a.H, a.out_bf16))
         return cudaErrorInvalidValue;
     cudaError_t err = cudaFuncSetAttribute(tc::kda_chunk_tc_kernel,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);

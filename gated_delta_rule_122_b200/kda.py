@@ -15,8 +15,8 @@ import threading
 
 import torch
 
-__all__ = ["KDAError", "forward", "forward_sequential", "decode_step", "library", "library_path",
-           "status_string", "version", "EXPORTED_SYMBOLS"]
+__all__ = ["KDAError", "forward", "forward_varlen", "forward_sequential", "decode_step", "library",
+           "library_path", "status_string", "version", "EXPORTED_SYMBOLS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libkda_b200.so")
@@ -24,8 +24,8 @@ _lib = None
 _lock = threading.Lock()
 
 EXPORTED_SYMBOLS = ("kda_forward", "kda_forward_workspace_bytes", "kda_workspace_status",
-                    "kda_forward_noalloc", "kda_forward_sequential", "kda_decode_step",
-                    "kda_status_string", "kda_version")
+                    "kda_forward_noalloc", "kda_forward_varlen", "kda_forward_sequential",
+                    "kda_decode_step", "kda_status_string", "kda_version")
 
 _DT = {torch.float32: 0, torch.bfloat16: 1}
 _vp = ctypes.c_void_p
@@ -61,6 +61,9 @@ def library() -> ctypes.CDLL:
             lib.kda_forward_sequential.restype = _i
             lib.kda_forward_noalloc.argtypes = fwd_args + [_vp]
             lib.kda_forward_noalloc.restype = _i
+            lib.kda_forward_varlen.argtypes = [_vp] * 9 + [_i] * 5 + [_f] + [_i] * 3 + \
+                [_vp, ctypes.c_size_t, _vp]
+            lib.kda_forward_varlen.restype = _i
             lib.kda_forward_workspace_bytes.argtypes = [_i] * 5
             lib.kda_forward_workspace_bytes.restype = ctypes.c_size_t
             lib.kda_workspace_status.argtypes = [_vp, _vp]
@@ -239,3 +242,66 @@ def decode_step(q, k, v, alpha, beta, state, scale=None, out_dtype=torch.float32
     if code != 0:
         raise KDAError("kda_decode_step", code)
     return out
+
+
+def forward_varlen(q, k, v, alpha, beta, cu_seqlens, initial_state=None, scale=None,
+                   output_final_state=True, out_dtype=torch.float32, out=None, final_state=None,
+                   workspace=None, check_status=False):
+    """Prefill over packed sequences of different lengths (C entry point ``kda_forward_varlen``).
+
+    q, k, alpha: [total_T,H,dk] (or [1,total_T,H,dk]); v: [total_T,H,dv]; beta: [total_T,H];
+    cu_seqlens: int32 [N+1] on the same device (0, then cumulative lengths).  initial_state:
+    float32 [N,H,dk,dv] or None.  check_status=True synchronizes and raises KDAError on
+    invalid offsets or a timed-out device wait.  Returns (o [total_T,H,dv], final_state or None).
+    """
+    device = q.device
+    if device.type != "cuda":
+        raise ValueError("KDA runs on CUDA devices only")
+    squeeze = q.dim() == 4
+    if squeeze:
+        if q.shape[0] != 1:
+            raise ValueError("packed tensors are [total_T,H,d] or [1,total_T,H,d]")
+        q, k, v, alpha, beta = (t[0] for t in (q, k, v, alpha, beta))
+    total_T, H, dk = q.shape
+    dv = v.shape[-1]
+    for name, t in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta", beta),
+                    ("cu_seqlens", cu_seqlens)):
+        _check(name, t, device)
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
+        raise ValueError("cu_seqlens must be a 1-D int32 tensor [N+1]")
+    N = cu_seqlens.numel() - 1
+    if tuple(k.shape) != (total_T, H, dk) or tuple(alpha.shape) != (total_T, H, dk) or \
+            tuple(v.shape) != (total_T, H, dv) or tuple(beta.shape) != (total_T, H):
+        raise ValueError("shapes: q,k,alpha [total_T,H,dk], v [total_T,H,dv], beta [total_T,H]")
+    if k.dtype != q.dtype or v.dtype != q.dtype or alpha.dtype != beta.dtype:
+        raise TypeError("q/k/v and alpha/beta must each share a dtype")
+    if initial_state is not None:
+        _check("initial_state", initial_state, device)
+        if initial_state.dtype != torch.float32 or tuple(initial_state.shape) != (N, H, dk, dv):
+            raise ValueError("initial_state must be float32 [N,H,dk,dv]")
+    if scale is None:
+        scale = dk ** -0.5
+    if out is None:
+        out = torch.empty((total_T, H, dv), device=device, dtype=out_dtype)
+    _check("out", out, device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((N, H, dk, dv), device=device, dtype=torch.float32)
+    if final_state is not None:
+        _check("final_state", final_state, device)
+    lib = library()
+    with torch.cuda.device(device):
+        stream = _vp(_stream_handle(device))
+        ws_bytes = lib.kda_forward_workspace_bytes(N, total_T, H, dk, dv)
+        ws = workspace
+        if ws is None or ws.numel() * ws.element_size() < ws_bytes:
+            ws = torch.empty(max(ws_bytes, 16), device=device, dtype=torch.uint8)
+        code = lib.kda_forward_varlen(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(cu_seqlens),
+            _ptr(initial_state), _ptr(out), _ptr(final_state), N, total_T, H, dk, dv,
+            float(scale), _DT[q.dtype], _dt(alpha, "alpha"), _dt(out, "out"), _ptr(ws),
+            ws.numel() * ws.element_size(), stream)
+        if code == 0 and check_status:
+            code = lib.kda_workspace_status(_ptr(ws), stream)
+    if code != 0:
+        raise KDAError("kda_forward_varlen", code)
+    return (out.unsqueeze(0) if squeeze else out), final_state

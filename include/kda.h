@@ -103,9 +103,10 @@ size_t kda_forward_workspace_bytes(int B, int T, int H, int d_k, int d_v);
 
 /*
  * kda_workspace_status -- synchronize `stream`, then read the status word a
- * kda_forward call left in `workspace`: KDA_OK, or KDA_ERR_TIMEOUT when one of
- * the kernel's bounded waits on its own tensor-core completions gave up (the
- * outputs of that call are then not valid).  KDA_ERR_LAUNCH if the copy or the
+ * kda_forward or kda_forward_varlen call left in `workspace`: KDA_OK,
+ * KDA_ERR_SHAPE when kda_forward_varlen met invalid sequence offsets, or
+ * KDA_ERR_TIMEOUT when one of the kernel's bounded waits on its own tensor-core
+ * completions gave up (the outputs of that call are then not valid).  KDA_ERR_LAUNCH if the copy or the
  * synchronization fails.  Not part of the recurrence; the pages have no
  * counterpart.
  */
@@ -131,6 +132,38 @@ kda_status kda_forward_noalloc(const void *q, const void *k, const void *v,
                                int d_k, int d_v, float scale,
                                kda_dtype qkv_dtype, kda_dtype gate_dtype,
                                kda_dtype out_dtype, cudaStream_t stream);
+
+/*
+ * kda_forward_varlen -- kda_forward over a packed batch of N sequences of
+ * different lengths (the serving layout: no padding between sequences).
+ * Sequence b owns token rows cu_seqlens[b] .. cu_seqlens[b+1]-1; each runs the
+ * recurrence from its own initial state.  Defined by the same passages as
+ * kda_forward.  The state of each sequence is per-request serving state
+ * ("Module 03 -- KDA I: The Delta-Rule Recurrence", jared-hpc.com, section 5,
+ * "State vs. checkpoint weights"); packing requests of different lengths into
+ * one launch is a serving layout, not part of the recurrence.
+ *
+ *   q, k, alpha   [total_T, H, d_k]  (a [1, total_T, H, d_k] batch)
+ *   v, o          [total_T, H, d_v]
+ *   beta          [total_T, H]
+ *   cu_seqlens    DEVICE int32 [N + 1]: 0 = cu_seqlens[0] <= ... <=
+ *                 cu_seqlens[N] <= total_T, 4-byte aligned, owned by the caller
+ *   initial_state [N, H, d_k, d_v] fp32 or NULL; final_state [N, H, d_k, d_v]
+ *                 fp32 or NULL (may equal initial_state)
+ * Other arguments as kda_forward.  The offsets live on the device, so they
+ * are checked by the kernel: a sequence whose offsets are out of order or out
+ * of range is skipped (nothing of it is written) and kda_workspace_status()
+ * then returns KDA_ERR_SHAPE.  An empty sequence copies its initial state (or
+ * zeros) to its final state.  Rows of o outside every sequence are not written.
+ */
+kda_status kda_forward_varlen(const void *q, const void *k, const void *v,
+                              const void *alpha, const void *beta,
+                              const int *cu_seqlens, const float *initial_state,
+                              void *o, float *final_state, int N, int total_T,
+                              int H, int d_k, int d_v, float scale,
+                              kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                              kda_dtype out_dtype, void *workspace,
+                              size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * kda_forward_sequential -- the same operation and arguments as kda_forward
