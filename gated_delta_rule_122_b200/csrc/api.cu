@@ -26,7 +26,7 @@ bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi && a.lo != a.
 kda_status check_forward(const void *q, const void *k, const void *v, const void *alpha,
                          const void *beta, const float *s_in, const void *o, const float *s_out,
                          int B, int T, int H, int dk, int dv, kda_dtype qkv, kda_dtype gate,
-                         kda_dtype out)
+                         kda_dtype out, bool gate_per_head = false)
 {
     if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return KDA_ERR_SHAPE;
     if (!dtype_ok(qkv) || !dtype_ok(gate) || !dtype_ok(out)) return KDA_ERR_DTYPE;
@@ -36,13 +36,16 @@ kda_status check_forward(const void *q, const void *k, const void *v, const void
     if (B * (long long)H == 0) return KDA_OK;
     if (T > 0 && (!q || !k || !v || !alpha || !beta || !o)) return KDA_ERR_NULL;
     // vector tensors: 16-byte aligned rows; beta (one scalar per token): element-aligned
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(alpha) ||
+    // (a per-head alpha, like beta, has one scalar per token)
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) ||
+        !(gate_per_head ? aligned_to(alpha, dsize(gate)) : aligned16(alpha)) ||
         !aligned_to(beta, dsize(gate)) || !aligned16(s_in) || !aligned16(o) || !aligned16(s_out))
         return KDA_ERR_ALIGN;
     if (T > 0) {
         const Range ro = range_of(o, tokens * dv * dsize(out));
         const Range ins[] = {range_of(q, tokens * dk * dsize(qkv)), range_of(k, tokens * dk * dsize(qkv)),
-                             range_of(v, tokens * dv * dsize(qkv)), range_of(alpha, tokens * dk * dsize(gate)),
+                             range_of(v, tokens * dv * dsize(qkv)),
+                             range_of(alpha, tokens * (gate_per_head ? 1 : dk) * dsize(gate)),
                              range_of(beta, tokens * dsize(gate)),
                              range_of(s_in, s_in ? (size_t)B * H * dk * dv * 4 : 0),
                              range_of(s_out, s_out ? (size_t)B * H * dk * dv * 4 : 0)};
@@ -175,6 +178,33 @@ kda_status kda_forward_varlen(const void *q, const void *k, const void *v, const
     return err == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
 }
 
+kda_status kda_forward_scalar_gate(const void *q, const void *k, const void *v, const void *alpha,
+                                   const void *beta, const float *initial_state, void *o,
+                                   float *final_state, int B, int T, int H, int d_k, int d_v,
+                                   float scale, kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                                   kda_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                                   cudaStream_t stream)
+{
+    kda_status st = check_forward(q, k, v, alpha, beta, initial_state, o, final_state, B, T, H,
+                                  d_k, d_v, qkv_dtype, gate_dtype, out_dtype, true);
+    if (st != KDA_OK) return st;
+    if (B * (long long)H == 0) return KDA_OK;
+    const size_t need = kda_forward_workspace_bytes(B, T, H, d_k, d_v);
+    if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return KDA_ERR_ALIGN;
+    if (cudaMemsetAsync(workspace, 0, need, stream) != cudaSuccess) return KDA_ERR_LAUNCH;
+    if (T == 0) return empty_sequence(initial_state, final_state, B, H, d_k, d_v, stream);
+    kda::ChunkArgs a{q, k, v, alpha, beta, initial_state, final_state, o, B, T, H, scale,
+                     qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16,
+                     static_cast<unsigned int *>(workspace), nullptr, 1};
+    cudaError_t err;
+    if (kda::chunk_tc_supported(d_k, d_v, qkv_dtype, gate_dtype))
+        err = kda::launch_chunk_tc(a, d_k, d_v, stream);
+    else
+        err = kda::launch_chunk_simt(a, d_k, d_v, stream);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+}
+
 kda_status kda_forward_sequential(const void *q, const void *k, const void *v, const void *alpha,
                                   const void *beta, const float *initial_state, void *o,
                                   float *final_state, int B, int T, int H, int d_k, int d_v,
@@ -206,6 +236,23 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const vo
     kda::RecurrentArgs a{q, k, v, alpha, beta, state, state, o, N, 1, H, scale,
                          qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16,
                          nullptr};
+    return kda::launch_recurrent(a, d_k, d_v, stream) == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+}
+
+kda_status kda_decode_step_scalar_gate(const void *q, const void *k, const void *v,
+                                       const void *alpha, const void *beta, float *state, void *o,
+                                       int N, int H, int d_k, int d_v, float scale,
+                                       kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                                       kda_dtype out_dtype, cudaStream_t stream)
+{
+    if (N * (long long)H > 0 && !state) return KDA_ERR_NULL;
+    kda_status st = check_forward(q, k, v, alpha, beta, state, o, nullptr, N, 1, H, d_k, d_v,
+                                  qkv_dtype, gate_dtype, out_dtype, true);
+    if (st != KDA_OK) return st;
+    if (N * (long long)H == 0) return KDA_OK;
+    kda::RecurrentArgs a{q, k, v, alpha, beta, state, state, o, N, 1, H, scale,
+                         qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16,
+                         nullptr, nullptr, 1};
     return kda::launch_recurrent(a, d_k, d_v, stream) == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
 }
 

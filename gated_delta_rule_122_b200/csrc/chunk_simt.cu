@@ -86,7 +86,7 @@ kda_chunk_simt_kernel(ChunkArgs ain)
                 const size_t row = ((size_t)b * a.T + t0 + r) * a.H + h;
                 qv = ld_elem(a.q, row * DK + d, a.qkv_bf16);
                 kv = ld_elem(a.k, row * DK + d, a.qkv_bf16);
-                gv = log_alpha(ld_elem(a.alpha, row * DK + d, a.gate_bf16));
+                gv = log_alpha(ld_elem(a.alpha, a.gate_per_head ? row : row * DK + d, a.gate_bf16));
             }
             Q[r * PK + d] = qv; K[r * PK + d] = kv; G[r * PK + d] = gv;
         }

@@ -47,6 +47,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -370,7 +371,8 @@ __device__ __forceinline__ void solve_diag_blocks(const float *At, float *Tm, in
 // Part A only touches slabs the A product (M1), the W'/U product (M2) and the O/E
 // product (M3) of the chunk two back have finished with, so it can run while that
 // chunk's state update (M4) still reads R.
-__device__ void stage_a(const ChunkArgs &p, uint8_t *sm, int n, int warp, int lane, uint32_t (&rw)[16])
+template <bool kHeadGate>
+__device__ void stage_a(const ChunkArgs &p, uint8_t *sm, int b, int h, int n, int warp, int lane, uint32_t (&rw)[16])
 {
     const int hf = warp >> 2, d = 32 * (warp & 3) + lane;
     const int Lc = min(C, p.T - n * C);
@@ -378,13 +380,20 @@ __device__ void stage_a(const ChunkArgs &p, uint8_t *sm, int n, int warp, int la
     float *cst = reinterpret_cast<float *>(sm + OFF_CST + (n % kCstSlots) * CST_BYTES);
     const float *cst_prev = reinterpret_cast<const float *>(sm + OFF_CST + ((n + kCstSlots - 1) % kCstSlots) * CST_BYTES);
     const uint8_t *stg = sm + OFF_STG;
+    // alpha of row r: the staged row's channel d, or with one gate per head, the token's
+    // gate straight from global memory (the same 32 values for every thread)
+    const __nv_bfloat16 *ah = (const __nv_bfloat16 *)p.alpha + ((size_t)b * p.T + (size_t)n * C) * p.H + h;
+    auto alpha_at = [&](int r) {
+        if constexpr (kHeadGate) return __bfloat162float(ah[(size_t)r * p.H]);
+        else return ld_bf16(stg + STG_A + stg_row(r) + 2 * d);
+    };
     float pr[16];
     float acc = 1.f;
     if (hf == 1) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int r = 16 + i;
-            const float x = ld_bf16(stg + STG_A + stg_row(r) + 2 * d);
+            const float x = (r < Lc) ? alpha_at(r) : 1.f;
             acc *= (r < Lc) ? fmaxf(x, kMinAlpha) : 1.f;   // rows past the end: identity steps
             pr[i] = acc;                                     // e_r
         }
@@ -393,7 +402,7 @@ __device__ void stage_a(const ChunkArgs &p, uint8_t *sm, int n, int warp, int la
 #pragma unroll
         for (int i = 15; i >= 0; --i) {
             pr[i] = acc;                                     // 1/e_r
-            const float x = ld_bf16(stg + STG_A + stg_row(i) + 2 * d);
+            const float x = (i < Lc) ? alpha_at(i) : 1.f;
             acc *= (i < Lc) ? fmaxf(x, kMinAlpha) : 1.f;
         }
         const float aexp = fmaxf(acc, kMinScale);           // exp(a)
@@ -447,17 +456,18 @@ __device__ void stage_b(uint8_t *sm, int n, int warp, int lane, const uint32_t (
 // t0 (b = sequence, t0 = 0 for the dense layout; b = 0, t0 = its offset when packed).
 struct TmaPos {
     int b, h, t0;
+    int gate_rows;   // alpha has a row per token (per-key-channel gate) to stage
 };
 
 // TMA loads of chunk n's q, k, alpha rows into the staging rows (one thread).  Rows
 // past the sequence's end are masked where they are used.
 __device__ __forceinline__ void load_qka(const TcMaps &maps, uint8_t *sm, const Bars &bars, const TmaPos &tp, int n)
 {
-    ptx::mbar_arrive_expect_tx(bars.stg, 3 * STG_T);
+    ptx::mbar_arrive_expect_tx(bars.stg, (tp.gate_rows ? 3 : 2) * STG_T);
     const uint32_t dst = ptx::smem_u32(sm + OFF_STG);
     ptx::tma_load_4d(dst + STG_Q, &maps.q, bars.stg, 0, tp.h, tp.t0 + n * C, tp.b);
     ptx::tma_load_4d(dst + STG_K, &maps.k, bars.stg, 0, tp.h, tp.t0 + n * C, tp.b);
-    ptx::tma_load_4d(dst + STG_A, &maps.a, bars.stg, 0, tp.h, tp.t0 + n * C, tp.b);
+    if (tp.gate_rows) ptx::tma_load_4d(dst + STG_A, &maps.a, bars.stg, 0, tp.h, tp.t0 + n * C, tp.b);
 }
 
 // TMA load of chunk n's v rows into V buffer n&1 (one thread).
@@ -659,11 +669,12 @@ __device__ __forceinline__ void write_state16(uint32_t tmem, uint32_t lane_base,
 
 // Chain warps, operands of chunk n (the staging rows must hold chunk n): part A,
 // then (later) part B, the signal to the issuer and the loads of chunk n+1.
-__device__ __forceinline__ void chain_stage_a(const ChunkArgs &p, uint8_t *sm, const Bars &bars, int n, int warp,
+template <bool kHeadGate>
+__device__ __forceinline__ void chain_stage_a(const ChunkArgs &p, uint8_t *sm, const Bars &bars, int b, int h, int n, int warp,
                                               int lane, uint32_t (&ie)[16], volatile int *err_flag)
 {
     if (!ptx::mbar_wait(bars.stg, (uint32_t)(n & 1), kWaitLimitNs)) *err_flag = 1;   // chunk n's rows
-    stage_a(p, sm, n, warp, lane, ie);
+    stage_a<kHeadGate>(p, sm, b, h, n, warp, lane, ie);
 }
 
 __device__ __forceinline__ void chain_stage_b(const TcMaps &maps, uint8_t *sm, const Bars &bars, const TmaPos &tp,
@@ -684,6 +695,7 @@ __device__ __forceinline__ void warp_signal_after_stage(const Bars &bars, int la
 }
 
 // ---- the chain warps: the serial recurrence over chunks --------------------------------
+template <bool kHeadGate>
 __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, uint32_t tmem, const Bars &bars,
                            const TmaPos &tp, int b, int h, int bh, int nchunks, volatile int *err_flag)
 {
@@ -697,7 +709,7 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
     uint32_t ie[16];   // R of the chunk being staged (split words), carried from part A to part B
     if (tid == 0) load_qka(maps, sm, bars, tp, 0);
     int staged = 0;   // chunks whose rows have been waited for
-    chain_stage_a(p, sm, bars, 0, warp, lane, ie, err_flag);
+    chain_stage_a<kHeadGate>(p, sm, bars, b, h, 0, warp, lane, ie, err_flag);
     staged = 1;
     chain_stage_b(maps, sm, bars, tp, 0, nchunks, tid, warp, lane, ie);
 
@@ -719,7 +731,7 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
     ptx::tc_fence_before();
     warp_signal(bars.rs, lane);
     if (nchunks > 1) {
-        chain_stage_a(p, sm, bars, 1, warp, lane, ie, err_flag);
+        chain_stage_a<kHeadGate>(p, sm, bars, b, h, 1, warp, lane, ie, err_flag);
         staged = 2;
         chain_stage_b(maps, sm, bars, tp, 1, nchunks, tid, warp, lane, ie);
     }
@@ -748,7 +760,7 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
         warp_signal(bars.re, lane);
         // Lk, Lq of chunk c+2 while the state update of chunk c runs
         if (c + 2 < nchunks) {
-            chain_stage_a(p, sm, bars, c + 2, warp, lane, ie, err_flag);
+            chain_stage_a<kHeadGate>(p, sm, bars, b, h, c + 2, warp, lane, ie, err_flag);
             staged = c + 3;
         }
 
@@ -865,6 +877,8 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
     if (tid == 0) ptx::bulk_wait();   // the output stores are complete
 }
 
+// kHeadGate: one retention factor per (token, head), alpha [B, T, H] (Gated DeltaNet).
+template <bool kHeadGate>
 __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs pa, const __grid_constant__ TcMaps maps)
 {
     extern __shared__ __align__(1024) uint8_t sm[];
@@ -878,7 +892,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs pa, const
         if (tid == 0 && pa.status) atomicOr(pa.status, 2u);
         return;
     }
-    const TmaPos tp{pa.cu_seqlens ? 0 : b, h, row0};
+    const TmaPos tp{pa.cu_seqlens ? 0 : b, h, row0, pa.gate_per_head ? 0 : 1};
     const int nchunks = (p.T + C - 1) / C;
     if (nchunks == 0) {
         // an empty sequence: the final state is the initial one (or zeros)
@@ -926,7 +940,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs pa, const
     } else if (warp >= NCW) {
         prep_role(p, maps, sm, tmem, bars, tp, b, h, nchunks, err_flag);
     } else {
-        chain_role(p, maps, sm, tmem, bars, tp, b, h, bh, nchunks, err_flag);
+        chain_role<kHeadGate>(p, maps, sm, tmem, bars, tp, b, h, bh, nchunks, err_flag);
     }
     if (*err_flag && tid == 0 && p.status) atomicOr(p.status, 1u);
     ptx::tc_fence_before();
@@ -1012,14 +1026,15 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, int dk, int dv, cudaStream_t str
     if (encode_fn() == nullptr) return cudaErrorNotSupported;
     tc::TcMaps maps;
     const int mb = a.cu_seqlens ? 1 : a.B;   // packed sequences: one [1, T, H, d] tensor
+    if (a.gate_per_head) memset(&maps.a, 0, sizeof(maps.a));   // alpha is read per token instead
     if (!encode_rows(&maps.q, a.q, mb, a.T, a.H) || !encode_rows(&maps.k, a.k, mb, a.T, a.H) ||
-        !encode_rows(&maps.a, a.alpha, mb, a.T, a.H) || !encode_v(&maps.v, a.v, mb, a.T, a.H) ||
+        (!a.gate_per_head && !encode_rows(&maps.a, a.alpha, mb, a.T, a.H)) || !encode_v(&maps.v, a.v, mb, a.T, a.H) ||
         !encode_out(&maps.o, a.o, mb, a.T, a.H, a.out_bf16))
         return cudaErrorInvalidValue;
-    cudaError_t err = cudaFuncSetAttribute(tc::kda_chunk_tc_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
+    auto kernel = a.gate_per_head ? tc::kda_chunk_tc_kernel<true> : tc::kda_chunk_tc_kernel<false>;
+    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
     if (err != cudaSuccess) return err;
-    tc::kda_chunk_tc_kernel<<<(unsigned)blocks, tc::NT, tc::SMEM_BYTES, stream>>>(a, maps);
+    kernel<<<(unsigned)blocks, tc::NT, tc::SMEM_BYTES, stream>>>(a, maps);
     return cudaGetLastError();
 }
 

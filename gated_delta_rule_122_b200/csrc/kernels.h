@@ -22,6 +22,9 @@ struct ChunkArgs {
     // cu_seqlens[b+1]-1 of tensors laid out [1, T, H, d] (T = total tokens).  Null
     // for the dense [B, T, H, d] layout.
     const int *cu_seqlens;
+    // One retention factor per (token, head) -- Gated DeltaNet's scalar gate -- with
+    // alpha laid out [B, T, H]; 0 for the per-key-channel gate [B, T, H, d_k].
+    int gate_per_head;
 };
 
 // The per-sequence view of a launch: with offsets, the sequence's rows are made
@@ -41,7 +44,7 @@ __host__ __device__ inline bool sequence_view(const ChunkArgs &a, int b, int dk,
     s.q = (const char *)a.q + rows * dk * qe;
     s.k = (const char *)a.k + rows * dk * qe;
     s.v = (const char *)a.v + rows * dv * qe;
-    s.alpha = (const char *)a.alpha + rows * dk * ge;
+    s.alpha = (const char *)a.alpha + rows * (a.gate_per_head ? 1 : dk) * ge;
     s.beta = (const char *)a.beta + rows * ge;
     s.o = (char *)a.o + rows * dv * oe;
     s.T = s1 - s0;

@@ -62,7 +62,7 @@ kda_recurrent_kernel(RecurrentArgs a)
         for (int i = tid; i < DK; i += NT) {
             s_q[buf][i] = ld_elem(a.q, row * DK + i, a.qkv_bf16);
             s_k[buf][i] = ld_elem(a.k, row * DK + i, a.qkv_bf16);
-            s_a[buf][i] = ld_elem(a.alpha, row * DK + i, a.gate_bf16);
+            s_a[buf][i] = ld_elem(a.alpha, a.gate_per_head ? row : row * DK + i, a.gate_bf16);
         }
         for (int j = tid; j < DV; j += NT) s_v[buf][j] = ld_elem(a.v, row * DV + j, a.qkv_bf16);
         if (tid == 0) s_beta[buf] = ld_elem(a.beta, row, a.gate_bf16);

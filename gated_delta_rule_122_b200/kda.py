@@ -15,8 +15,9 @@ import threading
 
 import torch
 
-__all__ = ["KDAError", "forward", "forward_varlen", "forward_sequential", "decode_step", "library",
-           "library_path", "status_string", "version", "EXPORTED_SYMBOLS"]
+__all__ = ["KDAError", "forward", "forward_varlen", "forward_scalar_gate", "forward_sequential",
+           "decode_step", "decode_step_scalar_gate", "library", "library_path", "status_string",
+           "version", "EXPORTED_SYMBOLS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libkda_b200.so")
@@ -24,8 +25,9 @@ _lib = None
 _lock = threading.Lock()
 
 EXPORTED_SYMBOLS = ("kda_forward", "kda_forward_workspace_bytes", "kda_workspace_status",
-                    "kda_forward_noalloc", "kda_forward_varlen", "kda_forward_sequential",
-                    "kda_decode_step", "kda_status_string", "kda_version")
+                    "kda_forward_noalloc", "kda_forward_varlen", "kda_forward_scalar_gate",
+                    "kda_forward_sequential", "kda_decode_step", "kda_decode_step_scalar_gate",
+                    "kda_status_string", "kda_version")
 
 _DT = {torch.float32: 0, torch.bfloat16: 1}
 _vp = ctypes.c_void_p
@@ -64,6 +66,10 @@ def library() -> ctypes.CDLL:
             lib.kda_forward_varlen.argtypes = [_vp] * 9 + [_i] * 5 + [_f] + [_i] * 3 + \
                 [_vp, ctypes.c_size_t, _vp]
             lib.kda_forward_varlen.restype = _i
+            lib.kda_forward_scalar_gate.argtypes = fwd_args + [_vp, ctypes.c_size_t, _vp]
+            lib.kda_forward_scalar_gate.restype = _i
+            lib.kda_decode_step_scalar_gate.argtypes = [_vp] * 7 + [_i] * 4 + [_f] + [_i] * 3 + [_vp]
+            lib.kda_decode_step_scalar_gate.restype = _i
             lib.kda_forward_workspace_bytes.argtypes = [_i] * 5
             lib.kda_forward_workspace_bytes.restype = ctypes.c_size_t
             lib.kda_workspace_status.argtypes = [_vp, _vp]
@@ -112,7 +118,7 @@ def _to_device(tensors, device):
 
 
 def _prefill(fn_name, q, k, v, alpha, beta, initial_state, scale, output_final_state,
-             out_dtype, out, final_state, workspace=None, check_status=False):
+             out_dtype, out, final_state, workspace=None, check_status=False, gate_per_head=False):
     host = q.device.type == "cpu"
     host_out = host_state = None
     if host:
@@ -136,9 +142,11 @@ def _prefill(fn_name, q, k, v, alpha, beta, initial_state, scale, output_final_s
         raise TypeError("q, k and v must share a dtype")
     if alpha.dtype != beta.dtype:
         raise TypeError("alpha and beta must share a dtype")
-    if tuple(k.shape) != (B, T, H, dk) or tuple(alpha.shape) != (B, T, H, dk) \
+    a_shape = (B, T, H) if gate_per_head else (B, T, H, dk)
+    if tuple(k.shape) != (B, T, H, dk) or tuple(alpha.shape) != a_shape \
             or tuple(v.shape) != (B, T, H, dv) or tuple(beta.shape) != (B, T, H):
-        raise ValueError("shapes: q,k,alpha [B,T,H,dk], v [B,T,H,dv], beta [B,T,H]")
+        raise ValueError("shapes: q,k [B,T,H,dk], alpha " + ("[B,T,H]" if gate_per_head else "[B,T,H,dk]")
+                         + ", v [B,T,H,dv], beta [B,T,H]")
     if initial_state is not None:
         _check("initial_state", initial_state, device)
         if initial_state.dtype != torch.float32 or tuple(initial_state.shape) != (B, H, dk, dv):
@@ -158,12 +166,12 @@ def _prefill(fn_name, q, k, v, alpha, beta, initial_state, scale, output_final_s
             _dt(out, "out")]
     with torch.cuda.device(device):
         stream = _vp(_stream_handle(device))
-        if fn_name == "kda_forward":
+        if fn_name in ("kda_forward", "kda_forward_scalar_gate"):
             ws_bytes = lib.kda_forward_workspace_bytes(B, T, H, dk, dv)
             ws = workspace
             if ws is None or ws.numel() * ws.element_size() < ws_bytes:
                 ws = torch.empty(max(ws_bytes, 16), device=device, dtype=torch.uint8)
-            code = lib.kda_forward(*args, _ptr(ws), ws.numel() * ws.element_size(), stream)
+            code = getattr(lib, fn_name)(*args, _ptr(ws), ws.numel() * ws.element_size(), stream)
             if code == 0 and check_status:
                 code = lib.kda_workspace_status(_ptr(ws), stream)
         else:
@@ -201,6 +209,16 @@ def forward(q, k, v, alpha, beta, initial_state=None, scale=None, output_final_s
                     output_final_state, out_dtype, out, final_state, workspace, check_status)
 
 
+def forward_scalar_gate(q, k, v, alpha, beta, initial_state=None, scale=None, output_final_state=True,
+                        out_dtype=torch.float32, out=None, final_state=None, workspace=None,
+                        check_status=False):
+    """Gated DeltaNet prefill: one retention factor per (token, head), alpha [B,T,H]
+    (C entry point ``kda_forward_scalar_gate``); otherwise the contract of ``forward``."""
+    return _prefill("kda_forward_scalar_gate", q, k, v, alpha, beta, initial_state, scale,
+                    output_final_state, out_dtype, out, final_state, workspace, check_status,
+                    gate_per_head=True)
+
+
 def forward_sequential(q, k, v, alpha, beta, initial_state=None, scale=None,
                        output_final_state=True, out_dtype=torch.float32, out=None,
                        final_state=None):
@@ -209,7 +227,8 @@ def forward_sequential(q, k, v, alpha, beta, initial_state=None, scale=None,
                     output_final_state, out_dtype, out, final_state)
 
 
-def decode_step(q, k, v, alpha, beta, state, scale=None, out_dtype=torch.float32, out=None):
+def decode_step(q, k, v, alpha, beta, state, scale=None, out_dtype=torch.float32, out=None,
+                _gate_per_head=False):
     """One token per sequence; ``state`` [N,H,dk,dv] float32 is updated in place.
 
     q, k, alpha: [N,H,dk]; v: [N,H,dv]; beta: [N,H].  Returns o [N,H,dv].
@@ -223,10 +242,12 @@ def decode_step(q, k, v, alpha, beta, state, scale=None, out_dtype=torch.float32
         _check(name, t, device)
     if state.dtype != torch.float32:
         raise TypeError("state must be float32")
+    a_shape = (N, H) if _gate_per_head else (N, H, dk)
     if tuple(q.shape) != (N, H, dk) or tuple(k.shape) != (N, H, dk) or \
-            tuple(alpha.shape) != (N, H, dk) or tuple(v.shape) != (N, H, dv) or \
+            tuple(alpha.shape) != a_shape or tuple(v.shape) != (N, H, dv) or \
             tuple(beta.shape) != (N, H):
-        raise ValueError("shapes: q,k,alpha [N,H,dk], v [N,H,dv], beta [N,H], state [N,H,dk,dv]")
+        raise ValueError("shapes: q,k [N,H,dk], alpha " + ("[N,H]" if _gate_per_head else "[N,H,dk]")
+                         + ", v [N,H,dv], beta [N,H], state [N,H,dk,dv]")
     if k.dtype != q.dtype or v.dtype != q.dtype or alpha.dtype != beta.dtype:
         raise TypeError("q/k/v and alpha/beta must each share a dtype")
     if scale is None:
@@ -235,13 +256,20 @@ def decode_step(q, k, v, alpha, beta, state, scale=None, out_dtype=torch.float32
         out = torch.empty((N, H, dv), device=device, dtype=out_dtype)
     _check("out", out, device)
     with torch.cuda.device(device):
-        code = library().kda_decode_step(
+        fn = "kda_decode_step_scalar_gate" if _gate_per_head else "kda_decode_step"
+        code = getattr(library(), fn)(
             _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state), _ptr(out),
             N, H, dk, dv, float(scale), _DT[q.dtype], _dt(alpha, "alpha"), _dt(out, "out"),
             _vp(_stream_handle(device)))
     if code != 0:
-        raise KDAError("kda_decode_step", code)
+        raise KDAError(fn, code)
     return out
+
+
+def decode_step_scalar_gate(q, k, v, alpha, beta, state, scale=None, out_dtype=torch.float32, out=None):
+    """Gated DeltaNet decode step: alpha [N,H], one retention factor per (sequence, head)
+    (C entry point ``kda_decode_step_scalar_gate``); otherwise the contract of ``decode_step``."""
+    return decode_step(q, k, v, alpha, beta, state, scale, out_dtype, out, _gate_per_head=True)
 
 
 def forward_varlen(q, k, v, alpha, beta, cu_seqlens, initial_state=None, scale=None,

@@ -166,6 +166,26 @@ kda_status kda_forward_varlen(const void *q, const void *k, const void *v,
                               size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * kda_forward_scalar_gate -- kda_forward with one retention factor per (token,
+ * head): Gated DeltaNet, S~_t = alpha_t S_{t-1} with a scalar alpha_t, which is
+ * KDA with alpha_t broadcast over the key channels ("From Fast Weight
+ * Programmers to KDA", jonahsamost.bearblog.dev, section "Gated Delta
+ * Networks"; "Notes on Linear Attention: From Linear Attention to KDA",
+ * zhilingong.com, section 6 "Why add a gate?").  Arguments as
+ * kda_forward except alpha, which is [B, T, H] (gate_dtype, element-aligned
+ * like beta).  The per-channel decay work becomes per-token, and alpha's bytes
+ * shrink by d_k.
+ */
+kda_status kda_forward_scalar_gate(const void *q, const void *k, const void *v,
+                                   const void *alpha, const void *beta,
+                                   const float *initial_state, void *o,
+                                   float *final_state, int B, int T, int H,
+                                   int d_k, int d_v, float scale,
+                                   kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                                   kda_dtype out_dtype, void *workspace,
+                                   size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * kda_forward_sequential -- the same operation and arguments as kda_forward
  * (no workspace), computed with the token-by-token schedule ("fused
  * recurrent" in "Two schedules for the same recurrence", brain.bigb.es): one
@@ -197,6 +217,20 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v,
                            void *o, int N, int H, int d_k, int d_v, float scale,
                            kda_dtype qkv_dtype, kda_dtype gate_dtype,
                            kda_dtype out_dtype, cudaStream_t stream);
+
+/*
+ * kda_decode_step_scalar_gate -- kda_decode_step with one retention factor per
+ * (sequence, head): alpha is [N, H] (gate_dtype, element-aligned), broadcast
+ * over the key channels (Gated DeltaNet; see kda_forward_scalar_gate).
+ */
+kda_status kda_decode_step_scalar_gate(const void *q, const void *k,
+                                       const void *v, const void *alpha,
+                                       const void *beta, float *state, void *o,
+                                       int N, int H, int d_k, int d_v,
+                                       float scale, kda_dtype qkv_dtype,
+                                       kda_dtype gate_dtype,
+                                       kda_dtype out_dtype,
+                                       cudaStream_t stream);
 
 /* Static, NUL-terminated description of a status code. */
 const char *kda_status_string(kda_status status);
