@@ -8,6 +8,8 @@ and the two share no code.
 ``forward`` runs the sequential five-step update of "Module 03 -- KDA I: The
 Delta-Rule Recurrence", section 2, in C (``kda_oracle.c``), in fp64, over all
 (sequence, head) pairs.  ``decode_step`` is the same loop for one token.
+``forward_gdn2`` is the same loop with the decoupled erase and write gates of
+"From Fast Weight Programmers to KDA", section "Gated DeltaNet-2".
 ``chunked.forward_chunked`` (numpy, fp64) is the second schedule of "Kimi Delta
 Attention (KDA)", "Two schedules for the same recurrence"; the tests pin it to
 the sequential loop.
@@ -60,6 +62,8 @@ def _load():
                                             ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                             ctypes.c_int, ctypes.c_int]
             lib.kda_ref_forward.restype = ctypes.c_int
+            lib.kda_ref_forward_gdn2.argtypes = [dp] * 9 + [ctypes.c_int] * 5 + [ctypes.c_double, ctypes.c_int]
+            lib.kda_ref_forward_gdn2.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -109,6 +113,30 @@ def forward(q, k, v, alpha, beta, s0=None, scale=None, mode="exact", n_threads=0
                                  float(scale), MODES[mode], int(n_threads))
     if rc != 0:
         raise RuntimeError(f"kda_ref_forward failed with code {rc}")
+    return o, s_final
+
+
+def forward_gdn2(q, k, v, alpha, erase, write, s0=None, scale=None, n_threads=0):
+    """Sequential fp64 GDN-2: per-key-channel erase gate [B,T,H,dk] and per-value-channel
+    write gate [B,T,H,dv] in place of beta; otherwise as ``forward``."""
+    q, k, v, alpha, erase, write = (_f64(x) for x in (q, k, v, alpha, erase, write))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    assert k.shape == q.shape and alpha.shape == q.shape and erase.shape == q.shape, "dk shapes"
+    assert v.shape == (B, T, H, dv) and write.shape == v.shape, "dv shapes"
+    s0a = None
+    if s0 is not None:
+        s0a = _f64(s0)
+        assert s0a.shape == (B, H, dk, dv), "s0 shape"
+    if scale is None:
+        scale = dk ** -0.5
+    o = np.zeros((B, T, H, dv), dtype=np.float64)
+    s_final = np.zeros((B, H, dk, dv), dtype=np.float64)
+    rc = _load().kda_ref_forward_gdn2(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(erase), _ptr(write),
+                                      _ptr(s0a), _ptr(o), _ptr(s_final), B, T, H, dk, dv,
+                                      float(scale), int(n_threads))
+    if rc != 0:
+        raise RuntimeError(f"kda_ref_forward_gdn2 failed with code {rc}")
     return o, s_final
 
 

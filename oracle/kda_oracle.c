@@ -35,6 +35,21 @@
  *                            "Gated DeltaNet: sometimes everything should
  *                            fade", brain.bigb.es).
  *
+ * Decoupled erase and write gates (kda_ref_forward_gdn2): "From Fast Weight
+ * Programmers to KDA" (jonahsamost.bearblog.dev), section "Gated DeltaNet-2",
+ * replaces beta_t by a per-key-channel erase gate b_t and a per-value-channel
+ * write gate w_t.  That page writes the state as d_v x d_k; in the d_k x d_v
+ * layout used here its update reads
+ *
+ *   (1) forget   S~  = Diag(alpha_t) S_{t-1}
+ *   (2) predict  vh  = S~^T (b_t * k_t)          retrieval through the gated key
+ *   (3) correct  e   = w_t * v_t - vh            the residual of the gated value
+ *   (4) write    S_t = S~ + k_t e^T              stored at the original key
+ *   (5) read     o_t = S_t^T (scale q_t)
+ *
+ * (* is the elementwise product).  b_t = beta_t 1, w_t = beta_t 1 gives the
+ * KDA update above.
+ *
  * Layouts (row-major, contiguous):
  *   q, k, alpha : [B, T, H, d_k]      v, o : [B, T, H, d_v]
  *   beta        : [B, T, H]           s0, s_final : [B, H, d_k, d_v]
@@ -55,6 +70,7 @@
 
 typedef struct {
     const double *q, *k, *v, *alpha, *beta, *s0;
+    const double *erase, *wgate;   /* GDN-2 gates [B,T,H,d_k], [B,T,H,d_v], or NULL */
     double *o, *s_final;
     int B, T, H, dk, dv, mode;
     double scale;
@@ -85,8 +101,32 @@ static int run_head(ref_job *J, int b, int h)
         const double *kt = J->k + row * dk;
         const double *at = J->alpha + row * dk;
         const double *vt = J->v + row * dv;
-        const double bt = J->beta[row];
+        const double bt = J->beta ? J->beta[row] : 0.0;
         double *ot = J->o + row * dv;
+
+        if (J->erase) {
+            /* GDN-2: (1) forget, (2) predict through b * k, (3) correct, (4) write */
+            const double *bk = J->erase + row * dk;
+            const double *wv = J->wgate + row * dv;
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j)
+                    S[(size_t)i * dv + j] *= at[i];
+            for (int j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (int i = 0; i < dk; ++i) acc += S[(size_t)i * dv + j] * (bk[i] * kt[i]);
+                vh[j] = acc;
+            }
+            for (int j = 0; j < dv; ++j) e[j] = wv[j] * vt[j] - vh[j];
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j)
+                    S[(size_t)i * dv + j] += kt[i] * e[j];
+            for (int j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (int i = 0; i < dk; ++i) acc += S[(size_t)i * dv + j] * (J->scale * qt[i]);
+                ot[j] = acc;
+            }
+            continue;
+        }
 
         if (J->mode == KDA_REF_SWAP_ORDER) {
             /* (I - beta k k^T) applied to the undecayed state ... */
@@ -162,6 +202,8 @@ static void *worker(void *arg)
     return NULL;
 }
 
+static int run_job(ref_job *Jp, int n_threads);
+
 int kda_ref_forward(const double *q, const double *k, const double *v,
                     const double *alpha, const double *beta, const double *s0,
                     double *o, double *s_final, int B, int T, int H, int dk,
@@ -172,10 +214,36 @@ int kda_ref_forward(const double *q, const double *k, const double *v,
     if (mode < KDA_REF_EXACT || mode > KDA_REF_PREDICT_FIRST) return -1;
     ref_job J;
     J.q = q; J.k = k; J.v = v; J.alpha = alpha; J.beta = beta; J.s0 = s0;
+    J.erase = NULL; J.wgate = NULL;
     J.o = o; J.s_final = s_final;
     J.B = B; J.T = T; J.H = H; J.dk = dk; J.dv = dv; J.mode = mode;
-    J.scale = scale; J.next_item = 0; J.failed = 0;
+    J.scale = scale;
+    return run_job(&J, n_threads);
+}
+
+/* GDN-2: erase [B,T,H,d_k] and write [B,T,H,d_v] gates instead of beta. */
+int kda_ref_forward_gdn2(const double *q, const double *k, const double *v,
+                         const double *alpha, const double *erase, const double *wgate,
+                         const double *s0, double *o, double *s_final, int B, int T,
+                         int H, int dk, int dv, double scale, int n_threads)
+{
+    if (!q || !k || !v || !alpha || !erase || !wgate || !o) return -1;
+    if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
+    ref_job J;
+    J.q = q; J.k = k; J.v = v; J.alpha = alpha; J.beta = NULL; J.s0 = s0;
+    J.erase = erase; J.wgate = wgate;
+    J.o = o; J.s_final = s_final;
+    J.B = B; J.T = T; J.H = H; J.dk = dk; J.dv = dv; J.mode = KDA_REF_EXACT;
+    J.scale = scale;
+    return run_job(&J, n_threads);
+}
+
+static int run_job(ref_job *Jp, int n_threads)
+{
+    ref_job J = *Jp;
+    J.next_item = 0; J.failed = 0;
     pthread_mutex_init(&J.lock, NULL);
+    const int B = J.B, H = J.H;
 
     const int n_items = B * H;
     if (n_threads <= 0) n_threads = (int)sysconf(_SC_NPROCESSORS_ONLN);
