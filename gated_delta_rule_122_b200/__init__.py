@@ -2,17 +2,23 @@
 
 Entry points (see include/kda.h): ``forward`` (chunkwise prefill),
 ``forward_varlen`` (prefill over packed sequences of different lengths),
-``forward_scalar_gate`` / ``decode_step_scalar_gate`` (one retention factor per head:
-Gated DeltaNet),
-``forward_sequential`` (token-by-token schedule), ``decode_step`` (one token per
-sequence, state updated in place).  ``inputs`` draws the seeded synthetic
-workloads.  All arithmetic runs in ``libkda_b200.so``; build it with
-``python -m gated_delta_rule_122_b200.build``.
+``forward_scalar_gate`` / ``decode_step_scalar_gate`` (one retention factor per
+head: Gated DeltaNet), ``forward_gdn2`` / ``decode_step_gdn2`` (decoupled erase
+and write gates: GDN-2), ``forward_raw`` / ``decode_step_raw`` (input
+preprocessing fused into the kernels: raw q and k, gate and beta logits),
+``decode_tokens`` / ``state_copy`` (serving: several tokens per sequence over a
+pool of state slots with per-token states for rollback; whole-state copies for
+fork and rollback), ``forward_sequential`` (token-by-token schedule),
+``decode_step`` (one token per sequence, state updated in place).  ``inputs``
+draws the seeded synthetic workloads.  All arithmetic runs in
+``libkda_b200.so``; build it with ``python -m gated_delta_rule_122_b200.build``.
 """
-from .kda import (EXPORTED_SYMBOLS, KDAError, decode_step, decode_step_scalar_gate, forward,
+from .kda import (EXPORTED_SYMBOLS, KDAError, decode_step, decode_step_gdn2, decode_step_raw,
+                  decode_step_scalar_gate, decode_tokens, forward, forward_gdn2, forward_raw,
                   forward_scalar_gate, forward_sequential, forward_varlen, library, library_path,
-                  status_string, version)
+                  state_copy, status_string, version)
 
-__all__ = ["forward", "forward_varlen", "forward_scalar_gate", "forward_sequential", "decode_step",
-           "decode_step_scalar_gate", "KDAError", "library", "library_path", "status_string",
-           "version", "EXPORTED_SYMBOLS"]
+__all__ = ["forward", "forward_varlen", "forward_scalar_gate", "forward_gdn2", "forward_raw",
+           "forward_sequential", "decode_step", "decode_step_scalar_gate", "decode_step_gdn2",
+           "decode_step_raw", "decode_tokens", "state_copy", "KDAError", "library", "library_path",
+           "status_string", "version", "EXPORTED_SYMBOLS"]

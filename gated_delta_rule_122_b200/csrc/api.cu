@@ -205,6 +205,91 @@ kda_status kda_forward_scalar_gate(const void *q, const void *k, const void *v, 
     return err == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
 }
 
+kda_status kda_forward_raw(const void *q, const void *k, const void *v, const void *gate_logit,
+                           const void *beta_logit, const float *initial_state, void *o, float *final_state,
+                           int B, int T, int H, int d_k, int d_v, float scale, kda_dtype qkv_dtype,
+                           kda_dtype gate_dtype, kda_dtype out_dtype, void *workspace,
+                           size_t workspace_bytes, cudaStream_t stream)
+{
+    kda_status st = check_forward(q, k, v, gate_logit, beta_logit, initial_state, o, final_state, B, T, H,
+                                  d_k, d_v, qkv_dtype, gate_dtype, out_dtype);
+    if (st != KDA_OK) return st;
+    if (B * (long long)H == 0) return KDA_OK;
+    const size_t need = kda_forward_workspace_bytes(B, T, H, d_k, d_v);
+    if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return KDA_ERR_ALIGN;
+    if (cudaMemsetAsync(workspace, 0, need, stream) != cudaSuccess) return KDA_ERR_LAUNCH;
+    if (T == 0) return empty_sequence(initial_state, final_state, B, H, d_k, d_v, stream);
+    kda::ChunkArgs a{q, k, v, gate_logit, beta_logit, initial_state, final_state, o, B, T, H, scale,
+                     qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16,
+                     static_cast<unsigned int *>(workspace)};
+    a.raw_inputs = 1;
+    cudaError_t err;
+    if (kda::chunk_tc_supported(d_k, d_v, qkv_dtype, gate_dtype))
+        err = kda::launch_chunk_tc(a, d_k, d_v, stream);
+    else
+        err = kda::launch_chunk_simt(a, d_k, d_v, stream);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+}
+
+kda_status kda_decode_step_raw(const void *q, const void *k, const void *v, const void *gate_logit,
+                               const void *beta_logit, float *state, void *o, int N, int H, int d_k,
+                               int d_v, float scale, kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                               kda_dtype out_dtype, cudaStream_t stream)
+{
+    if (N * (long long)H > 0 && !state) return KDA_ERR_NULL;
+    kda_status st = check_forward(q, k, v, gate_logit, beta_logit, state, o, nullptr, N, 1, H, d_k, d_v,
+                                  qkv_dtype, gate_dtype, out_dtype);
+    if (st != KDA_OK) return st;
+    if (N * (long long)H == 0) return KDA_OK;
+    kda::RecurrentArgs a{q, k, v, gate_logit, beta_logit, state, state, o, N, 1, H, scale,
+                         qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16, nullptr};
+    a.raw_inputs = 1;
+    return kda::launch_recurrent(a, d_k, d_v, stream) == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+}
+
+// GDN-2 entry points: the erase and write gates take the place of beta.
+static kda_status check_gdn2(const void *q, const void *k, const void *v, const void *alpha,
+                             const void *erase, const void *wgate, const float *s_in, const void *o,
+                             const float *s_out, int B, int T, int H, int dk, int dv, kda_dtype qkv,
+                             kda_dtype gate, kda_dtype out)
+{
+    // erase stands in for beta in the common checks (presence, alignment, aliasing of o)
+    kda_status st = check_forward(q, k, v, alpha, erase, s_in, o, s_out, B, T, H, dk, dv, qkv, gate, out);
+    if (st != KDA_OK) return st;
+    if (B * (long long)H == 0 || T == 0) return KDA_OK;
+    if (!wgate) return KDA_ERR_NULL;
+    if (!aligned16(erase) || !aligned16(wgate)) return KDA_ERR_ALIGN;
+    const unsigned long long tokens = (unsigned long long)B * T * H;
+    const Range ro = range_of(o, tokens * dv * dsize(out));
+    if (overlap(ro, range_of(erase, tokens * dk * dsize(gate))) ||
+        overlap(ro, range_of(wgate, tokens * dv * dsize(gate))))
+        return KDA_ERR_ALIAS;
+    return KDA_OK;
+}
+
+kda_status kda_forward_gdn2(const void *q, const void *k, const void *v, const void *alpha,
+                            const void *erase, const void *wgate, const float *initial_state, void *o,
+                            float *final_state, int B, int T, int H, int d_k, int d_v, float scale,
+                            kda_dtype qkv_dtype, kda_dtype gate_dtype, kda_dtype out_dtype,
+                            void *workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    kda_status st = check_gdn2(q, k, v, alpha, erase, wgate, initial_state, o, final_state, B, T, H,
+                               d_k, d_v, qkv_dtype, gate_dtype, out_dtype);
+    if (st != KDA_OK) return st;
+    if (B * (long long)H == 0) return KDA_OK;
+    const size_t need = kda_forward_workspace_bytes(B, T, H, d_k, d_v);
+    if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return KDA_ERR_ALIGN;
+    if (cudaMemsetAsync(workspace, 0, need, stream) != cudaSuccess) return KDA_ERR_LAUNCH;
+    if (T == 0) return empty_sequence(initial_state, final_state, B, H, d_k, d_v, stream);
+    kda::ChunkArgs a{q, k, v, alpha, nullptr, initial_state, final_state, o, B, T, H, scale,
+                     qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16,
+                     static_cast<unsigned int *>(workspace), nullptr, 0, erase, wgate};
+    // the CUDA-core chunk kernel serves every shape and dtype of GDN-2
+    return kda::launch_chunk_simt(a, d_k, d_v, stream) == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+}
+
 kda_status kda_forward_sequential(const void *q, const void *k, const void *v, const void *alpha,
                                   const void *beta, const float *initial_state, void *o,
                                   float *final_state, int B, int T, int H, int d_k, int d_v,
@@ -254,6 +339,72 @@ kda_status kda_decode_step_scalar_gate(const void *q, const void *k, const void 
                          qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16,
                          nullptr, nullptr, 1};
     return kda::launch_recurrent(a, d_k, d_v, stream) == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+}
+
+kda_status kda_decode_step_gdn2(const void *q, const void *k, const void *v, const void *alpha,
+                                const void *erase, const void *wgate, float *state, void *o, int N,
+                                int H, int d_k, int d_v, float scale, kda_dtype qkv_dtype,
+                                kda_dtype gate_dtype, kda_dtype out_dtype, cudaStream_t stream)
+{
+    if (N * (long long)H > 0 && !state) return KDA_ERR_NULL;
+    kda_status st = check_gdn2(q, k, v, alpha, erase, wgate, state, o, nullptr, N, 1, H, d_k, d_v,
+                               qkv_dtype, gate_dtype, out_dtype);
+    if (st != KDA_OK) return st;
+    if (N * (long long)H == 0) return KDA_OK;
+    kda::RecurrentArgs a{q, k, v, alpha, nullptr, state, state, o, N, 1, H, scale,
+                         qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16,
+                         nullptr, nullptr, 0, erase, wgate};
+    return kda::launch_recurrent(a, d_k, d_v, stream) == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+}
+
+kda_status kda_decode_tokens(const void *q, const void *k, const void *v, const void *alpha,
+                             const void *beta, float *state, const int *state_slots, int num_slots,
+                             int commit, float *token_states, void *o, int N, int T, int H, int d_k,
+                             int d_v, float scale, kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                             kda_dtype out_dtype, void *status, cudaStream_t stream)
+{
+    kda_status st = check_forward(q, k, v, alpha, beta, nullptr, o, nullptr, N, T, H, d_k, d_v,
+                                  qkv_dtype, gate_dtype, out_dtype);
+    if (st != KDA_OK) return st;
+    if (num_slots < 0 || (!state_slots && num_slots < N)) return KDA_ERR_SHAPE;
+    if (!aligned16(state) || !aligned16(token_states) || !aligned16(status) ||
+        !aligned_to(state_slots, sizeof(int)))
+        return KDA_ERR_ALIGN;
+    if (status && cudaMemsetAsync(status, 0, sizeof(unsigned int), stream) != cudaSuccess)
+        return KDA_ERR_LAUNCH;
+    if (N * (long long)H == 0 || T == 0) return KDA_OK;
+    if (!state) return KDA_ERR_NULL;
+    const size_t per_state = (size_t)H * d_k * d_v * sizeof(float);
+    const Range ro = range_of(o, (size_t)N * T * H * d_v * dsize(out_dtype));
+    const Range rp = range_of(state, (size_t)num_slots * per_state);
+    const Range rt = range_of(token_states, token_states ? (size_t)N * T * per_state : 0);
+    if (overlap(ro, rp) || overlap(ro, rt) || overlap(rp, rt)) return KDA_ERR_ALIAS;
+    kda::RecurrentArgs a{q, k, v, alpha, beta, state, commit ? state : nullptr, o, N, T, H, scale,
+                         qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16,
+                         static_cast<unsigned int *>(status)};
+    a.state_slots = state_slots;
+    a.num_slots = num_slots;
+    a.token_states = token_states;
+    return kda::launch_recurrent(a, d_k, d_v, stream) == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+}
+
+kda_status kda_state_copy(const float *src, const int *src_index, int src_slots, float *dst,
+                          const int *dst_index, int dst_slots, int count, int H, int d_k, int d_v,
+                          void *status, cudaStream_t stream)
+{
+    if (count < 0 || src_slots < 0 || dst_slots < 0 || H < 0) return KDA_ERR_SHAPE;
+    if (!head_size_ok(d_k) || !head_size_ok(d_v)) return KDA_ERR_UNSUPPORTED;
+    if ((!src_index && count > src_slots) || (!dst_index && count > dst_slots)) return KDA_ERR_SHAPE;
+    if (!aligned16(src) || !aligned16(dst) || !aligned16(status) || !aligned_to(src_index, sizeof(int)) ||
+        !aligned_to(dst_index, sizeof(int)))
+        return KDA_ERR_ALIGN;
+    if (status && cudaMemsetAsync(status, 0, sizeof(unsigned int), stream) != cudaSuccess)
+        return KDA_ERR_LAUNCH;
+    if (count == 0 || H == 0) return KDA_OK;
+    if (!src || !dst) return KDA_ERR_NULL;
+    kda::StateCopyArgs a{src, src_index, src_slots, dst, dst_index, dst_slots, count,
+                         (size_t)H * d_k * d_v / 4, static_cast<unsigned int *>(status)};
+    return kda::launch_state_copy(a, stream) == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
 }
 
 }  // extern "C"

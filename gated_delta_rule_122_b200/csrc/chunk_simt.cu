@@ -13,6 +13,13 @@
 //   S <- Diag(exp(G_end)) S + (K * exp(G_end - G))^T E
 // Every pairwise decay exp(G_r - G_s), s <= r, is formed directly, so no
 // factor ever exceeds 1 and no anchoring is needed on this path.
+// GDN-2 ("From Fast Weight Programmers to KDA", section "Gated DeltaNet-2"):
+// with an erase gate b_r (per key channel) and a write gate w_r (per value
+// channel) instead of beta_r, the same steps run with
+//   Akk[r][s] = sum_d b_rd k_rd k_sd exp(G_rd - G_sd),
+//   (I + Akk) W = (b * K) * exp(G),   (I + Akk) U = w * V.
+// With raw inputs the staging applies the preprocessing first: q_r and k_r divided
+// by their L2 norms, G from log alpha = -softplus(gate logit), beta = sigmoid(logit).
 // Algorithm: "Kimi Delta Attention (KDA)" (brain.bigb.es), "Two schedules for
 // the same recurrence"; "From Fast Weight Programmers to KDA"
 // (jonahsamost.bearblog.dev), section "Kimi Delta Attention".
@@ -39,13 +46,14 @@ struct SimtLayout {
     static constexpr int oAkk = oS + DK * DV;
     static constexpr int oAqk = oAkk + C * PC;
     static constexpr int oBeta = oAqk + C * PC;
-    static constexpr int floats = oBeta + C;
+    static constexpr int oNrm = oBeta + C;      // 1/||q_r||, 1/||k_r|| (raw inputs)
+    static constexpr int floats = oNrm + 2 * C;
     static constexpr size_t bytes = sizeof(float) * (size_t)floats;
 };
 
-template <int DK, int DV>
+template <int DK, int DV, bool kGdn2>
 __global__ void __launch_bounds__(kSimtThreads)
-kda_chunk_simt_kernel(ChunkArgs ain)
+kda_chunk_simt_kernel(ChunkArgs a)
 {
     using Ly = SimtLayout<DK, DV>;
     constexpr int C = Ly::C, PK = Ly::PK, PV = Ly::PV, PC = Ly::PC, NT = kSimtThreads;
@@ -57,17 +65,15 @@ kda_chunk_simt_kernel(ChunkArgs ain)
     extern __shared__ float sm[];
     float *Q = sm + Ly::oQ, *K = sm + Ly::oK, *G = sm + Ly::oG, *W = sm + Ly::oW;
     float *V = sm + Ly::oV, *E = sm + Ly::oE, *S = sm + Ly::oS;
-    float *Akk = sm + Ly::oAkk, *Aqk = sm + Ly::oAqk, *Bt = sm + Ly::oBeta;
+    float *Akk = sm + Ly::oAkk, *Aqk = sm + Ly::oAqk, *Bt = sm + Ly::oBeta, *Nrm = sm + Ly::oNrm;
 
     const int bh = blockIdx.x;                 // sequence * H + head (state tile)
-    const int h = bh % ain.H;
+    const int h = bh % a.H;
     const int tid = threadIdx.x;
     const size_t tile = (size_t)bh * DK * DV;
-    // the sequence's own rows (packed layout) as a batch of one
-    ChunkArgs a;
-    int b, row0;
-    if (!sequence_view(ain, bh / ain.H, DK, DV, a, b, row0)) {
-        if (tid == 0 && ain.status) atomicOr(ain.status, 2u);
+    SeqSpan sp;                                // the sequence's token rows
+    if (!sequence_span(a, bh / a.H, sp)) {
+        if (tid == 0 && a.status) atomicOr(a.status, 2u);
         return;
     }
 
@@ -76,33 +82,56 @@ kda_chunk_simt_kernel(ChunkArgs ain)
 
     const int jcol = tid % DV, rgrp = tid / DV;
 
-    for (int t0 = 0; t0 < a.T; t0 += C) {
-        const int L = min(C, a.T - t0);
+    for (int t0 = 0; t0 < sp.len; t0 += C) {
+        const int L = min(C, sp.len - t0);
         // 1. stage the chunk; rows >= L are identity steps (k = q = v = 0, alpha = 1, beta = 0)
         for (int idx = tid; idx < C * DK; idx += NT) {
             const int r = idx / DK, d = idx % DK;
             float qv = 0.f, kv = 0.f, gv = 0.f;
             if (r < L) {
-                const size_t row = ((size_t)b * a.T + t0 + r) * a.H + h;
+                const size_t row = (sp.tok0 + t0 + r) * a.H + h;
                 qv = ld_elem(a.q, row * DK + d, a.qkv_bf16);
                 kv = ld_elem(a.k, row * DK + d, a.qkv_bf16);
-                gv = log_alpha(ld_elem(a.alpha, a.gate_per_head ? row : row * DK + d, a.gate_bf16));
+                const float x = ld_elem(a.alpha, a.gate_per_head ? row : row * DK + d, a.gate_bf16);
+                gv = a.raw_inputs ? log_alpha_from_logit(x) : log_alpha(x);
             }
             Q[r * PK + d] = qv; K[r * PK + d] = kv; G[r * PK + d] = gv;
+            if constexpr (kGdn2) {   // the erase-gated key b * k, the left factor of Akk
+                const size_t row = (sp.tok0 + t0 + r) * a.H + h;
+                W[r * PK + d] = (r < L) ? ld_elem(a.erase, row * DK + d, a.gate_bf16) * kv : 0.f;
+            }
         }
         for (int idx = tid; idx < C * DV; idx += NT) {
             const int r = idx / DV, j = idx % DV;
             float vv = 0.f;
             if (r < L) {
-                const size_t row = ((size_t)b * a.T + t0 + r) * a.H + h;
+                const size_t row = (sp.tok0 + t0 + r) * a.H + h;
                 vv = ld_elem(a.v, row * DV + j, a.qkv_bf16);
             }
             V[r * PV + j] = vv;
         }
-        for (int r = tid; r < C; r += NT) {
-            Bt[r] = (r < L) ? ld_elem(a.beta, ((size_t)b * a.T + t0 + r) * a.H + h, a.gate_bf16) : 0.f;
+        if constexpr (!kGdn2) {   // GDN-2 has no beta tensor
+            for (int r = tid; r < C; r += NT) {
+                const float y = (r < L) ? ld_elem(a.beta, (sp.tok0 + t0 + r) * a.H + h, a.gate_bf16) : 0.f;
+                Bt[r] = (r < L) ? (a.raw_inputs ? sigmoid_of(y) : y) : 0.f;
+            }
         }
         __syncthreads();
+        if (a.raw_inputs) {   // q_r / ||q_r||, k_r / ||k_r||
+            for (int r = tid; r < 2 * C; r += NT) {
+                const float *x = (r < C) ? Q + r * PK : K + (r - C) * PK;
+                float ss = 0.f;
+                for (int d = 0; d < DK; ++d) ss = fmaf(x[d], x[d], ss);
+                Nrm[r] = inv_norm(ss);
+            }
+            __syncthreads();
+            for (int idx = tid; idx < C * DK; idx += NT) {
+                const int r = idx / DK, d = idx % DK;
+                Q[r * PK + d] *= Nrm[r];
+                K[r * PK + d] *= Nrm[C + r];
+            }
+            __syncthreads();
+        }
 
         // 2. inclusive cumulative log-decay per key channel
         for (int d = tid; d < DK; d += NT) {
@@ -118,20 +147,27 @@ kda_chunk_simt_kernel(ChunkArgs ain)
             if (s <= r) {
                 for (int d = 0; d < DK; ++d) {
                     const float ks = K[s * PK + d] * expf(G[r * PK + d] - G[s * PK + d]);
-                    akk = fmaf(K[r * PK + d], ks, akk);
+                    akk = fmaf(kGdn2 ? W[r * PK + d] : K[r * PK + d], ks, akk);
                     aqk = fmaf(Q[r * PK + d], ks, aqk);
                 }
             }
-            Akk[r * PC + s] = (s < r) ? Bt[r] * akk : 0.f;
+            Akk[r * PC + s] = (s < r) ? (kGdn2 ? akk : Bt[r] * akk) : 0.f;
             Aqk[r * PC + s] = aqk;
         }
+        if constexpr (kGdn2) __syncthreads();   // the Akk loop above read W
         for (int idx = tid; idx < C * DK; idx += NT) {
             const int r = idx / DK, d = idx % DK;
-            W[r * PK + d] = Bt[r] * K[r * PK + d] * expf(G[r * PK + d]);
+            if constexpr (kGdn2) W[r * PK + d] *= expf(G[r * PK + d]);
+            else W[r * PK + d] = Bt[r] * K[r * PK + d] * expf(G[r * PK + d]);
         }
         for (int idx = tid; idx < C * DV; idx += NT) {
             const int r = idx / DV, j = idx % DV;
-            V[r * PV + j] *= Bt[r];
+            if constexpr (kGdn2) {
+                const size_t row = (sp.tok0 + t0 + r) * a.H + h;
+                V[r * PV + j] *= (r < L) ? ld_elem(a.wgate, row * DV + j, a.gate_bf16) : 0.f;
+            } else {
+                V[r * PV + j] *= Bt[r];
+            }
         }
         __syncthreads();
 
@@ -185,7 +221,7 @@ kda_chunk_simt_kernel(ChunkArgs ain)
             float o = oacc[m];
             for (int s = 0; s <= r; ++s) o = fmaf(Aqk[r * PC + s], E[s * PV + jcol], o);
             if (r < L) {
-                const size_t row = ((size_t)b * a.T + t0 + r) * a.H + h;
+                const size_t row = (sp.tok0 + t0 + r) * a.H + h;
                 st_elem(a.o, row * DV + jcol, a.scale * o, a.out_bf16);
             }
         }
@@ -210,11 +246,10 @@ static cudaError_t launch_chunk_simt_t(const ChunkArgs &a, cudaStream_t stream)
     using Ly = SimtLayout<DK, DV>;
     const long long blocks = (long long)a.B * a.H;
     if (blocks == 0) return cudaSuccess;
-    cudaError_t err = cudaFuncSetAttribute(kda_chunk_simt_kernel<DK, DV>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)Ly::bytes);
+    auto kernel = a.erase ? kda_chunk_simt_kernel<DK, DV, true> : kda_chunk_simt_kernel<DK, DV, false>;
+    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Ly::bytes);
     if (err != cudaSuccess) return err;
-    kda_chunk_simt_kernel<DK, DV><<<(unsigned)blocks, kSimtThreads, Ly::bytes, stream>>>(a);
+    kernel<<<(unsigned)blocks, kSimtThreads, Ly::bytes, stream>>>(a);
     return cudaGetLastError();
 }
 

@@ -119,8 +119,9 @@ constexpr int OFF_XS = OFF_AQ + 2 * AQ_BYTES;          // A10 T0 of the solve fp
 constexpr int OFF_AKK = OFF_XS + C * P * 4;            // A_kk^T fp32 [32][36]
 constexpr int OFF_TS = OFF_AKK + C * (C + 4) * 4;      // T fp32 [32][33]
 constexpr int OFF_BETA = OFF_TS + C * P * 4;           // beta of the chunk being solved
+constexpr int OFF_NRM = OFF_BETA + C * 4;             // 1/||q_r||, 1/||k_r|| (raw inputs)
 constexpr int NBARS = 7;
-constexpr int OFF_BAR = (OFF_BETA + C * 4 + 7) / 8 * 8;
+constexpr int OFF_BAR = (OFF_NRM + 2 * C * 4 + 7) / 8 * 8;
 constexpr int OFF_SIG = OFF_BAR + NBARS * 8;           // 6 readiness counters
 constexpr int OFF_MISC = OFF_SIG + 32;                 // tmem base, error flag
 constexpr int SMEM_BYTES = OFF_MISC + 16;
@@ -180,11 +181,12 @@ __device__ __forceinline__ bool prep_bar_err(volatile int *err_flag)
     return ptx::named_bar_sync_or(kPrepBar, NPT, *err_flag != 0);
 }
 
-__device__ __forceinline__ float load_beta(const ChunkArgs &p, int b, int h, int n, int r)
+__device__ __forceinline__ float load_beta(const ChunkArgs &p, const SeqSpan &sp, int h, int n, int r)
 {
     const int t = n * C + r;
-    if (t >= p.T) return 0.f;
-    return __bfloat162float(((const __nv_bfloat16 *)p.beta)[((size_t)b * p.T + t) * p.H + h]);
+    if (t >= sp.len) return 0.f;
+    const float y = __bfloat162float(((const __nv_bfloat16 *)p.beta)[(sp.tok0 + t) * p.H + h]);
+    return p.raw_inputs ? sigmoid_of(y) : y;   // raw inputs: beta logits
 }
 
 // TMA descriptors of one launch: q, k, alpha as [B][T][H][128] boxes of 32 token
@@ -371,22 +373,25 @@ __device__ __forceinline__ void solve_diag_blocks(const float *At, float *Tm, in
 // Part A only touches slabs the A product (M1), the W'/U product (M2) and the O/E
 // product (M3) of the chunk two back have finished with, so it can run while that
 // chunk's state update (M4) still reads R.
-template <bool kHeadGate>
-__device__ void stage_a(const ChunkArgs &p, uint8_t *sm, int b, int h, int n, int warp, int lane, uint32_t (&rw)[16])
+template <bool kHeadGate, bool kRaw>
+__device__ void stage_a(const ChunkArgs &p, uint8_t *sm, const SeqSpan &sp, int h, int n, int warp, int lane, uint32_t (&rw)[16])
 {
     const int hf = warp >> 2, d = 32 * (warp & 3) + lane;
-    const int Lc = min(C, p.T - n * C);
+    const int Lc = min(C, sp.len - n * C);
     uint8_t *lqr = sm + OFF_LQR + (n & 1) * LQR_BYTES;
     float *cst = reinterpret_cast<float *>(sm + OFF_CST + (n % kCstSlots) * CST_BYTES);
     const float *cst_prev = reinterpret_cast<const float *>(sm + OFF_CST + ((n + kCstSlots - 1) % kCstSlots) * CST_BYTES);
     const uint8_t *stg = sm + OFF_STG;
     // alpha of row r: the staged row's channel d, or with one gate per head, the token's
     // gate straight from global memory (the same 32 values for every thread)
-    const __nv_bfloat16 *ah = (const __nv_bfloat16 *)p.alpha + ((size_t)b * p.T + (size_t)n * C) * p.H + h;
+    const __nv_bfloat16 *ah = (const __nv_bfloat16 *)p.alpha + (sp.tok0 + (size_t)n * C) * p.H + h;
     auto alpha_at = [&](int r) {
         if constexpr (kHeadGate) return __bfloat162float(ah[(size_t)r * p.H]);
+        // a gate logit x: alpha = exp(-softplus(x)) = 1 / (1 + e^x)
+        else if constexpr (kRaw) return ptx::rcp(1.f + __expf(ld_bf16(stg + STG_A + stg_row(r) + 2 * d)));
         else return ld_bf16(stg + STG_A + stg_row(r) + 2 * d);
     };
+    const float *nrm = reinterpret_cast<const float *>(sm + OFF_NRM);
     float pr[16];
     float acc = 1.f;
     if (hf == 1) {
@@ -426,6 +431,10 @@ __device__ void stage_a(const ChunkArgs &p, uint8_t *sm, int b, int h, int n, in
                 // rows past the sequence's end: zero (the staging may hold another sequence's rows)
                 kv[t] = (r < Lc) ? ld_bf16(stg + STG_K + stg_row(r) + 2 * d) : 0.f;
                 qv[t] = (r < Lc) ? ld_bf16(stg + STG_Q + stg_row(r) + 2 * d) : 0.f;
+                if constexpr (kRaw) {   // unit rows
+                    kv[t] = (r < Lc) ? kv[t] * nrm[C + r] : 0.f;
+                    qv[t] = (r < Lc) ? qv[t] * nrm[r] : 0.f;
+                }
             }
             const uint64_t e2 = ptx::pk2(e[0], e[1]);
             ptx::upk2(ptx::mul2(ptx::pk2(kv[0], kv[1]), e2), lk[i], lk[i + 1]);
@@ -484,7 +493,7 @@ __device__ __forceinline__ void load_v(const TcMaps &maps, uint8_t *sm, const Ba
 // shared memory; warp 1 forms A_kk and solves its diagonal blocks, warp 3 writes
 // A_qk, and all four finish the off-diagonal block of T and write T'.
 __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, uint32_t tmem, const Bars &bars,
-                          const TmaPos &tp, int b, int h, int nchunks, volatile int *err_flag)
+                          const TmaPos &tp, const SeqSpan &sp, int h, int nchunks, volatile int *err_flag)
 {
     const int pt = threadIdx.x - NCT;          // 0..127
     const int pw = pt >> 5, lane = pt & 31;    // warp = TMEM lane quadrant
@@ -505,10 +514,10 @@ __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, u
         if (nchunks > 1) load_v(maps, sm, bars, tp, 1);
     }
     v_loaded = nchunks > 1 ? 2 : 1;
-    float beta = (pw < 2) ? load_beta(p, b, h, 0, r) : 0.f;   // beta of row r
+    float beta = (pw < 2) ? load_beta(p, sp, h, 0, r) : 0.f;   // beta of row r
 
     for (int cn = 0; cn < nchunks; ++cn) {
-        const float beta_next = (pw < 2 && cn + 1 < nchunks) ? load_beta(p, b, h, cn + 1, r) : 0.f;
+        const float beta_next = (pw < 2 && cn + 1 < nchunks) ? load_beta(p, sp, h, cn + 1, r) : 0.f;
 
         // ---- G(cn): A_kk / A_qk from TMEM; the solve; T'
         if (!ptx::mbar_wait(bars.a, (uint32_t)(cn & 1), kWaitLimitNs)) *err_flag = 1;
@@ -537,10 +546,10 @@ __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, u
         // V(cn) has landed (every warp observes it before it signals M2's readiness)
         if (!ptx::mbar_wait(bars.v + 8 * (cn & 1), (uint32_t)((cn >> 1) & 1), kWaitLimitNs)) *err_flag = 1;
         v_seen = cn + 1;
-        if (p.T - cn * C < C) {
+        if (sp.len - cn * C < C) {
             // rows past the sequence's end hold zeros (dense layout) or the next
             // sequence's tokens (packed): clear them, T' does not see them anyway
-            const int Lc = p.T - cn * C;
+            const int Lc = sp.len - cn * C;
             uint8_t *vb = sm + OFF_V + (cn & 1) * V_BYTES;
             for (int i = pt; i < (C - Lc) * (D / 8); i += NPT) {
                 const int r = Lc + i / (D / 8), jb = i % (D / 8);
@@ -669,12 +678,47 @@ __device__ __forceinline__ void write_state16(uint32_t tmem, uint32_t lane_base,
 
 // Chain warps, operands of chunk n (the staging rows must hold chunk n): part A,
 // then (later) part B, the signal to the issuer and the loads of chunk n+1.
-template <bool kHeadGate>
-__device__ __forceinline__ void chain_stage_a(const ChunkArgs &p, uint8_t *sm, const Bars &bars, int b, int h, int n, int warp,
+// Raw inputs: 1/||q_r|| and 1/||k_r|| of the staged rows, four rows per chain warp
+// (each lane sums the squares of four channels; a butterfly finishes the rows).
+__device__ __forceinline__ void row_norms(uint8_t *sm, int warp, int lane)
+{
+    const uint8_t *stg = sm + OFF_STG;
+    float ss[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = 4 * warp + i;
+        const uint2 qw = *reinterpret_cast<const uint2 *>(stg + STG_Q + stg_row(r) + 8 * lane);
+        const uint2 kw = *reinterpret_cast<const uint2 *>(stg + STG_K + stg_row(r) + 8 * lane);
+        float a0 = __uint_as_float(qw.x << 16), a1 = __uint_as_float(qw.x & 0xFFFF0000u);
+        float a2 = __uint_as_float(qw.y << 16), a3 = __uint_as_float(qw.y & 0xFFFF0000u);
+        ss[i] = fmaf(a0, a0, fmaf(a1, a1, fmaf(a2, a2, a3 * a3)));
+        a0 = __uint_as_float(kw.x << 16); a1 = __uint_as_float(kw.x & 0xFFFF0000u);
+        a2 = __uint_as_float(kw.y << 16); a3 = __uint_as_float(kw.y & 0xFFFF0000u);
+        ss[4 + i] = fmaf(a0, a0, fmaf(a1, a1, fmaf(a2, a2, a3 * a3)));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss[i] += __shfl_xor_sync(0xffffffffu, ss[i], off);
+    if (lane < 8) {
+        float x = ss[0];
+#pragma unroll
+        for (int i = 1; i < 8; ++i) x = (lane == i) ? ss[i] : x;
+        const int r = 4 * warp + (lane & 3);
+        reinterpret_cast<float *>(sm + OFF_NRM)[(lane < 4 ? 0 : C) + r] = inv_norm(x);
+    }
+}
+
+template <bool kHeadGate, bool kRaw>
+__device__ __forceinline__ void chain_stage_a(const ChunkArgs &p, uint8_t *sm, const Bars &bars, const SeqSpan &sp, int h, int n, int warp,
                                               int lane, uint32_t (&ie)[16], volatile int *err_flag)
 {
     if (!ptx::mbar_wait(bars.stg, (uint32_t)(n & 1), kWaitLimitNs)) *err_flag = 1;   // chunk n's rows
-    stage_a<kHeadGate>(p, sm, b, h, n, warp, lane, ie);
+    if constexpr (kRaw) {
+        row_norms(sm, warp, lane);
+        chain_bar();   // every row's norms are in place
+    }
+    stage_a<kHeadGate, kRaw>(p, sm, sp, h, n, warp, lane, ie);
 }
 
 __device__ __forceinline__ void chain_stage_b(const TcMaps &maps, uint8_t *sm, const Bars &bars, const TmaPos &tp,
@@ -695,9 +739,9 @@ __device__ __forceinline__ void warp_signal_after_stage(const Bars &bars, int la
 }
 
 // ---- the chain warps: the serial recurrence over chunks --------------------------------
-template <bool kHeadGate>
+template <bool kHeadGate, bool kRaw>
 __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, uint32_t tmem, const Bars &bars,
-                           const TmaPos &tp, int b, int h, int bh, int nchunks, volatile int *err_flag)
+                           const TmaPos &tp, const SeqSpan &sp, int h, int bh, int nchunks, volatile int *err_flag)
 {
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -709,7 +753,7 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
     uint32_t ie[16];   // R of the chunk being staged (split words), carried from part A to part B
     if (tid == 0) load_qka(maps, sm, bars, tp, 0);
     int staged = 0;   // chunks whose rows have been waited for
-    chain_stage_a<kHeadGate>(p, sm, bars, b, h, 0, warp, lane, ie, err_flag);
+    chain_stage_a<kHeadGate, kRaw>(p, sm, bars, sp, h, 0, warp, lane, ie, err_flag);
     staged = 1;
     chain_stage_b(maps, sm, bars, tp, 0, nchunks, tid, warp, lane, ie);
 
@@ -731,7 +775,7 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
     ptx::tc_fence_before();
     warp_signal(bars.rs, lane);
     if (nchunks > 1) {
-        chain_stage_a<kHeadGate>(p, sm, bars, b, h, 1, warp, lane, ie, err_flag);
+        chain_stage_a<kHeadGate, kRaw>(p, sm, bars, sp, h, 1, warp, lane, ie, err_flag);
         staged = 2;
         chain_stage_b(maps, sm, bars, tp, 1, nchunks, tid, warp, lane, ie);
     }
@@ -760,7 +804,7 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
         warp_signal(bars.re, lane);
         // Lk, Lq of chunk c+2 while the state update of chunk c runs
         if (c + 2 < nchunks) {
-            chain_stage_a<kHeadGate>(p, sm, bars, b, h, c + 2, warp, lane, ie, err_flag);
+            chain_stage_a<kHeadGate, kRaw>(p, sm, bars, sp, h, c + 2, warp, lane, ie, err_flag);
             staged = c + 3;
         }
 
@@ -835,7 +879,7 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
             if (tid == 0) ptx::bulk_wait_read();
             chain_bar();
         }
-        const bool full = (c + 1) * C <= p.T;
+        const bool full = (c + 1) * C <= sp.len;
         if (full) {
             const int esz = p.out_bf16 ? 2 : 4;
             uint8_t *tile = sm + OFF_STG + (half ? STG_A : STG_Q) + j * esz;
@@ -851,10 +895,10 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
             // the sequence's last, partial chunk: only its own rows, one element per row
             // (a TMA box would also cover rows that belong to the next sequence)
             const size_t step = (size_t)p.H * D;
-            size_t idx = (((size_t)b * p.T + c * C + 16 * half) * p.H + h) * D + j;
+            size_t idx = ((sp.tok0 + c * C + 16 * half) * p.H + h) * D + j;
 #pragma unroll
             for (int i = 0; i < 16; ++i, idx += step)
-                if (c * C + 16 * half + i < p.T) st_elem(p.o, idx, ov[i], p.out_bf16);
+                if (c * C + 16 * half + i < sp.len) st_elem(p.o, idx, ov[i], p.out_bf16);
         }
         ptx::fence_proxy_async_smem();
         const bool stop = chain_bar_err(err_flag);   // output tile written, staging rows consumed
@@ -878,7 +922,8 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
 }
 
 // kHeadGate: one retention factor per (token, head), alpha [B, T, H] (Gated DeltaNet).
-template <bool kHeadGate>
+// kRaw: the input preprocessing is fused into the staging (raw q, k and logits).
+template <bool kHeadGate, bool kRaw>
 __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs pa, const __grid_constant__ TcMaps maps)
 {
     extern __shared__ __align__(1024) uint8_t sm[];
@@ -886,14 +931,15 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs pa, const
     const int warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x;                 // sequence * H + head (state tile)
     const int h = bh % pa.H;
-    ChunkArgs p;
-    int b, row0;                               // batch index within the view, first token row
-    if (!sequence_view(pa, bh / pa.H, D, D, p, b, row0)) {
+    const ChunkArgs p = pa;
+    SeqSpan sp;                                // the sequence's token rows
+    if (!sequence_span(pa, bh / pa.H, sp)) {
         if (tid == 0 && pa.status) atomicOr(pa.status, 2u);
         return;
     }
-    const TmaPos tp{pa.cu_seqlens ? 0 : b, h, row0, pa.gate_per_head ? 0 : 1};
-    const int nchunks = (p.T + C - 1) / C;
+    // TMA coordinates: dense tensors by (batch, token); packed ones as one batch by token row
+    const TmaPos tp{pa.cu_seqlens ? 0 : bh / pa.H, h, pa.cu_seqlens ? (int)sp.tok0 : 0, pa.gate_per_head ? 0 : 1};
+    const int nchunks = (sp.len + C - 1) / C;
     if (nchunks == 0) {
         // an empty sequence: the final state is the initial one (or zeros)
         if (p.s_out) {
@@ -938,9 +984,9 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs pa, const
     if (warp == kIssuerWarp) {
         if (lane == 0) issuer(sm, tmem, bars, nchunks, err_flag);
     } else if (warp >= NCW) {
-        prep_role(p, maps, sm, tmem, bars, tp, b, h, nchunks, err_flag);
+        prep_role(p, maps, sm, tmem, bars, tp, sp, h, nchunks, err_flag);
     } else {
-        chain_role<kHeadGate>(p, maps, sm, tmem, bars, tp, b, h, bh, nchunks, err_flag);
+        chain_role<kHeadGate, kRaw>(p, maps, sm, tmem, bars, tp, sp, h, bh, nchunks, err_flag);
     }
     if (*err_flag && tid == 0 && p.status) atomicOr(p.status, 1u);
     ptx::tc_fence_before();
@@ -1031,7 +1077,10 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, int dk, int dv, cudaStream_t str
         (!a.gate_per_head && !encode_rows(&maps.a, a.alpha, mb, a.T, a.H)) || !encode_v(&maps.v, a.v, mb, a.T, a.H) ||
         !encode_out(&maps.o, a.o, mb, a.T, a.H, a.out_bf16))
         return cudaErrorInvalidValue;
-    auto kernel = a.gate_per_head ? tc::kda_chunk_tc_kernel<true> : tc::kda_chunk_tc_kernel<false>;
+    if (a.gate_per_head && a.raw_inputs) return cudaErrorInvalidValue;
+    auto kernel = a.gate_per_head ? tc::kda_chunk_tc_kernel<true, false>
+                  : a.raw_inputs  ? tc::kda_chunk_tc_kernel<false, true>
+                                  : tc::kda_chunk_tc_kernel<false, false>;
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     kernel<<<(unsigned)blocks, tc::NT, tc::SMEM_BYTES, stream>>>(a, maps);

@@ -35,6 +35,26 @@ __device__ __forceinline__ float log_alpha(float a)
     return fmaxf(__logf(fmaxf(a, 1e-38f)), kLogAlphaFloor);
 }
 
+// Fused input preprocessing.  Gate logit x: log alpha = -softplus(x) <= 0, clamped
+// like log_alpha; beta logit y: beta = sigmoid(y); a row is scaled by 1/||row||
+// (0 for a zero row).
+__device__ __forceinline__ float log_alpha_from_logit(float x)
+{
+    return fmaxf(-(fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)))), kLogAlphaFloor);
+}
+
+__device__ __forceinline__ float sigmoid_of(float y)
+{
+    const float e = expf(-fabsf(y));
+    const float s = 1.f / (1.f + e);
+    return y >= 0.f ? s : e * s;
+}
+
+__device__ __forceinline__ float inv_norm(float sum_sq)
+{
+    return sum_sq > 0.f ? rsqrtf(sum_sq) : 0.f;
+}
+
 __device__ __forceinline__ float4 ld_f4(const float *p)
 {
     return *reinterpret_cast<const float4 *>(p);

@@ -25,37 +25,65 @@ struct ChunkArgs {
     // One retention factor per (token, head) -- Gated DeltaNet's scalar gate -- with
     // alpha laid out [B, T, H]; 0 for the per-key-channel gate [B, T, H, d_k].
     int gate_per_head;
+    // GDN-2: a per-key-channel erase gate [B, T, H, d_k] and a per-value-channel write
+    // gate [B, T, H, d_v] (gate dtype) in place of beta; null for KDA.
+    const void *erase, *wgate;
+    // Decode over a pool of state slots: sequence b reads s_in and writes s_out at
+    // slot state_slots[b] (a negative slot skips the sequence; a slot >= num_slots is
+    // skipped and sets status bit 1).  Null: slot b.
+    const int *state_slots;
+    int num_slots;
+    // The state after each token, [B, T, H, DK, DV] fp32, or null.
+    float *token_states;
+    // Fused input preprocessing: q and k arrive un-normalised (each token's row is
+    // divided by its L2 norm), alpha holds gate logits x (log alpha = -softplus(x))
+    // and beta holds beta logits y (beta = sigmoid(y)).
+    int raw_inputs;
 };
 
-// The per-sequence view of a launch: with offsets, the sequence's rows are made
-// to look like a batch of one (base pointers advanced, T = its length).  Returns
-// false when the offsets of sequence b are invalid.
-__host__ __device__ inline bool sequence_view(const ChunkArgs &a, int b, int dk, int dv, ChunkArgs &s,
-                                              int &b_local, int &row0)
+// Where sequence b's token rows sit.  Dense tensors are [B, T, H, d] and sequence b
+// owns rows b*T .. b*T+T-1; with offsets they are [1, T, H, d] (T = total tokens) and
+// sequence b owns rows cu_seqlens[b] .. cu_seqlens[b+1]-1.  Kernels index rows as
+// (tok0 + t) * H + h and never derive shifted pointers.  Returns false when the
+// offsets of sequence b are invalid.
+struct SeqSpan {
+    size_t tok0;   // the sequence's first token row
+    int len;       // its number of tokens
+};
+
+__host__ __device__ inline bool sequence_span(const ChunkArgs &a, int b, SeqSpan &sp)
 {
-    s = a;
-    b_local = b;
-    row0 = 0;
-    if (!a.cu_seqlens) return true;
+    if (!a.cu_seqlens) {
+        sp.tok0 = (size_t)b * a.T;
+        sp.len = a.T;
+        return true;
+    }
     const int s0 = a.cu_seqlens[b], s1 = a.cu_seqlens[b + 1];
     if (s0 < 0 || s1 < s0 || s1 > a.T) return false;
-    const size_t rows = (size_t)s0 * a.H;   // token-head rows before the sequence
-    const size_t qe = a.qkv_bf16 ? 2 : 4, ge = a.gate_bf16 ? 2 : 4, oe = a.out_bf16 ? 2 : 4;
-    s.q = (const char *)a.q + rows * dk * qe;
-    s.k = (const char *)a.k + rows * dk * qe;
-    s.v = (const char *)a.v + rows * dv * qe;
-    s.alpha = (const char *)a.alpha + rows * (a.gate_per_head ? 1 : dk) * ge;
-    s.beta = (const char *)a.beta + rows * ge;
-    s.o = (char *)a.o + rows * dv * oe;
-    s.T = s1 - s0;
-    b_local = 0;
-    row0 = s0;
+    sp.tok0 = (size_t)s0;
+    sp.len = s1 - s0;
     return true;
 }
 using RecurrentArgs = ChunkArgs;
 
 cudaError_t launch_recurrent(const RecurrentArgs &a, int dk, int dv, cudaStream_t s);
+
+// Entry i copies the [H, DK, DV] block src[src_index[i]] to dst[dst_index[i]]
+// (identity index when null; negative: skipped; out of range: skipped, status bit 1).
+struct StateCopyArgs {
+    const float *src;
+    const int *src_index;
+    int src_slots;
+    float *dst;
+    const int *dst_index;
+    int dst_slots;
+    int count;
+    size_t vec_per_state;   // H * DK * DV / 4
+    unsigned int *status;   // device status word or null
+};
+cudaError_t launch_state_copy(const StateCopyArgs &a, cudaStream_t s);
 cudaError_t launch_chunk_simt(const ChunkArgs &a, int dk, int dv, cudaStream_t s);
+// (both take GDN-2 gates when a.erase is set)
 bool chunk_tc_supported(int dk, int dv, kda_dtype qkv, kda_dtype gate);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, int dk, int dv, cudaStream_t s);
 

@@ -11,7 +11,14 @@
 //      o = scale (p + e (k . q))   [o = S_t^T q with S_t = S~ + k e^T]
 //   D  S <- S~ + k e^T in registers
 // The decode step is this with T = 1 and the state read from and written back
-// to the same buffer; the state is read once and written once.
+// to the same buffer; the state is read once and written once.  Multi-token
+// decode (the T draft tokens of a speculative step) is this with T > 1 over a
+// pool of state slots, optionally storing the state after every token so that
+// the step can be rolled back to any accepted prefix.
+// Raw inputs: q and k are read un-normalised and their norms, found with k . q,
+// scale the two reads and the write; alpha = exp(-softplus(x)), beta = sigmoid(y).
+// GDN-2 ("From Fast Weight Programmers to KDA", section "Gated DeltaNet-2"):
+// r = S~^T (b * k) with the erase gate b, and e = w * v - r with the write gate w.
 // Recurrence: "Module 03 -- KDA I: The Delta-Rule Recurrence", section 2;
 // schedule: "Kimi Delta Attention (KDA)", "Two schedules for the same
 // recurrence" (fused recurrent).
@@ -30,22 +37,35 @@ struct RecurrentShape {
 };
 
 
-template <int DK, int DV>
+template <int DK, int DV, bool kGdn2>
 __global__ void __launch_bounds__(RecurrentShape<DK, DV>::NT)
 kda_recurrent_kernel(RecurrentArgs a)
 {
     using Sh = RecurrentShape<DK, DV>;
     constexpr int NCG = Sh::NCG, NRG = Sh::NRG, RPT = Sh::RPT, NT = Sh::NT;
 
-    __shared__ float s_q[2][DK], s_k[2][DK], s_a[2][DK], s_v[2][DV], s_e[2][DV];
-    __shared__ float s_beta[2], s_kq[2];
-    __shared__ float red_r[NRG][DV], red_p[NRG][DV];
+    // s_e, red_r and red_p are accessed as float4: their alignment is stated, not left to layout
+    __shared__ float s_q[2][DK], s_k[2][DK], s_a[2][DK], s_v[2][DV];
+    __shared__ __align__(16) float s_e[2][DV];
+    __shared__ float s_beta[2], s_kq[2], s_nk[2], s_nq[2];
+    __shared__ float s_b[kGdn2 ? 2 : 1][kGdn2 ? DK : 1], s_w[kGdn2 ? 2 : 1][kGdn2 ? DV : 1];
+    __shared__ __align__(16) float red_r[NRG][DV];
+    __shared__ __align__(16) float red_p[NRG][DV];
 
     const int bh = blockIdx.x;           // b * H + h
     const int b = bh / a.H, h = bh % a.H;
     const int tid = threadIdx.x;
     const int cg = tid % NCG, rg = tid / NCG;
-    const size_t tile = (size_t)bh * DK * DV;
+    int slot = b;
+    if (a.state_slots) {   // decode over a slot pool
+        slot = a.state_slots[b];
+        if (slot < 0) return;
+        if (slot >= a.num_slots) {
+            if (tid == 0 && a.status) atomicOr(a.status, 2u);
+            return;
+        }
+    }
+    const size_t tile = ((size_t)slot * a.H + h) * DK * DV;
 
     float4 s[RPT];
 #pragma unroll
@@ -62,10 +82,19 @@ kda_recurrent_kernel(RecurrentArgs a)
         for (int i = tid; i < DK; i += NT) {
             s_q[buf][i] = ld_elem(a.q, row * DK + i, a.qkv_bf16);
             s_k[buf][i] = ld_elem(a.k, row * DK + i, a.qkv_bf16);
-            s_a[buf][i] = ld_elem(a.alpha, a.gate_per_head ? row : row * DK + i, a.gate_bf16);
+            const float x = ld_elem(a.alpha, a.gate_per_head ? row : row * DK + i, a.gate_bf16);
+            s_a[buf][i] = a.raw_inputs ? __expf(log_alpha_from_logit(x)) : x;
         }
         for (int j = tid; j < DV; j += NT) s_v[buf][j] = ld_elem(a.v, row * DV + j, a.qkv_bf16);
-        if (tid == 0) s_beta[buf] = ld_elem(a.beta, row, a.gate_bf16);
+        if constexpr (kGdn2) {
+            for (int i = tid; i < DK; i += NT) s_b[buf][i] = ld_elem(a.erase, row * DK + i, a.gate_bf16);
+            for (int j = tid; j < DV; j += NT) s_w[buf][j] = ld_elem(a.wgate, row * DV + j, a.gate_bf16);
+        } else {
+            if (tid == 0) {
+                const float y = ld_elem(a.beta, row, a.gate_bf16);
+                s_beta[buf] = a.raw_inputs ? sigmoid_of(y) : y;
+            }
+        }
         __syncthreads();
 
         // B: decay in registers and the two partial reductions
@@ -73,7 +102,8 @@ kda_recurrent_kernel(RecurrentArgs a)
 #pragma unroll
         for (int m = 0; m < RPT; ++m) {
             const int i = rg + NRG * m;
-            const float al = s_a[buf][i], kk = s_k[buf][i], qq = s_q[buf][i];
+            const float al = s_a[buf][i], qq = s_q[buf][i];
+            const float kk = kGdn2 ? s_b[buf][i] * s_k[buf][i] : s_k[buf][i];   // retrieval key
             s[m].x *= al; s[m].y *= al; s[m].z *= al; s[m].w *= al;
             r.x = fmaf(kk, s[m].x, r.x); r.y = fmaf(kk, s[m].y, r.y);
             r.z = fmaf(kk, s[m].z, r.z); r.w = fmaf(kk, s[m].w, r.w);
@@ -82,12 +112,26 @@ kda_recurrent_kernel(RecurrentArgs a)
         }
         *reinterpret_cast<float4 *>(&red_r[rg][4 * cg]) = r;
         *reinterpret_cast<float4 *>(&red_p[rg][4 * cg]) = p;
-        if (tid < 32) {   // k . q over the key channels
-            float kq = 0.f;
-            for (int i = tid; i < DK; i += 32) kq = fmaf(s_k[buf][i], s_q[buf][i], kq);
+        if (tid < 32) {   // k . q over the key channels (and, for raw inputs, the norms)
+            float kq = 0.f, kk = 0.f, qq = 0.f;
+            for (int i = tid; i < DK; i += 32) {
+                const float ki = s_k[buf][i], qi = s_q[buf][i];
+                kq = fmaf(ki, qi, kq);
+                kk = fmaf(ki, ki, kk);
+                qq = fmaf(qi, qi, qq);
+            }
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
-            if (tid == 0) s_kq[buf] = kq;
+            for (int off = 16; off > 0; off >>= 1) {
+                kq += __shfl_xor_sync(0xffffffffu, kq, off);
+                kk += __shfl_xor_sync(0xffffffffu, kk, off);
+                qq += __shfl_xor_sync(0xffffffffu, qq, off);
+            }
+            if (tid == 0) {
+                const float nk = a.raw_inputs ? inv_norm(kk) : 1.f, nq = a.raw_inputs ? inv_norm(qq) : 1.f;
+                s_kq[buf] = kq * nk * nq;
+                s_nk[buf] = nk;
+                s_nq[buf] = nq;
+            }
         }
         __syncthreads();
 
@@ -96,7 +140,9 @@ kda_recurrent_kernel(RecurrentArgs a)
             float rr = 0.f, pp = 0.f;
 #pragma unroll
             for (int g = 0; g < NRG; ++g) { rr += red_r[g][j]; pp += red_p[g][j]; }
-            const float e = s_beta[buf] * (s_v[buf][j] - rr);
+            rr *= s_nk[buf];   // reads with the unit key and query (1 unless inputs are raw)
+            pp *= s_nq[buf];
+            const float e = kGdn2 ? s_w[buf][j] * s_v[buf][j] - rr : s_beta[buf] * (s_v[buf][j] - rr);
             s_e[buf][j] = e;
             st_elem(a.o, row * DV + j, a.scale * fmaf(e, s_kq[buf], pp), a.out_bf16);
         }
@@ -106,9 +152,14 @@ kda_recurrent_kernel(RecurrentArgs a)
         const float4 e4 = *reinterpret_cast<const float4 *>(&s_e[buf][4 * cg]);
 #pragma unroll
         for (int m = 0; m < RPT; ++m) {
-            const float kk = s_k[buf][rg + NRG * m];
+            const float kk = s_k[buf][rg + NRG * m] * s_nk[buf];
             s[m].x = fmaf(kk, e4.x, s[m].x); s[m].y = fmaf(kk, e4.y, s[m].y);
             s[m].z = fmaf(kk, e4.z, s[m].z); s[m].w = fmaf(kk, e4.w, s[m].w);
+        }
+        if (a.token_states) {   // the state after this token
+            float *ts = a.token_states + (((size_t)b * a.T + t) * a.H + h) * DK * DV;
+#pragma unroll
+            for (int m = 0; m < RPT; ++m) st_f4_stream(ts + (size_t)(rg + NRG * m) * DV + 4 * cg, s[m]);
         }
     }
 
@@ -127,7 +178,10 @@ static cudaError_t launch_recurrent_t(const RecurrentArgs &a, cudaStream_t strea
     using Sh = RecurrentShape<DK, DV>;
     const long long blocks = (long long)a.B * a.H;
     if (blocks == 0) return cudaSuccess;
-    kda_recurrent_kernel<DK, DV><<<(unsigned)blocks, Sh::NT, 0, stream>>>(a);
+    if (a.erase)
+        kda_recurrent_kernel<DK, DV, true><<<(unsigned)blocks, Sh::NT, 0, stream>>>(a);
+    else
+        kda_recurrent_kernel<DK, DV, false><<<(unsigned)blocks, Sh::NT, 0, stream>>>(a);
     return cudaGetLastError();
 }
 

@@ -15,9 +15,10 @@ import threading
 
 import torch
 
-__all__ = ["KDAError", "forward", "forward_varlen", "forward_scalar_gate", "forward_sequential",
-           "decode_step", "decode_step_scalar_gate", "library", "library_path", "status_string",
-           "version", "EXPORTED_SYMBOLS"]
+__all__ = ["KDAError", "forward", "forward_varlen", "forward_scalar_gate", "forward_gdn2",
+           "forward_raw", "forward_sequential", "decode_step", "decode_step_raw",
+           "decode_step_scalar_gate", "decode_step_gdn2", "decode_tokens", "state_copy", "library",
+           "library_path", "status_string", "version", "EXPORTED_SYMBOLS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libkda_b200.so")
@@ -26,8 +27,9 @@ _lock = threading.Lock()
 
 EXPORTED_SYMBOLS = ("kda_forward", "kda_forward_workspace_bytes", "kda_workspace_status",
                     "kda_forward_noalloc", "kda_forward_varlen", "kda_forward_scalar_gate",
-                    "kda_forward_sequential", "kda_decode_step", "kda_decode_step_scalar_gate",
-                    "kda_status_string", "kda_version")
+                    "kda_forward_gdn2", "kda_forward_raw", "kda_forward_sequential", "kda_decode_step",
+                    "kda_decode_step_gdn2", "kda_decode_step_raw", "kda_decode_step_scalar_gate",
+                    "kda_decode_tokens", "kda_state_copy", "kda_status_string", "kda_version")
 
 _DT = {torch.float32: 0, torch.bfloat16: 1}
 _vp = ctypes.c_void_p
@@ -68,8 +70,22 @@ def library() -> ctypes.CDLL:
             lib.kda_forward_varlen.restype = _i
             lib.kda_forward_scalar_gate.argtypes = fwd_args + [_vp, ctypes.c_size_t, _vp]
             lib.kda_forward_scalar_gate.restype = _i
+            lib.kda_forward_raw.argtypes = fwd_args + [_vp, ctypes.c_size_t, _vp]
+            lib.kda_forward_raw.restype = _i
+            lib.kda_decode_step_raw.argtypes = [_vp] * 7 + [_i] * 4 + [_f] + [_i] * 3 + [_vp]
+            lib.kda_decode_step_raw.restype = _i
             lib.kda_decode_step_scalar_gate.argtypes = [_vp] * 7 + [_i] * 4 + [_f] + [_i] * 3 + [_vp]
             lib.kda_decode_step_scalar_gate.restype = _i
+            lib.kda_forward_gdn2.argtypes = [_vp] * 9 + [_i] * 5 + [_f] + [_i] * 3 + \
+                [_vp, ctypes.c_size_t, _vp]
+            lib.kda_forward_gdn2.restype = _i
+            lib.kda_decode_step_gdn2.argtypes = [_vp] * 8 + [_i] * 4 + [_f] + [_i] * 3 + [_vp]
+            lib.kda_decode_step_gdn2.restype = _i
+            lib.kda_decode_tokens.argtypes = [_vp] * 6 + [_vp, _i, _i, _vp, _vp] + [_i] * 5 + [_f] + \
+                [_i] * 3 + [_vp, _vp]
+            lib.kda_decode_tokens.restype = _i
+            lib.kda_state_copy.argtypes = [_vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp]
+            lib.kda_state_copy.restype = _i
             lib.kda_forward_workspace_bytes.argtypes = [_i] * 5
             lib.kda_forward_workspace_bytes.restype = ctypes.c_size_t
             lib.kda_workspace_status.argtypes = [_vp, _vp]
@@ -166,7 +182,7 @@ def _prefill(fn_name, q, k, v, alpha, beta, initial_state, scale, output_final_s
             _dt(out, "out")]
     with torch.cuda.device(device):
         stream = _vp(_stream_handle(device))
-        if fn_name in ("kda_forward", "kda_forward_scalar_gate"):
+        if fn_name in ("kda_forward", "kda_forward_scalar_gate", "kda_forward_raw"):
             ws_bytes = lib.kda_forward_workspace_bytes(B, T, H, dk, dv)
             ws = workspace
             if ws is None or ws.numel() * ws.element_size() < ws_bytes:
@@ -219,6 +235,16 @@ def forward_scalar_gate(q, k, v, alpha, beta, initial_state=None, scale=None, ou
                     gate_per_head=True)
 
 
+def forward_raw(q, k, v, gate_logit, beta_logit, initial_state=None, scale=None, output_final_state=True,
+                out_dtype=torch.float32, out=None, final_state=None, workspace=None, check_status=False):
+    """Prefill with the input preprocessing fused into the kernels (C entry point
+    ``kda_forward_raw``): q, k un-normalised (each row divided by its L2 norm in the
+    kernel), gate_logit [B,T,H,dk] with alpha = exp(-softplus(x)), beta_logit [B,T,H]
+    with beta = sigmoid(y); otherwise the contract of ``forward``."""
+    return _prefill("kda_forward_raw", q, k, v, gate_logit, beta_logit, initial_state, scale,
+                    output_final_state, out_dtype, out, final_state, workspace, check_status)
+
+
 def forward_sequential(q, k, v, alpha, beta, initial_state=None, scale=None,
                        output_final_state=True, out_dtype=torch.float32, out=None,
                        final_state=None):
@@ -228,7 +254,7 @@ def forward_sequential(q, k, v, alpha, beta, initial_state=None, scale=None,
 
 
 def decode_step(q, k, v, alpha, beta, state, scale=None, out_dtype=torch.float32, out=None,
-                _gate_per_head=False):
+                _gate_per_head=False, _fn="kda_decode_step"):
     """One token per sequence; ``state`` [N,H,dk,dv] float32 is updated in place.
 
     q, k, alpha: [N,H,dk]; v: [N,H,dv]; beta: [N,H].  Returns o [N,H,dv].
@@ -256,7 +282,7 @@ def decode_step(q, k, v, alpha, beta, state, scale=None, out_dtype=torch.float32
         out = torch.empty((N, H, dv), device=device, dtype=out_dtype)
     _check("out", out, device)
     with torch.cuda.device(device):
-        fn = "kda_decode_step_scalar_gate" if _gate_per_head else "kda_decode_step"
+        fn = "kda_decode_step_scalar_gate" if _gate_per_head else _fn
         code = getattr(library(), fn)(
             _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state), _ptr(out),
             N, H, dk, dv, float(scale), _DT[q.dtype], _dt(alpha, "alpha"), _dt(out, "out"),
@@ -270,6 +296,12 @@ def decode_step_scalar_gate(q, k, v, alpha, beta, state, scale=None, out_dtype=t
     """Gated DeltaNet decode step: alpha [N,H], one retention factor per (sequence, head)
     (C entry point ``kda_decode_step_scalar_gate``); otherwise the contract of ``decode_step``."""
     return decode_step(q, k, v, alpha, beta, state, scale, out_dtype, out, _gate_per_head=True)
+
+
+def decode_step_raw(q, k, v, gate_logit, beta_logit, state, scale=None, out_dtype=torch.float32, out=None):
+    """Decode step on raw inputs (C entry point ``kda_decode_step_raw``): the preprocessing
+    of ``forward_raw``; otherwise the contract of ``decode_step``."""
+    return decode_step(q, k, v, gate_logit, beta_logit, state, scale, out_dtype, out, _fn="kda_decode_step_raw")
 
 
 def forward_varlen(q, k, v, alpha, beta, cu_seqlens, initial_state=None, scale=None,
@@ -333,3 +365,172 @@ def forward_varlen(q, k, v, alpha, beta, cu_seqlens, initial_state=None, scale=N
     if code != 0:
         raise KDAError("kda_forward_varlen", code)
     return (out.unsqueeze(0) if squeeze else out), final_state
+
+
+def forward_gdn2(q, k, v, alpha, erase, write, initial_state=None, scale=None, output_final_state=True,
+                 out_dtype=torch.float32, out=None, final_state=None, workspace=None, check_status=False):
+    """GDN-2 prefill (C entry point ``kda_forward_gdn2``): erase [B,T,H,dk] and write
+    [B,T,H,dv] gates (alpha's dtype) in place of beta; otherwise the contract of ``forward``."""
+    device = q.device
+    if device.type != "cuda":
+        raise ValueError("KDA runs on CUDA devices only")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for name, t in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("erase", erase), ("write", write)):
+        _check(name, t, device)
+    if tuple(k.shape) != (B, T, H, dk) or tuple(alpha.shape) != (B, T, H, dk) or \
+            tuple(erase.shape) != (B, T, H, dk) or tuple(v.shape) != (B, T, H, dv) or \
+            tuple(write.shape) != (B, T, H, dv):
+        raise ValueError("shapes: q,k,alpha,erase [B,T,H,dk], v,write [B,T,H,dv]")
+    if k.dtype != q.dtype or v.dtype != q.dtype or erase.dtype != alpha.dtype or write.dtype != alpha.dtype:
+        raise TypeError("q/k/v and alpha/erase/write must each share a dtype")
+    if initial_state is not None:
+        _check("initial_state", initial_state, device)
+        if initial_state.dtype != torch.float32 or tuple(initial_state.shape) != (B, H, dk, dv):
+            raise ValueError("initial_state must be float32 [B,H,dk,dv]")
+    if scale is None:
+        scale = dk ** -0.5
+    if out is None:
+        out = torch.empty((B, T, H, dv), device=device, dtype=out_dtype)
+    _check("out", out, device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((B, H, dk, dv), device=device, dtype=torch.float32)
+    if final_state is not None:
+        _check("final_state", final_state, device)
+    lib = library()
+    with torch.cuda.device(device):
+        stream = _vp(_stream_handle(device))
+        ws_bytes = lib.kda_forward_workspace_bytes(B, T, H, dk, dv)
+        ws = workspace
+        if ws is None or ws.numel() * ws.element_size() < ws_bytes:
+            ws = torch.empty(max(ws_bytes, 16), device=device, dtype=torch.uint8)
+        code = lib.kda_forward_gdn2(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(erase), _ptr(write), _ptr(initial_state),
+            _ptr(out), _ptr(final_state), B, T, H, dk, dv, float(scale), _DT[q.dtype],
+            _dt(alpha, "alpha"), _dt(out, "out"), _ptr(ws), ws.numel() * ws.element_size(), stream)
+        if code == 0 and check_status:
+            code = lib.kda_workspace_status(_ptr(ws), stream)
+    if code != 0:
+        raise KDAError("kda_forward_gdn2", code)
+    return out, final_state
+
+
+def decode_step_gdn2(q, k, v, alpha, erase, write, state, scale=None, out_dtype=torch.float32, out=None):
+    """GDN-2 decode step (C entry point ``kda_decode_step_gdn2``): erase [N,H,dk] and write
+    [N,H,dv] in place of beta; ``state`` [N,H,dk,dv] float32 is updated in place."""
+    device = state.device
+    N, H, dk, dv = state.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("erase", erase), ("write", write),
+                    ("state", state)):
+        _check(name, t, device)
+    if tuple(q.shape) != (N, H, dk) or tuple(k.shape) != (N, H, dk) or tuple(alpha.shape) != (N, H, dk) \
+            or tuple(erase.shape) != (N, H, dk) or tuple(v.shape) != (N, H, dv) or tuple(write.shape) != (N, H, dv):
+        raise ValueError("shapes: q,k,alpha,erase [N,H,dk], v,write [N,H,dv], state [N,H,dk,dv]")
+    if scale is None:
+        scale = dk ** -0.5
+    if out is None:
+        out = torch.empty((N, H, dv), device=device, dtype=out_dtype)
+    _check("out", out, device)
+    with torch.cuda.device(device):
+        code = library().kda_decode_step_gdn2(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(erase), _ptr(write), _ptr(state), _ptr(out),
+            N, H, dk, dv, float(scale), _DT[q.dtype], _dt(alpha, "alpha"), _dt(out, "out"),
+            _vp(_stream_handle(device)))
+    if code != 0:
+        raise KDAError("kda_decode_step_gdn2", code)
+    return out
+
+
+def _status_word(device):
+    return torch.zeros(16, device=device, dtype=torch.uint8)
+
+
+def decode_tokens(q, k, v, alpha, beta, state, state_slots=None, commit=True, token_states=None,
+                  scale=None, out_dtype=torch.float32, out=None, check_status=False):
+    """T tokens per sequence through the decode recurrence (C entry point ``kda_decode_tokens``).
+
+    q, k, alpha [N,T,H,dk]; v [N,T,H,dv]; beta [N,T,H]; ``state`` is a pool
+    [slots,H,dk,dv] float32; sequence n uses slot ``state_slots[n]`` (int32 [N] on the
+    device; None: slot n; negative: skipped).  ``commit`` writes the state after the
+    T tokens back to the slot; ``token_states`` ([N,T,H,dk,dv] float32, or True to
+    allocate one) receives the state after every token.  Returns (o [N,T,H,dv],
+    token_states or None).
+    """
+    device = state.device
+    if device.type != "cuda":
+        raise ValueError("decode_tokens needs the state pool on a CUDA device")
+    slots, H, dk, dv = state.shape
+    N, T = q.shape[0], q.shape[1]
+    for name, t in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta", beta), ("state", state)):
+        _check(name, t, device)
+    if state.dtype != torch.float32:
+        raise TypeError("state must be float32")
+    if tuple(q.shape) != (N, T, H, dk) or tuple(k.shape) != (N, T, H, dk) or \
+            tuple(alpha.shape) != (N, T, H, dk) or tuple(v.shape) != (N, T, H, dv) or \
+            tuple(beta.shape) != (N, T, H):
+        raise ValueError("shapes: q,k,alpha [N,T,H,dk], v [N,T,H,dv], beta [N,T,H], state [slots,H,dk,dv]")
+    if k.dtype != q.dtype or v.dtype != q.dtype or alpha.dtype != beta.dtype:
+        raise TypeError("q/k/v and alpha/beta must each share a dtype")
+    if state_slots is not None:
+        _check("state_slots", state_slots, device)
+        if state_slots.dtype != torch.int32 or tuple(state_slots.shape) != (N,):
+            raise ValueError("state_slots must be int32 [N]")
+    if token_states is True:
+        token_states = torch.empty((N, T, H, dk, dv), device=device, dtype=torch.float32)
+    if token_states is not None:
+        _check("token_states", token_states, device)
+        if token_states.dtype != torch.float32 or tuple(token_states.shape) != (N, T, H, dk, dv):
+            raise ValueError("token_states must be float32 [N,T,H,dk,dv]")
+    if scale is None:
+        scale = dk ** -0.5
+    if out is None:
+        out = torch.empty((N, T, H, dv), device=device, dtype=out_dtype)
+    _check("out", out, device)
+    status = _status_word(device) if check_status else None
+    lib = library()
+    with torch.cuda.device(device):
+        stream = _vp(_stream_handle(device))
+        code = lib.kda_decode_tokens(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state), _ptr(state_slots), slots,
+            int(bool(commit)), _ptr(token_states), _ptr(out), N, T, H, dk, dv, float(scale), _DT[q.dtype],
+            _dt(alpha, "alpha"), _dt(out, "out"), _ptr(status), stream)
+        if code == 0 and status is not None:
+            code = lib.kda_workspace_status(_ptr(status), stream)
+    if code != 0:
+        raise KDAError("kda_decode_tokens", code)
+    return out, token_states
+
+
+def state_copy(src, dst, src_index=None, dst_index=None, count=None, check_status=False):
+    """Copy whole states between pools (C entry point ``kda_state_copy``): entry i copies
+    ``src[src_index[i]]`` to ``dst[dst_index[i]]`` (int32 [count] on the device; None:
+    identity; negative: skipped).  ``src`` and ``dst`` are float32 [slots,H,dk,dv] and
+    may be the same tensor (a fork inside one pool)."""
+    device = dst.device
+    if device.type != "cuda":
+        raise ValueError("state_copy needs CUDA tensors")
+    _check("src", src, device)
+    _check("dst", dst, device)
+    if src.dtype != torch.float32 or dst.dtype != torch.float32 or src.dim() != 4 or \
+            tuple(src.shape[1:]) != tuple(dst.shape[1:]):
+        raise ValueError("src and dst must be float32 [slots,H,dk,dv] with equal H, dk, dv")
+    for name, t in (("src_index", src_index), ("dst_index", dst_index)):
+        if t is not None:
+            _check(name, t, device)
+            if t.dtype != torch.int32 or t.dim() != 1:
+                raise ValueError(name + " must be int32 [count]")
+    if count is None:
+        idx = src_index if src_index is not None else dst_index
+        count = idx.numel() if idx is not None else min(src.shape[0], dst.shape[0])
+    _, H, dk, dv = dst.shape
+    status = _status_word(device) if check_status else None
+    lib = library()
+    with torch.cuda.device(device):
+        stream = _vp(_stream_handle(device))
+        code = lib.kda_state_copy(_ptr(src), _ptr(src_index), src.shape[0], _ptr(dst), _ptr(dst_index),
+                                  dst.shape[0], int(count), H, dk, dv, _ptr(status), stream)
+        if code == 0 and status is not None:
+            code = lib.kda_workspace_status(_ptr(status), stream)
+    if code != 0:
+        raise KDAError("kda_state_copy", code)
+    return dst

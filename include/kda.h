@@ -186,6 +186,31 @@ kda_status kda_forward_scalar_gate(const void *q, const void *k, const void *v,
                                    size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * kda_forward_gdn2 -- prefill of GDN-2, the gated delta rule with decoupled
+ * gates ("From Fast Weight Programmers to KDA", jonahsamost.bearblog.dev,
+ * section "Gated DeltaNet-2"): beta_t is replaced by an erase gate b_t (one
+ * per key channel) and a write gate w_t (one per value channel):
+ *
+ *   S~_t = Diag(alpha_t) S_{t-1},  vh_t = S~_t^T (b_t * k_t),
+ *   S_t  = S~_t + k_t (w_t * v_t - vh_t)^T,  o_t = S_t^T (scale q_t)
+ *
+ * (* elementwise; that page writes the state transposed).  b_t = beta_t 1 and
+ * w_t = beta_t 1 give kda_forward.  Arguments as kda_forward with
+ *   erase [B, T, H, d_k] and write [B, T, H, d_v]  (gate_dtype, 16-byte
+ *   aligned) in place of beta.
+ * Computed by the chunkwise schedule on CUDA cores, fp32, every supported head
+ * size and dtype.
+ */
+kda_status kda_forward_gdn2(const void *q, const void *k, const void *v,
+                            const void *alpha, const void *erase,
+                            const void *write, const float *initial_state,
+                            void *o, float *final_state, int B, int T, int H,
+                            int d_k, int d_v, float scale, kda_dtype qkv_dtype,
+                            kda_dtype gate_dtype, kda_dtype out_dtype,
+                            void *workspace, size_t workspace_bytes,
+                            cudaStream_t stream);
+
+/*
  * kda_forward_sequential -- the same operation and arguments as kda_forward
  * (no workspace), computed with the token-by-token schedule ("fused
  * recurrent" in "Two schedules for the same recurrence", brain.bigb.es): one
@@ -231,6 +256,113 @@ kda_status kda_decode_step_scalar_gate(const void *q, const void *k,
                                        kda_dtype gate_dtype,
                                        kda_dtype out_dtype,
                                        cudaStream_t stream);
+
+/*
+ * kda_forward_raw -- kda_forward with the input preprocessing fused into the
+ * kernels' load stage, so that no separate pass over the inputs is needed:
+ *   q, k        un-normalised projections; each token's q_t and k_t are
+ *               divided by their L2 norms in the kernel (a zero row stays
+ *               zero) -- "Notes on Linear Attention: From Linear Attention to
+ *               KDA", section 5.3 "Why L2-normalize the key?" (and the
+ *               query, as later DeltaNet-style models do: section 3)
+ *   gate_logit  [B, T, H, d_k] gate_dtype: x with log alpha = -softplus(x),
+ *               i.e. alpha = 1 / (1 + e^x) -- the log-decay g = log alpha <= 0
+ *               that implementations keep ("Kimi Delta Attention (KDA)",
+ *               brain.bigb.es), in the exp(-softplus) form of the gate
+ *   beta_logit  [B, T, H] gate_dtype: y with beta = sigmoid(y) ("From Fast
+ *               Weight Programmers to KDA", the delta rule's write strength)
+ * Everything else (layouts, workspace, aliasing, status) is as kda_forward.
+ */
+kda_status kda_forward_raw(const void *q, const void *k, const void *v,
+                           const void *gate_logit, const void *beta_logit,
+                           const float *initial_state, void *o,
+                           float *final_state, int B, int T, int H, int d_k,
+                           int d_v, float scale, kda_dtype qkv_dtype,
+                           kda_dtype gate_dtype, kda_dtype out_dtype,
+                           void *workspace, size_t workspace_bytes,
+                           cudaStream_t stream);
+
+/*
+ * kda_decode_step_raw -- kda_decode_step on raw inputs (the preprocessing of
+ * kda_forward_raw): q, k [N, H, d_k] un-normalised, gate_logit [N, H, d_k],
+ * beta_logit [N, H]; the state [N, H, d_k, d_v] is updated in place.
+ */
+kda_status kda_decode_step_raw(const void *q, const void *k, const void *v,
+                               const void *gate_logit, const void *beta_logit,
+                               float *state, void *o, int N, int H, int d_k,
+                               int d_v, float scale, kda_dtype qkv_dtype,
+                               kda_dtype gate_dtype, kda_dtype out_dtype,
+                               cudaStream_t stream);
+
+/*
+ * kda_decode_step_gdn2 -- kda_decode_step for GDN-2 (see kda_forward_gdn2):
+ * erase [N, H, d_k] and write [N, H, d_v] (gate_dtype, 16-byte aligned) in
+ * place of beta; the state [N, H, d_k, d_v] is updated in place.
+ */
+kda_status kda_decode_step_gdn2(const void *q, const void *k, const void *v,
+                                const void *alpha, const void *erase,
+                                const void *write, float *state, void *o,
+                                int N, int H, int d_k, int d_v, float scale,
+                                kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                                kda_dtype out_dtype, cudaStream_t stream);
+
+/*
+ * Serving operations.  A recurrent state is request-scoped, like a KV-cache
+ * slot: it is cached between turns and must be copied whenever a request is
+ * forked, shares a prefix, migrates or is rolled back after a speculative
+ * step ("Module 03 -- KDA I: The Delta-Rule Recurrence", section 5 "State vs.
+ * checkpoint weights").  States live in pools of slots [slots, H, d_k, d_v]
+ * fp32.
+ *
+ * kda_decode_tokens -- T tokens per sequence through the recurrence of
+ * kda_decode_step, token after token (the draft tokens of a speculative step;
+ * T = 1 is a plain decode step over a slot pool).
+ *   q, k, alpha   [N, T, H, d_k]   v [N, T, H, d_v]   beta [N, T, H]
+ *   o             [N, T, H, d_v]   out_dtype (written)
+ *   state         pool [num_slots, H, d_k, d_v] fp32; sequence n starts from
+ *                 slot state_slots[n] (slot n when state_slots is NULL, then
+ *                 num_slots >= N is required).  A negative slot skips the
+ *                 sequence (its rows of o are not written); a slot >=
+ *                 num_slots is skipped too and recorded in the status word.
+ *   commit        nonzero: the state after the T tokens is written back to the
+ *                 sequence's slot; zero: the pool is only read (verification).
+ *   token_states  [N, T, H, d_k, d_v] fp32 or NULL: the state after each
+ *                 token, so that a rejected suffix can be rolled back with
+ *                 kda_state_copy (accepted prefix of a_n >= 1 tokens: source
+ *                 index n*T + a_n - 1 of token_states viewed as N*T slots).
+ *   status        NULL or a 16-byte-aligned device word (for instance a
+ *                 workspace of kda_forward_workspace_bytes() bytes), zeroed
+ *                 by the call; read it with kda_workspace_status()
+ *                 (KDA_ERR_SHAPE: a slot index was out of range).
+ * Two sequences must not name the same slot when commit is set.  o, the pool
+ * and token_states must not overlap (KDA_ERR_ALIAS).
+ */
+kda_status kda_decode_tokens(const void *q, const void *k, const void *v,
+                             const void *alpha, const void *beta, float *state,
+                             const int *state_slots, int num_slots, int commit,
+                             float *token_states, void *o, int N, int T, int H,
+                             int d_k, int d_v, float scale, kda_dtype qkv_dtype,
+                             kda_dtype gate_dtype, kda_dtype out_dtype,
+                             void *status, cudaStream_t stream);
+
+/*
+ * kda_state_copy -- entry i (i < count) copies the state block
+ * src[src_index[i]] to dst[dst_index[i]], each block [H, d_k, d_v] fp32.
+ *   src, dst      pools of src_slots and dst_slots blocks (may be the same
+ *                 pool: a fork inside one pool)
+ *   src_index, dst_index  [count] int32 on the device, or NULL for the
+ *                 identity index i (then count may not exceed that pool's
+ *                 slots).  An entry with a negative index is skipped; one with
+ *                 an index past its pool is skipped and recorded in the status
+ *                 word (KDA_ERR_SHAPE from kda_workspace_status()).
+ *   status        as for kda_decode_tokens.
+ * A block that one entry writes must not be read or written by another entry
+ * of the same call.  The copy is asynchronous on `stream`.
+ */
+kda_status kda_state_copy(const float *src, const int *src_index, int src_slots,
+                          float *dst, const int *dst_index, int dst_slots,
+                          int count, int H, int d_k, int d_v, void *status,
+                          cudaStream_t stream);
 
 /* Static, NUL-terminated description of a status code. */
 const char *kda_status_string(kda_status status);

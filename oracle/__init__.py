@@ -10,7 +10,12 @@ Delta-Rule Recurrence", section 2, in C (``kda_oracle.c``), in fp64, over all
 (sequence, head) pairs.  ``decode_step`` is the same loop for one token.
 ``forward_gdn2`` is the same loop with the decoupled erase and write gates of
 "From Fast Weight Programmers to KDA", section "Gated DeltaNet-2".
-``chunked.forward_chunked`` (numpy, fp64) is the second schedule of "Kimi Delta
+``forward_raw`` applies the input preprocessing in fp64 first (q and k divided by
+their L2 norms, log alpha = -softplus(gate logit), beta = sigmoid(beta logit)) and
+then runs ``forward``.  ``token_states`` gives the state after every token (the forward loop run on each
+prefix) and ``state_copy`` the whole-state copy between slot pools, the two
+serving operations of "Module 03 -- KDA I", section 5 "State vs. checkpoint
+weights".  ``chunked.forward_chunked`` (numpy, fp64) is the second schedule of "Kimi Delta
 Attention (KDA)", "Two schedules for the same recurrence"; the tests pin it to
 the sequential loop.
 
@@ -149,3 +154,64 @@ def decode_step(q, k, v, alpha, beta, state, scale=None, mode="exact"):
     o, s = forward(q[:, None], k[:, None], v[:, None], alpha[:, None], beta[:, None],
                    s0=state, scale=scale, mode=mode)
     return o[:, 0], s
+
+
+def token_states(q, k, v, alpha, beta, s0=None, scale=None):
+    """State after each token, [B,T,H,dk,dv] fp64: entry t is the final state of ``forward``
+    run on tokens 0..t.  A state is request-scoped and a speculative step is rolled back
+    to the state after its last accepted token ("Module 03 -- KDA I", section 5)."""
+    q = _f64(q)
+    B, T, H, dk = q.shape
+    dv = _f64(v).shape[-1]
+    out = np.zeros((B, T, H, dk, dv))
+    for t in range(T):
+        sl = lambda x: _f64(x)[:, :t + 1]
+        _, S = forward(sl(q), sl(k), sl(v), sl(alpha), sl(beta), s0=s0, scale=scale)
+        out[:, t] = S
+    return out
+
+
+def state_copy(src, dst, src_index=None, dst_index=None, count=None):
+    """Whole-state copy between slot pools, on copies of the arrays: entry i sets
+    dst[dst_index[i]] = src[src_index[i]] (identity index when None); entries with a
+    negative or out-of-range index are skipped.  Returns (new dst, any index out of range)."""
+    src, dst = np.array(src, dtype=np.float64), np.array(dst, dtype=np.float64)
+    if count is None:
+        idx = src_index if src_index is not None else dst_index
+        count = len(idx) if idx is not None else min(len(src), len(dst))
+    bad = False
+    for i in range(count):
+        si = int(src_index[i]) if src_index is not None else i
+        di = int(dst_index[i]) if dst_index is not None else i
+        if si < 0 or di < 0:
+            continue
+        if si >= len(src) or di >= len(dst):
+            bad = True
+            continue
+        dst[di] = src[si]
+    return dst, bad
+
+
+def preprocess(q, k, gate_logit, beta_logit):
+    """The input preprocessing, in fp64: q_t / ||q_t|| and k_t / ||k_t|| (a zero row stays
+    zero; "Notes on Linear Attention", section 5.3 "Why L2-normalize the key?"),
+    alpha = exp(-softplus(x)) (the stored log-decay g = log alpha = -softplus(x) <= 0,
+    "Kimi Delta Attention (KDA)"), beta = sigmoid(y) ("From Fast Weight Programmers to
+    KDA", the delta rule's learned write strength).  Returns (q, k, alpha, beta)."""
+    def unit(x):
+        x = _f64(x)
+        n = np.sqrt(np.sum(x * x, axis=-1, keepdims=True))
+        return np.divide(x, n, out=np.zeros_like(x), where=n > 0)
+
+    x = _f64(gate_logit)
+    softplus = np.maximum(x, 0.0) + np.log1p(np.exp(-np.abs(x)))
+    y = _f64(beta_logit)
+    beta = np.where(y >= 0, 1.0 / (1.0 + np.exp(-np.abs(y))), np.exp(-np.abs(y)) / (1.0 + np.exp(-np.abs(y))))
+    return unit(q), unit(k), np.exp(-softplus), beta
+
+
+def forward_raw(q, k, v, gate_logit, beta_logit, s0=None, scale=None, n_threads=0):
+    """``forward`` on preprocessed inputs: un-normalised q, k [B,T,H,dk], gate logits
+    [B,T,H,dk] and beta logits [B,T,H] (see ``preprocess``)."""
+    qn, kn, alpha, beta = preprocess(q, k, gate_logit, beta_logit)
+    return forward(qn, kn, v, alpha, beta, s0=s0, scale=scale, n_threads=n_threads)
