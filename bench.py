@@ -12,6 +12,12 @@ all 64 heads) summed over ranks; the decode step is reported beside it in GB/s
 of algorithmic HBM traffic.  Inputs (1.07 GB prefill, 2.2 GB decode state) are
 far larger than the 126 MB L2, so no flush is needed between steps.
 
+After the timed steps, a single-GPU run also times each further entry point once
+on a workload of the same scale (``next_rows`` in the JSON line): the scalar-gate,
+raw-input, packed-sequence and GDN-2 prefills, the multi-token decode with
+per-token states, and the state copy, each with its algorithmic bytes and the
+fraction of the measured copy bandwidth they reach.
+
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 For N > 1 launch with torch.distributed.run; every rank runs the same workload
 on its own GPU (independent (sequence, head) shards, no collective on the data
@@ -59,6 +65,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rows", action="store_true", help="skip the per-entry-point measurements")
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="run one kernel per step (for profiling); the JSON line is then partial")
     ap.add_argument("--prefill-seqs", type=int, default=None,
@@ -96,6 +103,93 @@ def decode_bytes(w) -> int:
     gsz = torch.tensor([], dtype=w.gate_dtype).element_size()
     heads = w.B * w.H
     return heads * (2 * w.dk * w.dv * 4 + 2 * w.dk * qsz + w.dv * qsz + w.dk * gsz + gsz + w.dv * 4)
+
+
+def time_call(torch, fn, reps=5, warmup=2):
+    """Mean CUDA-event time of fn() in ms on the current stream, after warm-up calls."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def measure_rows(torch, kda, x, y, wp, hbm):
+    """Each further entry point once, at the scale of the prefill and decode workloads.
+    Returns {row: {workload, ms, throughput, algorithmic bytes, fraction of hbm}}."""
+    dev = x["q"].device
+    B, T, H, dk, dv = wp.B, wp.T, wp.H, wp.dk, wp.dv
+    tok_heads = B * T * H
+    state = B * H * dk * dv * 4
+    rows = {}
+
+    def row(name, workload, ms, nbytes, tokens=None):
+        r = {"workload": workload, "ms": ms, "algorithmic_bytes": nbytes,
+             "gbs": nbytes / (ms * 1e-3) / 1e9}
+        r["frac_of_measured_hbm"] = r["gbs"] / hbm
+        if tokens is not None:
+            r["mtokens_s"] = tokens / (ms * 1e-3) / 1e6
+        rows[name] = r
+
+    o = torch.empty((B, T, H, dv), device=dev)
+    S = torch.empty((B, H, dk, dv), device=dev)
+    # scalar gate: one retention factor per (token, head)
+    ah = x["alpha"][..., 0].contiguous()
+    ms = time_call(torch, lambda: kda.forward_scalar_gate(x["q"], x["k"], x["v"], ah, x["beta"], scale=x["scale"],
+                                                          out=o, final_state=S))
+    row("scalar_gate_prefill", f"B={B} T={T} H={H} d={dk} bf16, alpha [B,T,H]", ms,
+        tok_heads * (3 * 256 + 2 + 2 + 512) + state, B * T)
+    # raw inputs: logits in place of alpha and beta (same bytes as the plain prefill)
+    ms = time_call(torch, lambda: kda.forward_raw(x["q"], x["k"], x["v"], x["alpha"], x["beta"], scale=x["scale"],
+                                                  out=o, final_state=S))
+    row("raw_inputs_prefill", f"B={B} T={T} H={H} d={dk} bf16 raw q/k, gate and beta logits", ms,
+        tok_heads * 1538 + state, B * T)
+    # packed sequences: the same tokens as 8 sequences of mixed lengths
+    lengths = [4096, 1000, 3000, 200, 5000, 1084, 1500, 500]
+    assert sum(lengths) == B * T
+    cu = torch.tensor([0] + list(__import__("itertools").accumulate(lengths)), dtype=torch.int32, device=dev)
+    flat = {n: x[n].reshape(B * T, *x[n].shape[2:]) for n in ("q", "k", "v", "alpha", "beta")}
+    ov = o.view(B * T, H, dv)
+    Sv = torch.empty((len(lengths), H, dk, dv), device=dev)
+    ms = time_call(torch, lambda: kda.forward_varlen(flat["q"], flat["k"], flat["v"], flat["alpha"], flat["beta"], cu,
+                                                     scale=x["scale"], out=ov, final_state=Sv))
+    row("varlen_prefill", f"{B * T} tokens as sequences {lengths}, H={H} d={dk} bf16", ms,
+        tok_heads * 1538 + len(lengths) * H * dk * dv * 4, B * T)
+    # GDN-2 (CUDA-core chunk kernel): erase [.., d_k] and write [.., d_v] gates in place of beta
+    g = torch.Generator(device=dev).manual_seed(7)
+    er = torch.sigmoid(torch.randn(x["k"].shape, generator=g, device=dev)).to(torch.bfloat16)
+    wr = torch.sigmoid(torch.randn(x["v"].shape, generator=g, device=dev)).to(torch.bfloat16)
+    ms = time_call(torch, lambda: kda.forward_gdn2(x["q"], x["k"], x["v"], x["alpha"], er, wr, scale=x["scale"],
+                                                   out=o, final_state=S), reps=2, warmup=1)
+    row("gdn2_prefill", f"B={B} T={T} H={H} d={dk} bf16, erase/write gates (CUDA-core kernel)", ms,
+        tok_heads * (6 * 256 + 512) + state, B * T)
+    del er, wr
+    if y is not None:
+        N, Hd, d = y["state"].shape[0], y["state"].shape[1], y["state"].shape[2]
+        Td = 4
+        gd = torch.Generator(device=dev).manual_seed(8)
+        draft = {n: torch.cat([y[n].unsqueeze(1)] * Td, 1).contiguous() for n in ("q", "k", "v", "alpha", "beta")}
+        ts = torch.empty((N, Td, Hd, d, d), device=dev)
+        od = torch.empty((N, Td, Hd, d), device=dev)
+        ms = time_call(torch, lambda: kda.decode_tokens(draft["q"], draft["k"], draft["v"], draft["alpha"],
+                                                        draft["beta"], y["state"], commit=False, token_states=ts,
+                                                        scale=y["scale"], out=od))
+        heads = N * Hd
+        row("decode_tokens_verify", f"N={N} H={Hd} d={d}, {Td} draft tokens, per-token states, no commit", ms,
+            heads * (d * d * 4 * (1 + Td) + Td * (3 * 256 + 256 + 2 + 512)))
+        del ts, od, draft
+        pool = torch.empty_like(y["state"])
+        perm = torch.randperm(N, generator=gd, device=dev).to(torch.int32)
+        ms = time_call(torch, lambda: kda.state_copy(y["state"], pool, src_index=perm,
+                                                     dst_index=torch.arange(N, dtype=torch.int32, device=dev)))
+        row("state_copy", f"{N} states of H={Hd} d={d} gathered by a permutation", ms, 2 * N * Hd * d * d * 4)
+        del pool
+    return rows
 
 
 class ClockSampler(threading.Thread):
@@ -374,6 +468,10 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_prefill(x, wp)
+    rows = None
+    if world == 1 and not args.no_rows and args.only is None and args.prefill_seqs is None \
+            and args.prefill_len is None:
+        rows = measure_rows(torch, kda, x, y, wp, float(peaks["hbm_gbs"]))
 
     clocks = sampler.summary()
     if rank != 0:
@@ -401,6 +499,7 @@ def main():
             "value": dec_gbs, "unit": "GB/s", "us_per_step": dec_ms * 1e3, "algorithmic_bytes": db,
             "frac_of_measured_hbm": dec_gbs / hbm, "frac_of_8TBs": dec_gbs / 8000.0},
         "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": (1 if args.only else 2) * K, "clocks": clocks,
+        "next_rows": rows,
     }
     print(json.dumps(line), flush=True)
 

@@ -181,12 +181,14 @@ __device__ __forceinline__ bool prep_bar_err(volatile int *err_flag)
     return ptx::named_bar_sync_or(kPrepBar, NPT, *err_flag != 0);
 }
 
+template <bool kRaw>
 __device__ __forceinline__ float load_beta(const ChunkArgs &p, const SeqSpan &sp, int h, int n, int r)
 {
     const int t = n * C + r;
     if (t >= sp.len) return 0.f;
     const float y = __bfloat162float(((const __nv_bfloat16 *)p.beta)[(sp.tok0 + t) * p.H + h]);
-    return p.raw_inputs ? sigmoid_of(y) : y;   // raw inputs: beta logits
+    if constexpr (kRaw) return sigmoid_of(y);   // a beta logit
+    else return y;
 }
 
 // TMA descriptors of one launch: q, k, alpha as [B][T][H][128] boxes of 32 token
@@ -492,6 +494,7 @@ __device__ __forceinline__ void load_v(const TcMaps &maps, uint8_t *sm, const Ba
 // Lq_lo times R: warps 0 and 2 hand their partial sums to warps 1 and 3 through
 // shared memory; warp 1 forms A_kk and solves its diagonal blocks, warp 3 writes
 // A_qk, and all four finish the off-diagonal block of T and write T'.
+template <bool kRaw>
 __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, uint32_t tmem, const Bars &bars,
                           const TmaPos &tp, const SeqSpan &sp, int h, int nchunks, volatile int *err_flag)
 {
@@ -514,10 +517,10 @@ __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, u
         if (nchunks > 1) load_v(maps, sm, bars, tp, 1);
     }
     v_loaded = nchunks > 1 ? 2 : 1;
-    float beta = (pw < 2) ? load_beta(p, sp, h, 0, r) : 0.f;   // beta of row r
+    float beta = (pw < 2) ? load_beta<kRaw>(p, sp, h, 0, r) : 0.f;   // beta of row r
 
     for (int cn = 0; cn < nchunks; ++cn) {
-        const float beta_next = (pw < 2 && cn + 1 < nchunks) ? load_beta(p, sp, h, cn + 1, r) : 0.f;
+        const float beta_next = (pw < 2 && cn + 1 < nchunks) ? load_beta<kRaw>(p, sp, h, cn + 1, r) : 0.f;
 
         // ---- G(cn): A_kk / A_qk from TMEM; the solve; T'
         if (!ptx::mbar_wait(bars.a, (uint32_t)(cn & 1), kWaitLimitNs)) *err_flag = 1;
@@ -984,7 +987,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs pa, const
     if (warp == kIssuerWarp) {
         if (lane == 0) issuer(sm, tmem, bars, nchunks, err_flag);
     } else if (warp >= NCW) {
-        prep_role(p, maps, sm, tmem, bars, tp, sp, h, nchunks, err_flag);
+        prep_role<kRaw>(p, maps, sm, tmem, bars, tp, sp, h, nchunks, err_flag);
     } else {
         chain_role<kHeadGate, kRaw>(p, maps, sm, tmem, bars, tp, sp, h, bh, nchunks, err_flag);
     }
