@@ -40,11 +40,11 @@ if ROOT not in sys.path:
 METRIC = "KDA prefill Mtokens/s (H=64,d=128); decode-step HBM GB/s vs ~8 TB/s peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of the prefill
-# kernel (1.08 GB read + 0.509 GB written), from the capture summarised under
+# kernel (1.08 GB read + 0.5087 GB written), from the capture summarised under
 # profiles/, with the hash of the kernel sources it was taken for: once the
 # sources change, the line reports traffic as null until it is captured again.
-PREFILL_TRAFFIC_BYTES = 1_589_000_000
-PREFILL_TRAFFIC_SOURCES = "8b257c2abe040c77"
+PREFILL_TRAFFIC_BYTES = 1_588_650_000
+PREFILL_TRAFFIC_SOURCES = "4459036eb8fc0c1a"
 
 
 def kernel_sources_hash() -> str:
@@ -150,7 +150,7 @@ def measure_rows(torch, kda, x, y, wp, hbm):
     row("raw_inputs_prefill", f"B={B} T={T} H={H} d={dk} bf16 raw q/k, gate and beta logits", ms,
         tok_heads * 1538 + state, B * T)
     # packed sequences: the same tokens as 8 sequences of mixed lengths
-    lengths = [4096, 1000, 3000, 200, 5000, 1084, 1500, 500]
+    lengths = [4096, 1000, 3000, 200, 5000, 1084, 1500, 504]
     assert sum(lengths) == B * T
     cu = torch.tensor([0] + list(__import__("itertools").accumulate(lengths)), dtype=torch.int32, device=dev)
     flat = {n: x[n].reshape(B * T, *x[n].shape[2:]) for n in ("q", "k", "v", "alpha", "beta")}

@@ -876,12 +876,13 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
         }
         // outputs of chunk c into the staging rows q and alpha have left (rows 16h..16h+15
         // into the q rows for h = 0, the alpha rows for h = 1), as one TMA box each.
-        // The previous chunk's output store must have read those rows: a staging fill
-        // orders that (thread 0 issues it after the read); without one, sync here.
-        if (c > 0 && c + 2 >= nchunks) {
-            if (tid == 0) ptx::bulk_wait_read();
-            chain_bar();
-        }
+        // Those rows still hold chunk c+2's q, k and alpha until every chain warp has
+        // finished its stage A of chunk c+2, so the tile is written only after a chain
+        // barrier.  The previous chunk's output store must also have read the rows: a
+        // staging fill orders that (thread 0 issues it after the read); without one,
+        // thread 0 waits for the read here, before the barrier.
+        if (c > 0 && c + 2 >= nchunks && tid == 0) ptx::bulk_wait_read();
+        chain_bar();
         const bool full = (c + 1) * C <= sp.len;
         if (full) {
             const int esz = p.out_bf16 ? 2 : 4;
