@@ -26,6 +26,7 @@ path) and the time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import itertools
 import json
 import os
 import statistics
@@ -152,7 +153,7 @@ def measure_rows(torch, kda, x, y, wp, hbm):
     # packed sequences: the same tokens as 8 sequences of mixed lengths
     lengths = [4096, 1000, 3000, 200, 5000, 1084, 1500, 504]
     assert sum(lengths) == B * T
-    cu = torch.tensor([0] + list(__import__("itertools").accumulate(lengths)), dtype=torch.int32, device=dev)
+    cu = torch.tensor([0] + list(itertools.accumulate(lengths)), dtype=torch.int32, device=dev)
     flat = {n: x[n].reshape(B * T, *x[n].shape[2:]) for n in ("q", "k", "v", "alpha", "beta")}
     ov = o.view(B * T, H, dv)
     Sv = torch.empty((len(lengths), H, dk, dv), device=dev)

@@ -122,7 +122,7 @@ constexpr int OFF_BETA = OFF_TS + C * P * 4;           // beta of the chunk bein
 constexpr int OFF_NRM = OFF_BETA + C * 4;             // 1/||q_r||, 1/||k_r|| (raw inputs)
 constexpr int NBARS = 7;
 constexpr int OFF_BAR = (OFF_NRM + 2 * C * 4 + 7) / 8 * 8;
-constexpr int OFF_SIG = OFF_BAR + NBARS * 8;           // 6 readiness counters
+constexpr int OFF_SIG = OFF_BAR + NBARS * 8;           // 6 readiness counters (8 slots)
 constexpr int OFF_MISC = OFF_SIG + 32;                 // tmem base, error flag
 constexpr int SMEM_BYTES = OFF_MISC + 16;
 static_assert(SMEM_BYTES <= 232448, "shared memory plan exceeds the per-block limit");
@@ -187,7 +187,7 @@ __device__ __forceinline__ float load_beta(const ChunkArgs &p, const SeqSpan &sp
     const int t = n * C + r;
     if (t >= sp.len) return 0.f;
     const float y = __bfloat162float(((const __nv_bfloat16 *)p.beta)[(sp.tok0 + t) * p.H + h]);
-    if constexpr (kRaw) return sigmoid_of(y);   // a beta logit
+    if constexpr (kRaw) return ptx::rcp(1.f + __expf(-y));   // a beta logit: sigmoid(y)
     else return y;
 }
 
@@ -196,7 +196,11 @@ __device__ __forceinline__ float load_beta(const ChunkArgs &p, const SeqSpan &sp
 // MN-major core-matrix layout of the U^T product; o as boxes of 16 token rows.
 struct TcMaps {
     CUtensorMap q, k, a, v, o;
+    // one gate per head: 1 when map a stages each chunk's gates as a box of 8 heads x 32
+    // tokens (H a multiple of 8, alpha 16-byte aligned); 0 when they are read from memory
+    int head_gate_tma;
 };
+constexpr int HG_ROW = 16;   // bytes per token row of a staged per-head gate box
 
 // Every warp of a role adds 1 to a readiness counter once its writes are visible
 // (the counter of chunk n's step reaches (n + 1) x the role's warps).
@@ -376,7 +380,8 @@ __device__ __forceinline__ void solve_diag_blocks(const float *At, float *Tm, in
 // product (M3) of the chunk two back have finished with, so it can run while that
 // chunk's state update (M4) still reads R.
 template <bool kHeadGate, bool kRaw>
-__device__ void stage_a(const ChunkArgs &p, uint8_t *sm, const SeqSpan &sp, int h, int n, int warp, int lane, uint32_t (&rw)[16])
+__device__ void stage_a(const ChunkArgs &p, uint8_t *sm, const SeqSpan &sp, int h, int n, int warp, int lane,
+                        uint32_t (&rw)[16], bool head_staged)
 {
     const int hf = warp >> 2, d = 32 * (warp & 3) + lane;
     const int Lc = min(C, sp.len - n * C);
@@ -388,7 +393,8 @@ __device__ void stage_a(const ChunkArgs &p, uint8_t *sm, const SeqSpan &sp, int 
     // gate straight from global memory (the same 32 values for every thread)
     const __nv_bfloat16 *ah = (const __nv_bfloat16 *)p.alpha + (sp.tok0 + (size_t)n * C) * p.H + h;
     auto alpha_at = [&](int r) {
-        if constexpr (kHeadGate) return __bfloat162float(ah[(size_t)r * p.H]);
+        if constexpr (kHeadGate)
+            return head_staged ? ld_bf16(stg + STG_A + HG_ROW * r + 2 * (h & 7)) : __bfloat162float(ah[(size_t)r * p.H]);
         // a gate logit x: alpha = exp(-softplus(x)) = 1 / (1 + e^x)
         else if constexpr (kRaw) return ptx::rcp(1.f + __expf(ld_bf16(stg + STG_A + stg_row(r) + 2 * d)));
         else return ld_bf16(stg + STG_A + stg_row(r) + 2 * d);
@@ -467,18 +473,22 @@ __device__ void stage_b(uint8_t *sm, int n, int warp, int lane, const uint32_t (
 // t0 (b = sequence, t0 = 0 for the dense layout; b = 0, t0 = its offset when packed).
 struct TmaPos {
     int b, h, t0;
-    int gate_rows;   // alpha has a row per token (per-key-channel gate) to stage
+    int gate_rows;   // 1: alpha rows per token (per-key-channel gate); 2: a per-head gate box; 0: none
 };
 
 // TMA loads of chunk n's q, k, alpha rows into the staging rows (one thread).  Rows
 // past the sequence's end are masked where they are used.
+template <bool kHeadGate>
 __device__ __forceinline__ void load_qka(const TcMaps &maps, uint8_t *sm, const Bars &bars, const TmaPos &tp, int n)
 {
-    ptx::mbar_arrive_expect_tx(bars.stg, (tp.gate_rows ? 3 : 2) * STG_T);
     const uint32_t dst = ptx::smem_u32(sm + OFF_STG);
+    if constexpr (!kHeadGate) ptx::mbar_arrive_expect_tx(bars.stg, 3 * STG_T);
+    else ptx::mbar_arrive_expect_tx(bars.stg, 2 * STG_T + (tp.gate_rows == 2 ? C * HG_ROW : 0));
     ptx::tma_load_4d(dst + STG_Q, &maps.q, bars.stg, 0, tp.h, tp.t0 + n * C, tp.b);
     ptx::tma_load_4d(dst + STG_K, &maps.k, bars.stg, 0, tp.h, tp.t0 + n * C, tp.b);
-    if (tp.gate_rows) ptx::tma_load_4d(dst + STG_A, &maps.a, bars.stg, 0, tp.h, tp.t0 + n * C, tp.b);
+    if constexpr (!kHeadGate) ptx::tma_load_4d(dst + STG_A, &maps.a, bars.stg, 0, tp.h, tp.t0 + n * C, tp.b);
+    // heads h & ~7 .. (h & ~7) + 7 of 32 tokens: the x coordinate is a multiple of 8 elements
+    else if (tp.gate_rows == 2) ptx::tma_load_3d(dst + STG_A, &maps.a, bars.stg, tp.h & ~7, tp.t0 + n * C, tp.b);
 }
 
 // TMA load of chunk n's v rows into V buffer n&1 (one thread).
@@ -681,49 +691,41 @@ __device__ __forceinline__ void write_state16(uint32_t tmem, uint32_t lane_base,
 
 // Chain warps, operands of chunk n (the staging rows must hold chunk n): part A,
 // then (later) part B, the signal to the issuer and the loads of chunk n+1.
-// Raw inputs: 1/||q_r|| and 1/||k_r|| of the staged rows, four rows per chain warp
-// (each lane sums the squares of four channels; a butterfly finishes the rows).
+// Raw inputs: 1/||q_r|| and 1/||k_r|| of the staged rows, four rows of each per chain
+// warp, one row at a time (each lane sums the squares of four channels; a butterfly
+// finishes the row), so that few registers are live next to the chain's own.
 __device__ __forceinline__ void row_norms(uint8_t *sm, int warp, int lane)
 {
     const uint8_t *stg = sm + OFF_STG;
-    float ss[8];
+    float mine = 0.f;
+#pragma unroll 1
+    for (int i = 0; i < 8; ++i) {
+        const int r = 4 * warp + (i & 3);
+        const uint2 w = *reinterpret_cast<const uint2 *>(stg + (i < 4 ? STG_Q : STG_K) + stg_row(r) + 8 * lane);
+        const float a0 = __uint_as_float(w.x << 16), a1 = __uint_as_float(w.x & 0xFFFF0000u);
+        const float a2 = __uint_as_float(w.y << 16), a3 = __uint_as_float(w.y & 0xFFFF0000u);
+        float ss = fmaf(a0, a0, fmaf(a1, a1, fmaf(a2, a2, a3 * a3)));
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int r = 4 * warp + i;
-        const uint2 qw = *reinterpret_cast<const uint2 *>(stg + STG_Q + stg_row(r) + 8 * lane);
-        const uint2 kw = *reinterpret_cast<const uint2 *>(stg + STG_K + stg_row(r) + 8 * lane);
-        float a0 = __uint_as_float(qw.x << 16), a1 = __uint_as_float(qw.x & 0xFFFF0000u);
-        float a2 = __uint_as_float(qw.y << 16), a3 = __uint_as_float(qw.y & 0xFFFF0000u);
-        ss[i] = fmaf(a0, a0, fmaf(a1, a1, fmaf(a2, a2, a3 * a3)));
-        a0 = __uint_as_float(kw.x << 16); a1 = __uint_as_float(kw.x & 0xFFFF0000u);
-        a2 = __uint_as_float(kw.y << 16); a3 = __uint_as_float(kw.y & 0xFFFF0000u);
-        ss[4 + i] = fmaf(a0, a0, fmaf(a1, a1, fmaf(a2, a2, a3 * a3)));
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        if (lane == i) mine = ss;
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) ss[i] += __shfl_xor_sync(0xffffffffu, ss[i], off);
-    if (lane < 8) {
-        float x = ss[0];
-#pragma unroll
-        for (int i = 1; i < 8; ++i) x = (lane == i) ? ss[i] : x;
-        const int r = 4 * warp + (lane & 3);
-        reinterpret_cast<float *>(sm + OFF_NRM)[(lane < 4 ? 0 : C) + r] = inv_norm(x);
-    }
+    if (lane < 8)
+        reinterpret_cast<float *>(sm + OFF_NRM)[(lane < 4 ? 0 : C) + 4 * warp + (lane & 3)] = inv_norm(mine);
 }
 
 template <bool kHeadGate, bool kRaw>
 __device__ __forceinline__ void chain_stage_a(const ChunkArgs &p, uint8_t *sm, const Bars &bars, const SeqSpan &sp, int h, int n, int warp,
-                                              int lane, uint32_t (&ie)[16], volatile int *err_flag)
+                                              int lane, uint32_t (&ie)[16], volatile int *err_flag, bool head_staged)
 {
     if (!ptx::mbar_wait(bars.stg, (uint32_t)(n & 1), kWaitLimitNs)) *err_flag = 1;   // chunk n's rows
     if constexpr (kRaw) {
         row_norms(sm, warp, lane);
         chain_bar();   // every row's norms are in place
     }
-    stage_a<kHeadGate, kRaw>(p, sm, sp, h, n, warp, lane, ie);
+    stage_a<kHeadGate, kRaw>(p, sm, sp, h, n, warp, lane, ie, head_staged);
 }
 
+template <bool kHeadGate>
 __device__ __forceinline__ void chain_stage_b(const TcMaps &maps, uint8_t *sm, const Bars &bars, const TmaPos &tp,
                                               int n, int nchunks, int tid, int warp, int lane,
                                               const uint32_t (&ie)[16])
@@ -732,7 +734,7 @@ __device__ __forceinline__ void chain_stage_b(const TcMaps &maps, uint8_t *sm, c
     ptx::fence_proxy_async_smem();
     warp_signal(bars.rc, lane);
     chain_bar();   // staging consumed, constants visible to every chain warp
-    if (tid == 0 && n + 1 < nchunks) load_qka(maps, sm, bars, tp, n + 1);
+    if (tid == 0 && n + 1 < nchunks) load_qka<kHeadGate>(maps, sm, bars, tp, n + 1);
 }
 
 __device__ __forceinline__ void warp_signal_after_stage(const Bars &bars, int lane)
@@ -754,11 +756,11 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
     const size_t tile = (size_t)bh * D * D;
 
     uint32_t ie[16];   // R of the chunk being staged (split words), carried from part A to part B
-    if (tid == 0) load_qka(maps, sm, bars, tp, 0);
+    if (tid == 0) load_qka<kHeadGate>(maps, sm, bars, tp, 0);
     int staged = 0;   // chunks whose rows have been waited for
-    chain_stage_a<kHeadGate, kRaw>(p, sm, bars, sp, h, 0, warp, lane, ie, err_flag);
+    chain_stage_a<kHeadGate, kRaw>(p, sm, bars, sp, h, 0, warp, lane, ie, err_flag, tp.gate_rows == 2);
     staged = 1;
-    chain_stage_b(maps, sm, bars, tp, 0, nchunks, tid, warp, lane, ie);
+    chain_stage_b<kHeadGate>(maps, sm, bars, tp, 0, nchunks, tid, warp, lane, ie);
 
     // S'_0 = Diag(exp(a_0)) S_0; cleared O accumulator
     {
@@ -778,9 +780,9 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
     ptx::tc_fence_before();
     warp_signal(bars.rs, lane);
     if (nchunks > 1) {
-        chain_stage_a<kHeadGate, kRaw>(p, sm, bars, sp, h, 1, warp, lane, ie, err_flag);
+        chain_stage_a<kHeadGate, kRaw>(p, sm, bars, sp, h, 1, warp, lane, ie, err_flag, tp.gate_rows == 2);
         staged = 2;
-        chain_stage_b(maps, sm, bars, tp, 1, nchunks, tid, warp, lane, ie);
+        chain_stage_b<kHeadGate>(maps, sm, bars, tp, 1, nchunks, tid, warp, lane, ie);
     }
 
     for (int c = 0; c < nchunks; ++c) {
@@ -807,7 +809,7 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
         warp_signal(bars.re, lane);
         // Lk, Lq of chunk c+2 while the state update of chunk c runs
         if (c + 2 < nchunks) {
-            chain_stage_a<kHeadGate, kRaw>(p, sm, bars, sp, h, c + 2, warp, lane, ie, err_flag);
+            chain_stage_a<kHeadGate, kRaw>(p, sm, bars, sp, h, c + 2, warp, lane, ie, err_flag, tp.gate_rows == 2);
             staged = c + 3;
         }
 
@@ -914,7 +916,7 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
             ptx::bulk_commit();
             if (c + 3 < nchunks) {
                 ptx::bulk_wait_read();   // the tile has been read: the staging rows can be refilled
-                load_qka(maps, sm, bars, tp, c + 3);
+                load_qka<kHeadGate>(maps, sm, bars, tp, c + 3);
             }
         }
         if (stop) break;
@@ -942,7 +944,8 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs pa, const
         return;
     }
     // TMA coordinates: dense tensors by (batch, token); packed ones as one batch by token row
-    const TmaPos tp{pa.cu_seqlens ? 0 : bh / pa.H, h, pa.cu_seqlens ? (int)sp.tok0 : 0, pa.gate_per_head ? 0 : 1};
+    const TmaPos tp{pa.cu_seqlens ? 0 : bh / pa.H, h, pa.cu_seqlens ? (int)sp.tok0 : 0,
+                    pa.gate_per_head ? (maps.head_gate_tma ? 2 : 0) : 1};
     const int nchunks = (sp.len + C - 1) / C;
     if (nchunks == 0) {
         // an empty sequence: the final state is the initial one (or zeros)
@@ -1039,6 +1042,18 @@ bool encode_rows(CUtensorMap *m, const void *base, int B, int T, int H)
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// one gate per (token, head), [B][T][H] bf16: dims (h, t, b), box (8, 32, 1) -- 16-byte rows
+bool encode_head_gate(CUtensorMap *m, const void *base, int B, int T, int H)
+{
+    const cuuint64_t dims[3] = {(cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[2] = {(cuuint64_t)H * 2, (cuuint64_t)T * H * 2};
+    const cuuint32_t box[3] = {8, (cuuint32_t)tc::C, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // v [B][T][H][128] bf16 as (j%8, t, j/8, h, b), box (8, 32, 16, 1, 1): the box lands
 // as j/8-major, token-minor 16-byte rows, the MN-major core matrices of V^T.
 bool encode_v(CUtensorMap *m, const void *base, int B, int T, int H)
@@ -1076,7 +1091,14 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, int dk, int dv, cudaStream_t str
     if (encode_fn() == nullptr) return cudaErrorNotSupported;
     tc::TcMaps maps;
     const int mb = a.cu_seqlens ? 1 : a.B;   // packed sequences: one [1, T, H, d] tensor
-    if (a.gate_per_head) memset(&maps.a, 0, sizeof(maps.a));   // alpha is read per token instead
+    maps.head_gate_tma = 0;
+    if (a.gate_per_head) {
+        // [B][T][H] gates as boxes of 8 heads x 32 tokens when the layout allows a TMA box
+        // (16-byte rows of heads and a 16-byte-aligned base); otherwise read per token
+        memset(&maps.a, 0, sizeof(maps.a));
+        if (a.H % 8 == 0 && ((uintptr_t)a.alpha & 15u) == 0 && encode_head_gate(&maps.a, a.alpha, mb, a.T, a.H))
+            maps.head_gate_tma = 1;
+    }
     if (!encode_rows(&maps.q, a.q, mb, a.T, a.H) || !encode_rows(&maps.k, a.k, mb, a.T, a.H) ||
         (!a.gate_per_head && !encode_rows(&maps.a, a.alpha, mb, a.T, a.H)) || !encode_v(&maps.v, a.v, mb, a.T, a.H) ||
         !encode_out(&maps.o, a.o, mb, a.T, a.H, a.out_bf16))

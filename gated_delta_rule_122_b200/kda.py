@@ -253,26 +253,22 @@ def forward_sequential(q, k, v, alpha, beta, initial_state=None, scale=None,
                     output_final_state, out_dtype, out, final_state)
 
 
-def decode_step(q, k, v, alpha, beta, state, scale=None, out_dtype=torch.float32, out=None,
-                _gate_per_head=False, _fn="kda_decode_step"):
-    """One token per sequence; ``state`` [N,H,dk,dv] float32 is updated in place.
-
-    q, k, alpha: [N,H,dk]; v: [N,H,dv]; beta: [N,H].  Returns o [N,H,dv].
-    """
+def _decode(fn, q, k, v, alpha, beta, state, scale, out_dtype, out, gate_per_head=False):
+    """Shared marshalling of the one-token decode entry points (C function ``fn``)."""
     device = state.device
     if device.type != "cuda":
-        raise ValueError("decode_step needs the state on a CUDA device")
+        raise ValueError("the decode step needs the state on a CUDA device")
     N, H, dk, dv = state.shape
     for name, t in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta", beta),
                     ("state", state)):
         _check(name, t, device)
     if state.dtype != torch.float32:
         raise TypeError("state must be float32")
-    a_shape = (N, H) if _gate_per_head else (N, H, dk)
+    a_shape = (N, H) if gate_per_head else (N, H, dk)
     if tuple(q.shape) != (N, H, dk) or tuple(k.shape) != (N, H, dk) or \
             tuple(alpha.shape) != a_shape or tuple(v.shape) != (N, H, dv) or \
             tuple(beta.shape) != (N, H):
-        raise ValueError("shapes: q,k [N,H,dk], alpha " + ("[N,H]" if _gate_per_head else "[N,H,dk]")
+        raise ValueError("shapes: q,k [N,H,dk], alpha " + ("[N,H]" if gate_per_head else "[N,H,dk]")
                          + ", v [N,H,dv], beta [N,H], state [N,H,dk,dv]")
     if k.dtype != q.dtype or v.dtype != q.dtype or alpha.dtype != beta.dtype:
         raise TypeError("q/k/v and alpha/beta must each share a dtype")
@@ -282,7 +278,6 @@ def decode_step(q, k, v, alpha, beta, state, scale=None, out_dtype=torch.float32
         out = torch.empty((N, H, dv), device=device, dtype=out_dtype)
     _check("out", out, device)
     with torch.cuda.device(device):
-        fn = "kda_decode_step_scalar_gate" if _gate_per_head else _fn
         code = getattr(library(), fn)(
             _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state), _ptr(out),
             N, H, dk, dv, float(scale), _DT[q.dtype], _dt(alpha, "alpha"), _dt(out, "out"),
@@ -292,16 +287,26 @@ def decode_step(q, k, v, alpha, beta, state, scale=None, out_dtype=torch.float32
     return out
 
 
+def decode_step(q, k, v, alpha, beta, state, scale=None, out_dtype=torch.float32, out=None):
+    """One token per sequence (C entry point ``kda_decode_step``); ``state`` [N,H,dk,dv]
+    float32 is updated in place.
+
+    q, k, alpha: [N,H,dk]; v: [N,H,dv]; beta: [N,H].  Returns o [N,H,dv].
+    """
+    return _decode("kda_decode_step", q, k, v, alpha, beta, state, scale, out_dtype, out)
+
+
 def decode_step_scalar_gate(q, k, v, alpha, beta, state, scale=None, out_dtype=torch.float32, out=None):
     """Gated DeltaNet decode step: alpha [N,H], one retention factor per (sequence, head)
     (C entry point ``kda_decode_step_scalar_gate``); otherwise the contract of ``decode_step``."""
-    return decode_step(q, k, v, alpha, beta, state, scale, out_dtype, out, _gate_per_head=True)
+    return _decode("kda_decode_step_scalar_gate", q, k, v, alpha, beta, state, scale, out_dtype, out,
+                   gate_per_head=True)
 
 
 def decode_step_raw(q, k, v, gate_logit, beta_logit, state, scale=None, out_dtype=torch.float32, out=None):
     """Decode step on raw inputs (C entry point ``kda_decode_step_raw``): the preprocessing
     of ``forward_raw``; otherwise the contract of ``decode_step``."""
-    return decode_step(q, k, v, gate_logit, beta_logit, state, scale, out_dtype, out, _fn="kda_decode_step_raw")
+    return _decode("kda_decode_step_raw", q, k, v, gate_logit, beta_logit, state, scale, out_dtype, out)
 
 
 def forward_varlen(q, k, v, alpha, beta, cu_seqlens, initial_state=None, scale=None,

@@ -3,8 +3,9 @@
 The scalar gate is KDA with alpha_t repeated over the key channels, so the
 per-head entry points must give exactly the per-channel ones on the broadcast
 tensor (same kernels, same arithmetic), and the oracle on the broadcast tensor.
-Covers the tensor-core prefill (d = 128, bf16), the CUDA-core prefill (fp32,
-d = 64) and the decode step.
+Covers the tensor-core prefill (d = 128, bf16; gates staged by TMA boxes when H is a
+multiple of 8, read per token otherwise), the CUDA-core prefill (fp32, d = 64) and the
+decode step.
 """
 import pytest
 import torch
@@ -24,6 +25,8 @@ def _head_gate(B, T, H, dtype, seed):
 
 
 @pytest.mark.parametrize("name,over,tol", [("prefill", dict(B=2, H=3, T=133), TOL_BF16),
+                                           ("prefill", dict(B=2, H=8, T=133), TOL_BF16),    # gates staged by TMA
+                                           ("long", dict(B=1, H=16, T=65), TOL_BF16),
                                            ("small", dict(B=1, H=2, T=97, qkv_dtype=torch.float32), TOL_F32)])
 def test_scalar_gate_prefill(name, over, tol):
     w = WORKLOADS[name].scaled(**over)
