@@ -145,9 +145,16 @@ def measure_rows(torch, kda, x, y, wp, hbm):
                                                           out=o, final_state=S))
     row("scalar_gate_prefill", f"B={B} T={T} H={H} d={dk} bf16, alpha [B,T,H]", ms,
         tok_heads * (3 * 256 + 2 + 2 + 512) + state, B * T)
-    # raw inputs: logits in place of alpha and beta (same bytes as the plain prefill)
-    ms = time_call(torch, lambda: kda.forward_raw(x["q"], x["k"], x["v"], x["alpha"], x["beta"], scale=x["scale"],
+    # raw inputs: the logits whose maps give the workload's alpha and beta (same bytes as the
+    # plain prefill and the same recurrence; q and k go through the norm pass as they are)
+    a = x["alpha"].float().clamp(1e-30, 1 - 1e-7)
+    gl = torch.log((1 - a) / a).to(x["alpha"].dtype)
+    del a
+    bt = x["beta"].float().clamp(1e-7, 1 - 1e-7)
+    bl = torch.log(bt / (1 - bt)).to(x["beta"].dtype)
+    ms = time_call(torch, lambda: kda.forward_raw(x["q"], x["k"], x["v"], gl, bl, scale=x["scale"],
                                                   out=o, final_state=S))
+    del gl, bl
     row("raw_inputs_prefill", f"B={B} T={T} H={H} d={dk} bf16 raw q/k, gate and beta logits", ms,
         tok_heads * 1538 + state, B * T)
     # packed sequences: the same tokens as 8 sequences of mixed lengths

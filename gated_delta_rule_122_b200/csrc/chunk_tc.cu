@@ -119,14 +119,20 @@ constexpr int OFF_XS = OFF_AQ + 2 * AQ_BYTES;          // A10 T0 of the solve fp
 constexpr int OFF_AKK = OFF_XS + C * P * 4;            // A_kk^T fp32 [32][36]
 constexpr int OFF_TS = OFF_AKK + C * (C + 4) * 4;      // T fp32 [32][33]
 constexpr int OFF_BETA = OFF_TS + C * P * 4;           // beta of the chunk being solved
-constexpr int OFF_NRM = OFF_BETA + C * 4;             // 1/||q_r||, 1/||k_r|| (raw inputs)
+// raw inputs: 1/||q_r||, 1/||k_r|| of a chunk, a ring of kNrmSlots chunks (stage A writes
+// chunk n, the prep warps and the chain's E and O readouts of chunk n read it)
+constexpr int kNrmSlots = 4;
+constexpr int NRM_BYTES = 2 * C * 4;
+constexpr int OFF_NRM = OFF_BETA + C * 4;
+constexpr int OFF_TPU = (OFF_NRM + kNrmSlots * NRM_BYTES + 127) / 128 * 128;   // raw: T Diag(beta), B of U
 constexpr int NBARS = 7;
-constexpr int OFF_BAR = (OFF_NRM + 2 * C * 4 + 7) / 8 * 8;
+constexpr int OFF_BAR = (OFF_TPU + C * C * 4 + 7) / 8 * 8;
 constexpr int OFF_SIG = OFF_BAR + NBARS * 8;           // 6 readiness counters (8 slots)
 constexpr int OFF_MISC = OFF_SIG + 32;                 // tmem base, error flag
 constexpr int SMEM_BYTES = OFF_MISC + 16;
 static_assert(SMEM_BYTES <= 232448, "shared memory plan exceeds the per-block limit");
-static_assert(OFF_AKK % 16 == 0 && OFF_LQR % 128 == 0, "vector and operand alignment");
+static_assert(OFF_AKK % 16 == 0 && OFF_LQR % 128 == 0 && OFF_TP % 128 == 0 && OFF_TPU % 128 == 0,
+              "vector and operand alignment");
 
 // TMEM columns
 constexpr uint32_t TM_A = 0;      // [A_kk; A_qk] per plane of Lk, Lq (M=128, N=64)
@@ -267,6 +273,7 @@ __device__ __forceinline__ void issue_m1(uint8_t *sm, uint32_t tmem, const Bars 
     ptx::mma_commit(bars.a);
 }
 
+template <bool kRaw>
 __device__ __forceinline__ void issue_m2(uint8_t *sm, uint32_t tmem, const Bars &bars, const MmaIds &id, int n2)
 {
     ptx::tc_fence_after();
@@ -279,9 +286,10 @@ __device__ __forceinline__ void issue_m2(uint8_t *sm, uint32_t tmem, const Bars 
             ptx::mma_bf16(tmem + TM_W,
                           ptx::smem_desc(base + (SL_LK + pl) * SLAB + 4 * SLAB * ks, 2 * SLAB, 128),
                           ptx::smem_desc(tp + 256 * ks, 128, 512), id.W, ks > 0 || pl > 0);
+    const uint32_t tu = kRaw ? ptx::smem_u32(sm + OFF_TPU) : tp;   // raw inputs: T Diag(beta) for U
     for (int ks = 0; ks < C / 16; ++ks)
         ptx::mma_bf16(tmem + TM_E, ptx::smem_desc(vv + 256 * ks, 128, (C / 8) * 128),
-                      ptx::smem_desc(tp + 256 * ks, 128, 512), id.U, ks > 0);
+                      ptx::smem_desc(tu + 256 * ks, 128, 512), id.U, ks > 0);
     ptx::mma_commit(bars.w);
 }
 
@@ -289,6 +297,7 @@ __device__ __forceinline__ void issue_m2(uint8_t *sm, uint32_t tmem, const Bars 
 // (ra), so it runs while the prep warps solve chunk n-1; M2(n) needs T' and A_qk (rg; the prep warps signal it after reading
 // W'(n-1)) and M4(n-1) issued, since U goes into TM_E; M3(n) needs S'(n) (rs,
 // whose first count is the initial state) and -W'(n) (rj); M4(n) needs E^T(n) (re).
+template <bool kRaw>
 __device__ void issuer(uint8_t *sm, uint32_t tmem, const Bars &bars, int nchunks, volatile int *err_flag)
 {
     MmaIds id;
@@ -322,7 +331,7 @@ __device__ void issuer(uint8_t *sm, uint32_t tmem, const Bars &bars, int nchunks
             else { (void)ptx::ld_acquire(bars.ra); (void)ptx::ld_acquire(bars.rc); }
             if (g == 3) issue_m3(sm, tmem, bars, id, n3++);
             else if (g == 4) issue_m4(sm, tmem, bars, id, n4++);
-            else if (g == 2) issue_m2(sm, tmem, bars, id, n2++);
+            else if (g == 2) issue_m2<kRaw>(sm, tmem, bars, id, n2++);
             else issue_m1(sm, tmem, bars, id, n1++);
             idle = 0;
         } else if ((++idle & 1023u) == 0) {
@@ -399,7 +408,6 @@ __device__ void stage_a(const ChunkArgs &p, uint8_t *sm, const SeqSpan &sp, int 
         else if constexpr (kRaw) return ptx::rcp(1.f + __expf(ld_bf16(stg + STG_A + stg_row(r) + 2 * d)));
         else return ld_bf16(stg + STG_A + stg_row(r) + 2 * d);
     };
-    const float *nrm = reinterpret_cast<const float *>(sm + OFF_NRM);
     float pr[16];
     float acc = 1.f;
     if (hf == 1) {
@@ -439,10 +447,6 @@ __device__ void stage_a(const ChunkArgs &p, uint8_t *sm, const SeqSpan &sp, int 
                 // rows past the sequence's end: zero (the staging may hold another sequence's rows)
                 kv[t] = (r < Lc) ? ld_bf16(stg + STG_K + stg_row(r) + 2 * d) : 0.f;
                 qv[t] = (r < Lc) ? ld_bf16(stg + STG_Q + stg_row(r) + 2 * d) : 0.f;
-                if constexpr (kRaw) {   // unit rows
-                    kv[t] = (r < Lc) ? kv[t] * nrm[C + r] : 0.f;
-                    qv[t] = (r < Lc) ? qv[t] * nrm[r] : 0.f;
-                }
             }
             const uint64_t e2 = ptx::pk2(e[0], e[1]);
             ptx::upk2(ptx::mul2(ptx::pk2(kv[0], kv[1]), e2), lk[i], lk[i + 1]);
@@ -535,6 +539,9 @@ __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, u
         // ---- G(cn): A_kk / A_qk from TMEM; the solve; T'
         if (!ptx::mbar_wait(bars.a, (uint32_t)(cn & 1), kWaitLimitNs)) *err_flag = 1;
         ptx::tc_fence_after();
+        // raw inputs: the chain's stage A of chunk cn wrote its norms before adding to the
+        // count rc, which M1(cn) waited for; acquiring rc makes them visible here
+        if constexpr (kRaw) (void)ptx::ld_acquire(bars.rc);
         float a32[32];   // this plane's row r times R, summed over R's planes
 #pragma unroll
         for (int hs = 0; hs < 2; ++hs) {
@@ -571,11 +578,16 @@ __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, u
             ptx::fence_proxy_async_smem();
         }
         if (pw < 2) {
-            // A_kk^T: row r of A_kk scaled by beta_r, strictly lower
+            // A_kk^T: row r of A_kk scaled by beta_r, strictly lower (raw inputs: and by
+            // nk_r nk_s)
+            float rs = beta;
+            const float *nk = reinterpret_cast<const float *>(sm + OFF_NRM + (cn % kNrmSlots) * NRM_BYTES) + C;
+            if constexpr (kRaw) rs *= nk[r];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int s = 16 * pl + i;
-                At[s * PT + r] = (s < r) ? beta * ar[i] : 0.f;
+                const float cs = kRaw ? nk[s] : 1.f;
+                At[s * PT + r] = (s < r) ? rs * cs * ar[i] : 0.f;
             }
             if (pl == 0) sbeta[r] = beta;
         } else {
@@ -619,13 +631,20 @@ __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, u
         }
         const bool stop = prep_bar_err(err_flag);
         {
-            // T' = T Diag(beta): row rt, columns 8sc..8sc+7, as hi/lo planes
+            // T' = T Diag(beta): row rt, columns 8sc..8sc+7, as hi/lo planes (raw inputs:
+            // T Diag(beta nk) for W', and T Diag(beta) for U in its own buffer)
             const int rt = 8 * pw + (lane & 7), sc = lane >> 3;
             float x[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int s = 8 * sc + i;
                 x[i] = (rt < 16 && s >= 16) ? 0.f : Tm[rt * P + s] * sbeta[s];
+            }
+            if constexpr (kRaw) {
+                st_split8(sm + OFF_TPU + ipl(rt, 8 * sc, 0), C * 16, x);
+                const float *nk = reinterpret_cast<const float *>(sm + OFF_NRM + (cn % kNrmSlots) * NRM_BYTES) + C;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) x[i] *= nk[8 * sc + i];
             }
             st_split8(sm + OFF_TP + ipl(rt, 8 * sc, 0), C * 16, x);
             ptx::fence_proxy_async_smem();
@@ -691,10 +710,14 @@ __device__ __forceinline__ void write_state16(uint32_t tmem, uint32_t lane_base,
 
 // Chain warps, operands of chunk n (the staging rows must hold chunk n): part A,
 // then (later) part B, the signal to the issuer and the loads of chunk n+1.
-// Raw inputs: 1/||q_r|| and 1/||k_r|| of the staged rows, four rows of each per chain
-// warp, one row at a time (each lane sums the squares of four channels; a butterfly
-// finishes the row), so that few registers are live next to the chain's own.
-__device__ __forceinline__ void row_norms(uint8_t *sm, int warp, int lane)
+// Raw inputs: 1/||q_r|| and 1/||k_r|| of chunk n's staged rows (0 past the sequence's
+// end) into the norm ring, four rows of each per chain warp, one row at a time (each
+// lane sums the squares of four channels; a butterfly finishes the row).  The factors
+// are applied after the products, where each one is a row or column scaling:
+//   A_kk -> Diag(nk) A_kk Diag(nk) and W' -> T Diag(beta nk) Lk (prep warps),
+//   the E operand of the state update and of O -> Diag(nk) E, O -> Diag(nq) O (chain),
+// so stage A itself is unchanged and needs no barrier.
+__device__ __forceinline__ void row_norms(uint8_t *sm, int n, int len, int warp, int lane)
 {
     const uint8_t *stg = sm + OFF_STG;
     float mine = 0.f;
@@ -709,8 +732,11 @@ __device__ __forceinline__ void row_norms(uint8_t *sm, int warp, int lane)
         for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
         if (lane == i) mine = ss;
     }
-    if (lane < 8)
-        reinterpret_cast<float *>(sm + OFF_NRM)[(lane < 4 ? 0 : C) + 4 * warp + (lane & 3)] = inv_norm(mine);
+    if (lane < 8) {
+        const int r = 4 * warp + (lane & 3);
+        reinterpret_cast<float *>(sm + OFF_NRM + (n % kNrmSlots) * NRM_BYTES)[(lane < 4 ? 0 : C) + r] =
+            (n * C + r < len) ? inv_norm(mine) : 0.f;
+    }
 }
 
 template <bool kHeadGate, bool kRaw>
@@ -718,10 +744,7 @@ __device__ __forceinline__ void chain_stage_a(const ChunkArgs &p, uint8_t *sm, c
                                               int lane, uint32_t (&ie)[16], volatile int *err_flag, bool head_staged)
 {
     if (!ptx::mbar_wait(bars.stg, (uint32_t)(n & 1), kWaitLimitNs)) *err_flag = 1;   // chunk n's rows
-    if constexpr (kRaw) {
-        row_norms(sm, warp, lane);
-        chain_bar();   // every row's norms are in place
-    }
+    if constexpr (kRaw) row_norms(sm, n, sp.len, warp, lane);
     stage_a<kHeadGate, kRaw>(p, sm, sp, h, n, warp, lane, ie, head_staged);
 }
 
@@ -801,6 +824,14 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
                 e0[i] = v0[i] + v0[8 + i];
                 e1[i] = v1[i] + v1[8 + i];
             }
+            if constexpr (kRaw) {   // the operand is Diag(nk) E (tokens 16 half + i, 16 half + 8 + i)
+                const float *nk = reinterpret_cast<const float *>(sm + OFF_NRM + (c % kNrmSlots) * NRM_BYTES) + C;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    e0[i] *= nk[16 * half + i];
+                    e1[i] *= nk[16 * half + 8 + i];
+                }
+            }
             st_split8(sm + OFF_ET + ipl(j, 16 * half, 0), C * 16, e0);
             st_split8(sm + OFF_ET + ipl(j, 16 * half + 8, 0), C * 16, e1);
         }
@@ -832,6 +863,11 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
             for (int i = 0; i < 8; ++i) {
                 ov[i] = v0[i] + v0[8 + i];
                 ov[8 + i] = v1[i] + v1[8 + i];
+            }
+            if constexpr (kRaw) {   // O -> Diag(nq) O
+                const float *nq = reinterpret_cast<const float *>(sm + OFF_NRM + (c % kNrmSlots) * NRM_BYTES);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) ov[i] *= nq[16 * half + i];
             }
         }
         if (c + 1 < nchunks) {
@@ -989,7 +1025,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs pa, const
     const uint32_t tmem = *tmem_slot;
 
     if (warp == kIssuerWarp) {
-        if (lane == 0) issuer(sm, tmem, bars, nchunks, err_flag);
+        if (lane == 0) issuer<kRaw>(sm, tmem, bars, nchunks, err_flag);
     } else if (warp >= NCW) {
         prep_role<kRaw>(p, maps, sm, tmem, bars, tp, sp, h, nchunks, err_flag);
     } else {
