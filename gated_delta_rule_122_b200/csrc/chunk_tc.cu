@@ -404,9 +404,15 @@ __device__ void stage_a(const ChunkArgs &p, uint8_t *sm, const SeqSpan &sp, int 
     auto alpha_at = [&](int r) {
         if constexpr (kHeadGate)
             return head_staged ? ld_bf16(stg + STG_A + HG_ROW * r + 2 * (h & 7)) : __bfloat162float(ah[(size_t)r * p.H]);
-        // a gate logit x: alpha = exp(-softplus(x)) = 1 / (1 + e^x)
-        else if constexpr (kRaw) return ptx::rcp(1.f + __expf(ld_bf16(stg + STG_A + stg_row(r) + 2 * d)));
         else return ld_bf16(stg + STG_A + stg_row(r) + 2 * d);
+    };
+    // Per-token factor of the running products: alpha (floored at e^-80), or with a gate
+    // logit x its inverse 1/alpha = 1 + e^x (capped at e^80): the products then hold the
+    // inverse decays, and the one reciprocal per row below gives the other side, so the
+    // logit costs one exponential and no reciprocal.
+    auto factor = [&](int r) {
+        if constexpr (kRaw) return fminf(1.f + __expf(alpha_at(r)), 1.f / kMinAlpha);
+        else return fmaxf(alpha_at(r), kMinAlpha);
     };
     float pr[16];
     float acc = 1.f;
@@ -414,22 +420,21 @@ __device__ void stage_a(const ChunkArgs &p, uint8_t *sm, const SeqSpan &sp, int 
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int r = 16 + i;
-            const float x = (r < Lc) ? alpha_at(r) : 1.f;
-            acc *= (r < Lc) ? fmaxf(x, kMinAlpha) : 1.f;   // rows past the end: identity steps
-            pr[i] = acc;                                     // e_r
+            acc *= (r < Lc) ? factor(r) : 1.f;             // rows past the end: identity steps
+            pr[i] = acc;                                     // e_r (raw: 1/e_r)
         }
-        cst[D + d] = fmaxf(acc, kMinScale);                 // exp(G_end - a)
+        cst[D + d] = fmaxf(kRaw ? ptx::rcp(acc) : acc, kMinScale);   // exp(G_end - a)
     } else {
 #pragma unroll
         for (int i = 15; i >= 0; --i) {
-            pr[i] = acc;                                     // 1/e_r
-            const float x = (i < Lc) ? alpha_at(i) : 1.f;
-            acc *= (i < Lc) ? fmaxf(x, kMinAlpha) : 1.f;
+            pr[i] = acc;                                     // 1/e_r (raw: e_r)
+            acc *= (i < Lc) ? factor(i) : 1.f;
         }
-        const float aexp = fmaxf(acc, kMinScale);           // exp(a)
+        const float aexp = fmaxf(kRaw ? ptx::rcp(acc) : acc, kMinScale);   // exp(a)
         cst[d] = aexp;
         cst[2 * D + d] = (n > 0) ? aexp * cst_prev[D + d] : 0.f;   // state-update factor
     }
+    const bool e_in_pr = (hf == 1) != kRaw;   // pr holds e (else 1/e)
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
         float lk[8], lq[8], ie[8];
@@ -442,8 +447,8 @@ __device__ void stage_a(const ChunkArgs &p, uint8_t *sm, const SeqSpan &sp, int 
                 const int r = 16 * hf + 8 * u + i + t;
                 const float m = fminf(fmaxf(pr[8 * u + i + t], kMinScale), 1.f / kMinScale);
                 const float rm = ptx::rcp(m);
-                e[t] = hf ? m : rm;
-                ie[i + t] = hf ? rm : m;
+                e[t] = e_in_pr ? m : rm;
+                ie[i + t] = e_in_pr ? rm : m;
                 // rows past the sequence's end: zero (the staging may hold another sequence's rows)
                 kv[t] = (r < Lc) ? ld_bf16(stg + STG_K + stg_row(r) + 2 * d) : 0.f;
                 qv[t] = (r < Lc) ? ld_bf16(stg + STG_Q + stg_row(r) + 2 * d) : 0.f;
@@ -711,8 +716,10 @@ __device__ __forceinline__ void write_state16(uint32_t tmem, uint32_t lane_base,
 // Chain warps, operands of chunk n (the staging rows must hold chunk n): part A,
 // then (later) part B, the signal to the issuer and the loads of chunk n+1.
 // Raw inputs: 1/||q_r|| and 1/||k_r|| of chunk n's staged rows (0 past the sequence's
-// end) into the norm ring, four rows of each per chain warp, one row at a time (each
-// lane sums the squares of four channels; a butterfly finishes the row).  The factors
+// end) into the norm ring, four rows of each per chain warp.  Each lane sums the squares
+// of four channels; a transposed butterfly then reduces the eight rows together (over
+// lane bits 4, 3, 2 each lane keeps half of its sums and adds its partner's matching
+// half, ending with sum (lane >> 2) & 7; bits 1, 0 finish it), nine shuffles in all.  The factors
 // are applied after the products, where each one is a row or column scaling:
 //   A_kk -> Diag(nk) A_kk Diag(nk) and W' -> T Diag(beta nk) Lk (prep warps),
 //   the E operand of the state update and of O -> Diag(nk) E, O -> Diag(nq) O (chain),
@@ -720,22 +727,29 @@ __device__ __forceinline__ void write_state16(uint32_t tmem, uint32_t lane_base,
 __device__ __forceinline__ void row_norms(uint8_t *sm, int n, int len, int warp, int lane)
 {
     const uint8_t *stg = sm + OFF_STG;
-    float mine = 0.f;
-#pragma unroll 1
-    for (int i = 0; i < 8; ++i) {
-        const int r = 4 * warp + (i & 3);
-        const uint2 w = *reinterpret_cast<const uint2 *>(stg + (i < 4 ? STG_Q : STG_K) + stg_row(r) + 8 * lane);
+    auto sq4 = [&](int off, int r) {   // this lane's four channels of a staged row, squared and summed
+        const uint2 w = *reinterpret_cast<const uint2 *>(stg + off + stg_row(r) + 8 * lane);
         const float a0 = __uint_as_float(w.x << 16), a1 = __uint_as_float(w.x & 0xFFFF0000u);
         const float a2 = __uint_as_float(w.y << 16), a3 = __uint_as_float(w.y & 0xFFFF0000u);
-        float ss = fmaf(a0, a0, fmaf(a1, a1, fmaf(a2, a2, a3 * a3)));
+        return fmaf(a0, a0, fmaf(a1, a1, fmaf(a2, a2, a3 * a3)));
+    };
+    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+    float w4[4], w2[2];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-        if (lane == i) mine = ss;
+    for (int i = 0; i < 4; ++i) {
+        const float vq = sq4(STG_Q, 4 * warp + i), vk = sq4(STG_K, 4 * warp + i);
+        w4[i] = (b4 ? vk : vq) + __shfl_xor_sync(0xffffffffu, b4 ? vq : vk, 16);
     }
-    if (lane < 8) {
-        const int r = 4 * warp + (lane & 3);
-        reinterpret_cast<float *>(sm + OFF_NRM + (n % kNrmSlots) * NRM_BYTES)[(lane < 4 ? 0 : C) + r] =
-            (n * C + r < len) ? inv_norm(mine) : 0.f;
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+        w2[i] = (b3 ? w4[2 + i] : w4[i]) + __shfl_xor_sync(0xffffffffu, b3 ? w4[i] : w4[2 + i], 8);
+    float w1 = (b2 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? w2[0] : w2[1], 4);
+    w1 += __shfl_xor_sync(0xffffffffu, w1, 2);
+    w1 += __shfl_xor_sync(0xffffffffu, w1, 1);
+    if ((lane & 3) == 0) {
+        const int idx = lane >> 2, r = 4 * warp + (idx & 3);
+        reinterpret_cast<float *>(sm + OFF_NRM + (n % kNrmSlots) * NRM_BYTES)[(idx < 4 ? 0 : C) + r] =
+            (n * C + r < len) ? inv_norm(w1) : 0.f;
     }
 }
 

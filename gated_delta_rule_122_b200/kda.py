@@ -133,9 +133,78 @@ def _to_device(tensors, device):
     return [None if t is None else t.to(device, non_blocking=True) for t in tensors]
 
 
+# Host-buffer prefills of at least two segments run as a pipeline over token segments
+# of this many tokens: the copy of segment j+1 in and of segment j-1's outputs back
+# overlap the kernel on segment j, which continues from segment j-1's final state.
+_HOST_SEGMENT = 1024
+_PIPELINED = ("kda_forward", "kda_forward_scalar_gate", "kda_forward_raw")
+
+
+def _prefill_host_pipelined(fn_name, q, k, v, alpha, beta, initial_state, scale, output_final_state,
+                            out_dtype, out, final_state, check_status, gate_per_head):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    a_shape = (B, T, H) if gate_per_head else (B, T, H, dk)
+    if tuple(k.shape) != (B, T, H, dk) or tuple(v.shape[:3]) != (B, T, H) or tuple(alpha.shape) != a_shape \
+            or tuple(beta.shape) != (B, T, H):
+        raise ValueError("shapes: q,k [B,T,H,dk], alpha " + ("[B,T,H]" if gate_per_head else "[B,T,H,dk]")
+                         + ", v [B,T,H,dv], beta [B,T,H]")
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=out_dtype, pin_memory=True)
+    if tuple(out.shape) != (B, T, H, dv) or out.device.type != "cpu":
+        raise ValueError("out must be a host tensor [B,T,H,dv]")
+    keep = []   # device tensors that must outlive the streams' work
+    with torch.cuda.device(dev):
+        compute = torch.cuda.current_stream(dev)
+        h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        if initial_state is None:
+            state = torch.zeros((B, H, dk, dv), device=dev, dtype=torch.float32)
+        else:
+            state = torch.empty((B, H, dk, dv), device=dev, dtype=torch.float32)
+            state.copy_(initial_state, non_blocking=True)
+        for t0 in range(0, T, _HOST_SEGMENT):
+            t1 = min(T, t0 + _HOST_SEGMENT)
+            seg_in = []
+            with torch.cuda.stream(h2d):
+                for t in (q, k, v, alpha, beta):
+                    d = torch.empty((B, t1 - t0) + tuple(t.shape[2:]), device=dev, dtype=t.dtype)
+                    for b in range(B):   # one contiguous host run per sequence
+                        d[b].copy_(t[b, t0:t1], non_blocking=True)
+                    seg_in.append(d)
+                ready = torch.cuda.Event()
+                ready.record(h2d)
+            compute.wait_event(ready)
+            o_seg = torch.empty((B, t1 - t0, H, dv), device=dev, dtype=out.dtype)
+            _prefill(fn_name, *seg_in, state, scale, True, out_dtype, o_seg, state, None, check_status,
+                     gate_per_head)
+            done = torch.cuda.Event()
+            done.record(compute)
+            d2h.wait_event(done)
+            with torch.cuda.stream(d2h):
+                for b in range(B):
+                    out[b, t0:t1].copy_(o_seg[b], non_blocking=True)
+            keep.append((seg_in, o_seg))
+        if final_state is None and output_final_state:
+            final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, pin_memory=True)
+        if final_state is not None:
+            done = torch.cuda.Event()
+            done.record(compute)
+            d2h.wait_event(done)
+            with torch.cuda.stream(d2h):
+                final_state.copy_(state, non_blocking=True)
+        d2h.synchronize()
+        h2d.synchronize()
+        compute.synchronize()
+    return out, final_state
+
+
 def _prefill(fn_name, q, k, v, alpha, beta, initial_state, scale, output_final_state,
              out_dtype, out, final_state, workspace=None, check_status=False, gate_per_head=False):
     host = q.device.type == "cpu"
+    if host and fn_name in _PIPELINED and q.dim() == 4 and q.shape[1] >= 2 * _HOST_SEGMENT:
+        return _prefill_host_pipelined(fn_name, q, k, v, alpha, beta, initial_state, scale, output_final_state,
+                                       out_dtype, out, final_state, check_status, gate_per_head)
     host_out = host_state = None
     if host:
         # end-to-end path: host inputs are copied in (asynchronously when pinned),

@@ -220,6 +220,26 @@ def test_host_buffers_round_trip():
     assert o_h.device.type == "cpu" and torch.equal(o_h, o_d.cpu()) and torch.equal(S_h, S_d.cpu())
 
 
+@pytest.mark.parametrize("gate", ["channel", "head"])
+def test_host_buffers_pipelined_match_device(gate):
+    """Host tensors of at least two 1024-token segments take the pipelined host path
+    (copies overlapped with the kernel, state carried between segments); it must agree
+    with the device path to fp32 rounding of the carried state, including a partial last
+    segment and an initial state."""
+    w = WORKLOADS["prefill"].scaled(B=2, H=8, T=2100, init_state=True)
+    x = make_inputs(w)
+    if gate == "head":
+        x["alpha"] = x["alpha"][..., 0].contiguous()
+    fn = kda.forward if gate == "channel" else kda.forward_scalar_gate
+    hx = {n: x[n].pin_memory() for n in ("q", "k", "v", "alpha", "beta", "s0")}
+    o_h, s_h = fn(hx["q"], hx["k"], hx["v"], hx["alpha"], hx["beta"], initial_state=hx["s0"], scale=x["scale"])
+    assert o_h.device.type == "cpu" and s_h.device.type == "cpu"
+    d = to_device(x)
+    o_d, s_d = fn(d["q"], d["k"], d["v"], d["alpha"], d["beta"], initial_state=d["s0"], scale=x["scale"])
+    assert o_err(o_h, o_d.cpu().double().numpy()) < 1e-5
+    assert s_err(s_h, s_d.cpu().double().numpy()) < 1e-5
+
+
 def test_status_errors_raise():
     x = to_device(make_inputs(WORKLOADS["tiny"].scaled(T=8, dk=48, dv=16)))
     with pytest.raises(kda.KDAError, match="head size"):
