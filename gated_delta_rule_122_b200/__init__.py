@@ -16,9 +16,10 @@ draws the seeded synthetic workloads.  All arithmetic runs in
 from .kda import (EXPORTED_SYMBOLS, KDAError, decode_step, decode_step_gdn2, decode_step_raw,
                   decode_step_scalar_gate, decode_tokens, forward, forward_gdn2, forward_raw,
                   forward_scalar_gate, forward_sequential, forward_varlen, library, library_path,
-                  state_copy, status_string, version)
+                  selftest_bounded_wait, state_copy, status_string, version)
 
 __all__ = ["forward", "forward_varlen", "forward_scalar_gate", "forward_gdn2", "forward_raw",
            "forward_sequential", "decode_step", "decode_step_scalar_gate", "decode_step_gdn2",
-           "decode_step_raw", "decode_tokens", "state_copy", "KDAError", "library", "library_path",
+           "decode_step_raw", "decode_tokens", "state_copy", "selftest_bounded_wait", "KDAError", "library",
+           "library_path",
            "status_string", "version", "EXPORTED_SYMBOLS"]

@@ -407,4 +407,16 @@ kda_status kda_state_copy(const float *src, const int *src_index, int src_slots,
     return kda::launch_state_copy(a, stream) == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
 }
 
+kda_status kda_selftest_bounded_wait(int arrive, unsigned int limit_us, void *status, cudaStream_t stream)
+{
+    if (!status) return KDA_ERR_NULL;
+    if (!aligned16(status)) return KDA_ERR_ALIGN;
+    if (limit_us == 0 || limit_us > 2000000u) return KDA_ERR_SHAPE;
+    if (cudaMemsetAsync(status, 0, sizeof(unsigned int), stream) != cudaSuccess) return KDA_ERR_LAUNCH;
+    return kda::launch_bounded_wait_selftest(arrive, 1000ull * limit_us, static_cast<unsigned int *>(status),
+                                             stream) == cudaSuccess
+               ? KDA_OK
+               : KDA_ERR_LAUNCH;
+}
+
 }  // extern "C"

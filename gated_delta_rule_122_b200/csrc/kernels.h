@@ -82,6 +82,8 @@ struct StateCopyArgs {
     unsigned int *status;   // device status word or null
 };
 cudaError_t launch_state_copy(const StateCopyArgs &a, cudaStream_t s);
+cudaError_t launch_bounded_wait_selftest(int arrive, unsigned long long limit_ns, unsigned int *status,
+                                         cudaStream_t s);
 cudaError_t launch_chunk_simt(const ChunkArgs &a, int dk, int dv, cudaStream_t s);
 // (both take GDN-2 gates when a.erase is set)
 bool chunk_tc_supported(int dk, int dv, kda_dtype qkv, kda_dtype gate);

@@ -17,7 +17,8 @@ import torch
 
 __all__ = ["KDAError", "forward", "forward_varlen", "forward_scalar_gate", "forward_gdn2",
            "forward_raw", "forward_sequential", "decode_step", "decode_step_raw",
-           "decode_step_scalar_gate", "decode_step_gdn2", "decode_tokens", "state_copy", "library",
+           "decode_step_scalar_gate", "decode_step_gdn2", "decode_tokens", "state_copy",
+           "selftest_bounded_wait", "library",
            "library_path", "status_string", "version", "EXPORTED_SYMBOLS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -29,7 +30,8 @@ EXPORTED_SYMBOLS = ("kda_forward", "kda_forward_workspace_bytes", "kda_workspace
                     "kda_forward_noalloc", "kda_forward_varlen", "kda_forward_scalar_gate",
                     "kda_forward_gdn2", "kda_forward_raw", "kda_forward_sequential", "kda_decode_step",
                     "kda_decode_step_gdn2", "kda_decode_step_raw", "kda_decode_step_scalar_gate",
-                    "kda_decode_tokens", "kda_state_copy", "kda_status_string", "kda_version")
+                    "kda_decode_tokens", "kda_state_copy", "kda_selftest_bounded_wait", "kda_status_string",
+                    "kda_version")
 
 _DT = {torch.float32: 0, torch.bfloat16: 1}
 _vp = ctypes.c_void_p
@@ -86,6 +88,8 @@ def library() -> ctypes.CDLL:
             lib.kda_decode_tokens.restype = _i
             lib.kda_state_copy.argtypes = [_vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp]
             lib.kda_state_copy.restype = _i
+            lib.kda_selftest_bounded_wait.argtypes = [_i, ctypes.c_uint, _vp, _vp]
+            lib.kda_selftest_bounded_wait.restype = _i
             lib.kda_forward_workspace_bytes.argtypes = [_i] * 5
             lib.kda_forward_workspace_bytes.restype = ctypes.c_size_t
             lib.kda_workspace_status.argtypes = [_vp, _vp]
@@ -608,3 +612,18 @@ def state_copy(src, dst, src_index=None, dst_index=None, count=None, check_statu
     if code != 0:
         raise KDAError("kda_state_copy", code)
     return dst
+
+
+def selftest_bounded_wait(arrive, limit_us=20000, device=None):
+    """Run the device-side bounded-wait check (C entry point ``kda_selftest_bounded_wait``)
+    and return the status code that ``kda_workspace_status`` reads back: 0 when the
+    barrier was completed (arrive=True), KDA_ERR_TIMEOUT (8) after a wait that gave up."""
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    status = _status_word(device)
+    lib = library()
+    with torch.cuda.device(device):
+        stream = _vp(_stream_handle(device))
+        code = lib.kda_selftest_bounded_wait(int(bool(arrive)), int(limit_us), _ptr(status), stream)
+        if code != 0:
+            raise KDAError("kda_selftest_bounded_wait", code)
+        return lib.kda_workspace_status(_ptr(status), stream)

@@ -364,6 +364,20 @@ kda_status kda_state_copy(const float *src, const int *src_index, int src_slots,
                           int count, int H, int d_k, int d_v, void *status,
                           cudaStream_t stream);
 
+/*
+ * kda_selftest_bounded_wait -- a check of the device-side failure detection that
+ * the tensor-core prefill uses (no counterpart on the pages): one thread waits on an
+ * mbarrier with the prefill's bounded-wait helper.  arrive != 0 completes the
+ * barrier's phase first (the wait succeeds); arrive == 0 leaves it incomplete, so
+ * the wait gives up after limit_us microseconds (1 .. 2,000,000) and records the
+ * timeout in the status word.  status: a 16-byte-aligned device word (for instance a
+ * workspace of kda_forward_workspace_bytes() bytes), zeroed by the call; read it with
+ * kda_workspace_status(): KDA_ERR_TIMEOUT after a wait that gave up, KDA_OK
+ * otherwise.  The kernel returns normally either way; the context stays usable.
+ */
+kda_status kda_selftest_bounded_wait(int arrive, unsigned int limit_us, void *status,
+                                     cudaStream_t stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char *kda_status_string(kda_status status);
 
