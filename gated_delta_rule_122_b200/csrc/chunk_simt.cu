@@ -198,20 +198,25 @@ kda_chunk_simt_kernel(ChunkArgs a)
         }
         __syncthreads();
 
-        // 5. E = U - W S and the inter-chunk read (Q * gamma) S
-        float oacc[RPT_C];
+        // 5. E = U - W S and the inter-chunk read (Q * gamma) S: each S element is read
+        //    once per thread and used for all of the thread's rows
+        float oacc[RPT_C], eacc[RPT_C];
 #pragma unroll
         for (int m = 0; m < RPT_C; ++m) {
-            const int r = rgrp + NRG * m;
-            float e = V[r * PV + jcol], o = 0.f;
-            for (int d = 0; d < DK; ++d) {
-                const float sdj = S[d * DV + jcol];
-                e = fmaf(-W[r * PK + d], sdj, e);
-                o = fmaf(Q[r * PK + d], sdj, o);
-            }
-            E[r * PV + jcol] = e;
-            oacc[m] = o;
+            eacc[m] = V[(rgrp + NRG * m) * PV + jcol];
+            oacc[m] = 0.f;
         }
+        for (int d = 0; d < DK; ++d) {
+            const float sdj = S[d * DV + jcol];
+#pragma unroll
+            for (int m = 0; m < RPT_C; ++m) {
+                const int r = rgrp + NRG * m;
+                eacc[m] = fmaf(-W[r * PK + d], sdj, eacc[m]);
+                oacc[m] = fmaf(Q[r * PK + d], sdj, oacc[m]);
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < RPT_C; ++m) E[(rgrp + NRG * m) * PV + jcol] = eacc[m];
         __syncthreads();
 
         // 6. outputs: O = scale (inter + Aqk E)
@@ -225,13 +230,23 @@ kda_chunk_simt_kernel(ChunkArgs a)
                 st_elem(a.o, row * DV + jcol, a.scale * o, a.out_bf16);
             }
         }
-        // 7. state fast-forward: S <- Diag(gamma_end) S + K_end^T E
-#pragma unroll 4
-        for (int m = 0; m < RPT_K; ++m) {
-            const int i = rgrp + NRG * m;
-            float s = S[i * DV + jcol] * expf(G[(C - 1) * PK + i]);
-            for (int r = 0; r < C; ++r) s = fmaf(K[r * PK + i], E[r * PV + jcol], s);
-            S[i * DV + jcol] = s;
+        // 7. state fast-forward: S <- Diag(gamma_end) S + K_end^T E, eight state rows at a
+        //    time so that each E element read serves eight of them
+        constexpr int SG = (RPT_K % 8 == 0) ? 8 : 1;
+        for (int m0 = 0; m0 < RPT_K; m0 += SG) {
+            float acc[SG];
+#pragma unroll
+            for (int g = 0; g < SG; ++g) {
+                const int i = rgrp + NRG * (m0 + g);
+                acc[g] = S[i * DV + jcol] * expf(G[(C - 1) * PK + i]);
+            }
+            for (int r = 0; r < C; ++r) {
+                const float erj = E[r * PV + jcol];
+#pragma unroll
+                for (int g = 0; g < SG; ++g) acc[g] = fmaf(K[r * PK + rgrp + NRG * (m0 + g)], erj, acc[g]);
+            }
+#pragma unroll
+            for (int g = 0; g < SG; ++g) S[(rgrp + NRG * (m0 + g)) * DV + jcol] = acc[g];
         }
         __syncthreads();
     }

@@ -256,8 +256,9 @@ __device__ __forceinline__ void issue_m4(uint8_t *sm, uint32_t tmem, const Bars 
                           ptx::smem_desc(aq + 256 * ks, 128, 512), id.O2, 1);
     for (int ks = 0; ks < C / 16; ++ks)
         for (int pa = 0; pa < 2; ++pa)
-            for (int pb = 0; pb < 2; ++pb)
-                // R as the K-major (N = d, K = s) operand: token blocks 2 slabs apart
+            for (int pb = 0; pb < 2 - pa; ++pb)
+                // R as the K-major (N = d, K = s) operand: token blocks 2 slabs apart.  The
+                // E_lo R_lo term (2^-16 of the product) is left out: three cross terms.
                 ptx::mma_bf16(tmem + TM_S, ptx::smem_desc(et + C * 16 * pa + 256 * ks, 128, C * 32),
                               ptx::smem_desc(rr + SLAB * pb + 4 * SLAB * ks, 2 * SLAB, 128), id.dS, 1);
     ptx::mma_commit(bars.s);
