@@ -41,11 +41,11 @@ if ROOT not in sys.path:
 METRIC = "KDA prefill Mtokens/s (H=64,d=128); decode-step HBM GB/s vs ~8 TB/s peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of the prefill
-# kernel (1.08 GB read + 0.5094 GB written), from the capture summarised under
+# kernel (1.08 GB read + 0.5087 GB written), from the capture summarised under
 # profiles/, with the hash of the kernel sources it was taken for: once the
 # sources change, the line reports traffic as null until it is captured again.
-PREFILL_TRAFFIC_BYTES = 1_589_420_000
-PREFILL_TRAFFIC_SOURCES = "f74743b1bf745d09"
+PREFILL_TRAFFIC_BYTES = 1_588_670_000
+PREFILL_TRAFFIC_SOURCES = "01c9f9f2031d0f2b"
 
 
 def kernel_sources_hash() -> str:
