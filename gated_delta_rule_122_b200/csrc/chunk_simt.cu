@@ -30,7 +30,13 @@ namespace kda {
 
 
 constexpr int kSimtChunk = 32;
-constexpr int kSimtThreads = 256;
+// 512 threads per block where the thread mappings below allow it (16 warps per SM hide
+// the shared-memory latency of the fp32 loops better than 8), else 256.
+template <int DK, int DV>
+constexpr int simt_threads()
+{
+    return (512 % DV == 0 && 32 % (512 / DV) == 0 && DK % (512 / DV) == 0) ? 512 : 256;
+}
 
 template <int DK, int DV>
 struct SimtLayout {
@@ -52,11 +58,11 @@ struct SimtLayout {
 };
 
 template <int DK, int DV, bool kGdn2>
-__global__ void __launch_bounds__(kSimtThreads)
+__global__ void __launch_bounds__(simt_threads<DK, DV>())
 kda_chunk_simt_kernel(ChunkArgs a)
 {
     using Ly = SimtLayout<DK, DV>;
-    constexpr int C = Ly::C, PK = Ly::PK, PV = Ly::PV, PC = Ly::PC, NT = kSimtThreads;
+    constexpr int C = Ly::C, PK = Ly::PK, PV = Ly::PV, PC = Ly::PC, NT = simt_threads<DK, DV>();
     constexpr int NRG = NT / DV;          // row groups for value-column loops
     constexpr int RPT_C = C / NRG;        // chunk rows per thread
     constexpr int RPT_K = DK / NRG;       // key rows per thread (state update)
@@ -264,7 +270,7 @@ static cudaError_t launch_chunk_simt_t(const ChunkArgs &a, cudaStream_t stream)
     auto kernel = a.erase ? kda_chunk_simt_kernel<DK, DV, true> : kda_chunk_simt_kernel<DK, DV, false>;
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Ly::bytes);
     if (err != cudaSuccess) return err;
-    kernel<<<(unsigned)blocks, kSimtThreads, Ly::bytes, stream>>>(a);
+    kernel<<<(unsigned)blocks, simt_threads<DK, DV>(), Ly::bytes, stream>>>(a);
     return cudaGetLastError();
 }
 
