@@ -37,7 +37,7 @@ struct RecurrentShape {
 };
 
 
-template <int DK, int DV, bool kGdn2>
+template <int DK, int DV, bool kGdn2, bool kRaw>
 __global__ void __launch_bounds__(RecurrentShape<DK, DV>::NT)
 kda_recurrent_kernel(RecurrentArgs a)
 {
@@ -83,7 +83,7 @@ kda_recurrent_kernel(RecurrentArgs a)
             s_q[buf][i] = ld_elem(a.q, row * DK + i, a.qkv_bf16);
             s_k[buf][i] = ld_elem(a.k, row * DK + i, a.qkv_bf16);
             const float x = ld_elem(a.alpha, a.gate_per_head ? row : row * DK + i, a.gate_bf16);
-            s_a[buf][i] = a.raw_inputs ? __expf(log_alpha_from_logit(x)) : x;
+            s_a[buf][i] = kRaw ? __expf(log_alpha_from_logit(x)) : x;
         }
         for (int j = tid; j < DV; j += NT) s_v[buf][j] = ld_elem(a.v, row * DV + j, a.qkv_bf16);
         if constexpr (kGdn2) {
@@ -92,7 +92,7 @@ kda_recurrent_kernel(RecurrentArgs a)
         } else {
             if (tid == 0) {
                 const float y = ld_elem(a.beta, row, a.gate_bf16);
-                s_beta[buf] = a.raw_inputs ? sigmoid_of(y) : y;
+                s_beta[buf] = kRaw ? sigmoid_of(y) : y;
             }
         }
         __syncthreads();
@@ -117,17 +117,21 @@ kda_recurrent_kernel(RecurrentArgs a)
             for (int i = tid; i < DK; i += 32) {
                 const float ki = s_k[buf][i], qi = s_q[buf][i];
                 kq = fmaf(ki, qi, kq);
-                kk = fmaf(ki, ki, kk);
-                qq = fmaf(qi, qi, qq);
+                if constexpr (kRaw) {
+                    kk = fmaf(ki, ki, kk);
+                    qq = fmaf(qi, qi, qq);
+                }
             }
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) {
                 kq += __shfl_xor_sync(0xffffffffu, kq, off);
-                kk += __shfl_xor_sync(0xffffffffu, kk, off);
-                qq += __shfl_xor_sync(0xffffffffu, qq, off);
+                if constexpr (kRaw) {
+                    kk += __shfl_xor_sync(0xffffffffu, kk, off);
+                    qq += __shfl_xor_sync(0xffffffffu, qq, off);
+                }
             }
             if (tid == 0) {
-                const float nk = a.raw_inputs ? inv_norm(kk) : 1.f, nq = a.raw_inputs ? inv_norm(qq) : 1.f;
+                const float nk = kRaw ? inv_norm(kk) : 1.f, nq = kRaw ? inv_norm(qq) : 1.f;
                 s_kq[buf] = kq * nk * nq;
                 s_nk[buf] = nk;
                 s_nq[buf] = nq;
@@ -140,8 +144,10 @@ kda_recurrent_kernel(RecurrentArgs a)
             float rr = 0.f, pp = 0.f;
 #pragma unroll
             for (int g = 0; g < NRG; ++g) { rr += red_r[g][j]; pp += red_p[g][j]; }
-            rr *= s_nk[buf];   // reads with the unit key and query (1 unless inputs are raw)
-            pp *= s_nq[buf];
+            if constexpr (kRaw) {   // reads with the unit key and query
+                rr *= s_nk[buf];
+                pp *= s_nq[buf];
+            }
             const float e = kGdn2 ? s_w[buf][j] * s_v[buf][j] - rr : s_beta[buf] * (s_v[buf][j] - rr);
             s_e[buf][j] = e;
             st_elem(a.o, row * DV + j, a.scale * fmaf(e, s_kq[buf], pp), a.out_bf16);
@@ -152,7 +158,7 @@ kda_recurrent_kernel(RecurrentArgs a)
         const float4 e4 = *reinterpret_cast<const float4 *>(&s_e[buf][4 * cg]);
 #pragma unroll
         for (int m = 0; m < RPT; ++m) {
-            const float kk = s_k[buf][rg + NRG * m] * s_nk[buf];
+            const float kk = kRaw ? s_k[buf][rg + NRG * m] * s_nk[buf] : s_k[buf][rg + NRG * m];
             s[m].x = fmaf(kk, e4.x, s[m].x); s[m].y = fmaf(kk, e4.y, s[m].y);
             s[m].z = fmaf(kk, e4.z, s[m].z); s[m].w = fmaf(kk, e4.w, s[m].w);
         }
@@ -178,10 +184,13 @@ static cudaError_t launch_recurrent_t(const RecurrentArgs &a, cudaStream_t strea
     using Sh = RecurrentShape<DK, DV>;
     const long long blocks = (long long)a.B * a.H;
     if (blocks == 0) return cudaSuccess;
+    if (a.erase && a.raw_inputs) return cudaErrorInvalidValue;   // no entry point combines them
     if (a.erase)
-        kda_recurrent_kernel<DK, DV, true><<<(unsigned)blocks, Sh::NT, 0, stream>>>(a);
+        kda_recurrent_kernel<DK, DV, true, false><<<(unsigned)blocks, Sh::NT, 0, stream>>>(a);
+    else if (a.raw_inputs)
+        kda_recurrent_kernel<DK, DV, false, true><<<(unsigned)blocks, Sh::NT, 0, stream>>>(a);
     else
-        kda_recurrent_kernel<DK, DV, false><<<(unsigned)blocks, Sh::NT, 0, stream>>>(a);
+        kda_recurrent_kernel<DK, DV, false, false><<<(unsigned)blocks, Sh::NT, 0, stream>>>(a);
     return cudaGetLastError();
 }
 
