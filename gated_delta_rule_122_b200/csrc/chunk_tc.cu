@@ -202,11 +202,13 @@ __device__ __forceinline__ float load_beta(const ChunkArgs &p, const SeqSpan &sp
 // MN-major core-matrix layout of the U^T product; o as boxes of 16 token rows.
 struct TcMaps {
     CUtensorMap q, k, a, v, o;
-    // one gate per head: 1 when map a stages each chunk's gates as a box of 8 heads x 32
-    // tokens (H a multiple of 8, alpha 16-byte aligned); 0 when they are read from memory
-    int head_gate_tma;
 };
 constexpr int HG_ROW = 16;   // bytes per token row of a staged per-head gate box
+
+// The gate kind is a template parameter of the kernel (a run-time choice inside stage A
+// costs the chain measurably): alpha rows per token and key channel, one gate per
+// (token, head) staged by TMA as boxes of 8 heads x 32 tokens, or read from memory.
+constexpr int kGateChannel = 0, kGateHeadTma = 1, kGateHeadMem = 2;
 
 // Every warp of a role adds 1 to a readiness counter once its writes are visible
 // (the counter of chunk n's step reaches (n + 1) x the role's warps).
@@ -389,9 +391,9 @@ __device__ __forceinline__ void solve_diag_blocks(const float *At, float *Tm, in
 // Part A only touches slabs the A product (M1), the W'/U product (M2) and the O/E
 // product (M3) of the chunk two back have finished with, so it can run while that
 // chunk's state update (M4) still reads R.
-template <bool kHeadGate, bool kRaw>
+template <int kGate, bool kRaw>
 __device__ void stage_a(const ChunkArgs &p, uint8_t *sm, const SeqSpan &sp, int h, int n, int warp, int lane,
-                        uint32_t (&rw)[16], bool head_staged)
+                        uint32_t (&rw)[16])
 {
     const int hf = warp >> 2, d = 32 * (warp & 3) + lane;
     const int Lc = min(C, sp.len - n * C);
@@ -403,8 +405,8 @@ __device__ void stage_a(const ChunkArgs &p, uint8_t *sm, const SeqSpan &sp, int 
     // gate straight from global memory (the same 32 values for every thread)
     const __nv_bfloat16 *ah = (const __nv_bfloat16 *)p.alpha + (sp.tok0 + (size_t)n * C) * p.H + h;
     auto alpha_at = [&](int r) {
-        if constexpr (kHeadGate)
-            return head_staged ? ld_bf16(stg + STG_A + HG_ROW * r + 2 * (h & 7)) : __bfloat162float(ah[(size_t)r * p.H]);
+        if constexpr (kGate == kGateHeadTma) return ld_bf16(stg + STG_A + HG_ROW * r + 2 * (h & 7));
+        else if constexpr (kGate == kGateHeadMem) return __bfloat162float(ah[(size_t)r * p.H]);
         else return ld_bf16(stg + STG_A + stg_row(r) + 2 * d);
     };
     // Per-token factor of the running products: alpha (floored at e^-80), or with a gate
@@ -483,22 +485,20 @@ __device__ void stage_b(uint8_t *sm, int n, int warp, int lane, const uint32_t (
 // t0 (b = sequence, t0 = 0 for the dense layout; b = 0, t0 = its offset when packed).
 struct TmaPos {
     int b, h, t0;
-    int gate_rows;   // 1: alpha rows per token (per-key-channel gate); 2: a per-head gate box; 0: none
 };
 
 // TMA loads of chunk n's q, k, alpha rows into the staging rows (one thread).  Rows
 // past the sequence's end are masked where they are used.
-template <bool kHeadGate>
+template <int kGate>
 __device__ __forceinline__ void load_qka(const TcMaps &maps, uint8_t *sm, const Bars &bars, const TmaPos &tp, int n)
 {
     const uint32_t dst = ptx::smem_u32(sm + OFF_STG);
-    if constexpr (!kHeadGate) ptx::mbar_arrive_expect_tx(bars.stg, 3 * STG_T);
-    else ptx::mbar_arrive_expect_tx(bars.stg, 2 * STG_T + (tp.gate_rows == 2 ? C * HG_ROW : 0));
+    ptx::mbar_arrive_expect_tx(bars.stg, 2 * STG_T + (kGate == kGateChannel ? STG_T : kGate == kGateHeadTma ? C * HG_ROW : 0));
     ptx::tma_load_4d(dst + STG_Q, &maps.q, bars.stg, 0, tp.h, tp.t0 + n * C, tp.b);
     ptx::tma_load_4d(dst + STG_K, &maps.k, bars.stg, 0, tp.h, tp.t0 + n * C, tp.b);
-    if constexpr (!kHeadGate) ptx::tma_load_4d(dst + STG_A, &maps.a, bars.stg, 0, tp.h, tp.t0 + n * C, tp.b);
+    if constexpr (kGate == kGateChannel) ptx::tma_load_4d(dst + STG_A, &maps.a, bars.stg, 0, tp.h, tp.t0 + n * C, tp.b);
     // heads h & ~7 .. (h & ~7) + 7 of 32 tokens: the x coordinate is a multiple of 8 elements
-    else if (tp.gate_rows == 2) ptx::tma_load_3d(dst + STG_A, &maps.a, bars.stg, tp.h & ~7, tp.t0 + n * C, tp.b);
+    if constexpr (kGate == kGateHeadTma) ptx::tma_load_3d(dst + STG_A, &maps.a, bars.stg, tp.h & ~7, tp.t0 + n * C, tp.b);
 }
 
 // TMA load of chunk n's v rows into V buffer n&1 (one thread).
@@ -754,16 +754,16 @@ __device__ __forceinline__ void row_norms(uint8_t *sm, int n, int len, int warp,
     }
 }
 
-template <bool kHeadGate, bool kRaw>
+template <int kGate, bool kRaw>
 __device__ __forceinline__ void chain_stage_a(const ChunkArgs &p, uint8_t *sm, const Bars &bars, const SeqSpan &sp, int h, int n, int warp,
-                                              int lane, uint32_t (&ie)[16], volatile int *err_flag, bool head_staged)
+                                              int lane, uint32_t (&ie)[16], volatile int *err_flag)
 {
     if (!ptx::mbar_wait(bars.stg, (uint32_t)(n & 1), kWaitLimitNs)) *err_flag = 1;   // chunk n's rows
     if constexpr (kRaw) row_norms(sm, n, sp.len, warp, lane);
-    stage_a<kHeadGate, kRaw>(p, sm, sp, h, n, warp, lane, ie, head_staged);
+    stage_a<kGate, kRaw>(p, sm, sp, h, n, warp, lane, ie);
 }
 
-template <bool kHeadGate>
+template <int kGate>
 __device__ __forceinline__ void chain_stage_b(const TcMaps &maps, uint8_t *sm, const Bars &bars, const TmaPos &tp,
                                               int n, int nchunks, int tid, int warp, int lane,
                                               const uint32_t (&ie)[16])
@@ -772,7 +772,7 @@ __device__ __forceinline__ void chain_stage_b(const TcMaps &maps, uint8_t *sm, c
     ptx::fence_proxy_async_smem();
     warp_signal(bars.rc, lane);
     chain_bar();   // staging consumed, constants visible to every chain warp
-    if (tid == 0 && n + 1 < nchunks) load_qka<kHeadGate>(maps, sm, bars, tp, n + 1);
+    if (tid == 0 && n + 1 < nchunks) load_qka<kGate>(maps, sm, bars, tp, n + 1);
 }
 
 __device__ __forceinline__ void warp_signal_after_stage(const Bars &bars, int lane)
@@ -782,7 +782,7 @@ __device__ __forceinline__ void warp_signal_after_stage(const Bars &bars, int la
 }
 
 // ---- the chain warps: the serial recurrence over chunks --------------------------------
-template <bool kHeadGate, bool kRaw>
+template <int kGate, bool kRaw>
 __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, uint32_t tmem, const Bars &bars,
                            const TmaPos &tp, const SeqSpan &sp, int h, int bh, int nchunks, volatile int *err_flag)
 {
@@ -794,11 +794,11 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
     const size_t tile = (size_t)bh * D * D;
 
     uint32_t ie[16];   // R of the chunk being staged (split words), carried from part A to part B
-    if (tid == 0) load_qka<kHeadGate>(maps, sm, bars, tp, 0);
+    if (tid == 0) load_qka<kGate>(maps, sm, bars, tp, 0);
     int staged = 0;   // chunks whose rows have been waited for
-    chain_stage_a<kHeadGate, kRaw>(p, sm, bars, sp, h, 0, warp, lane, ie, err_flag, tp.gate_rows == 2);
+    chain_stage_a<kGate, kRaw>(p, sm, bars, sp, h, 0, warp, lane, ie, err_flag);
     staged = 1;
-    chain_stage_b<kHeadGate>(maps, sm, bars, tp, 0, nchunks, tid, warp, lane, ie);
+    chain_stage_b<kGate>(maps, sm, bars, tp, 0, nchunks, tid, warp, lane, ie);
 
     // S'_0 = Diag(exp(a_0)) S_0; cleared O accumulator
     {
@@ -818,9 +818,9 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
     ptx::tc_fence_before();
     warp_signal(bars.rs, lane);
     if (nchunks > 1) {
-        chain_stage_a<kHeadGate, kRaw>(p, sm, bars, sp, h, 1, warp, lane, ie, err_flag, tp.gate_rows == 2);
+        chain_stage_a<kGate, kRaw>(p, sm, bars, sp, h, 1, warp, lane, ie, err_flag);
         staged = 2;
-        chain_stage_b<kHeadGate>(maps, sm, bars, tp, 1, nchunks, tid, warp, lane, ie);
+        chain_stage_b<kGate>(maps, sm, bars, tp, 1, nchunks, tid, warp, lane, ie);
     }
 
     for (int c = 0; c < nchunks; ++c) {
@@ -855,7 +855,7 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
         warp_signal(bars.re, lane);
         // Lk, Lq of chunk c+2 while the state update of chunk c runs
         if (c + 2 < nchunks) {
-            chain_stage_a<kHeadGate, kRaw>(p, sm, bars, sp, h, c + 2, warp, lane, ie, err_flag, tp.gate_rows == 2);
+            chain_stage_a<kGate, kRaw>(p, sm, bars, sp, h, c + 2, warp, lane, ie, err_flag);
             staged = c + 3;
         }
 
@@ -967,7 +967,7 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
             ptx::bulk_commit();
             if (c + 3 < nchunks) {
                 ptx::bulk_wait_read();   // the tile has been read: the staging rows can be refilled
-                load_qka<kHeadGate>(maps, sm, bars, tp, c + 3);
+                load_qka<kGate>(maps, sm, bars, tp, c + 3);
             }
         }
         if (stop) break;
@@ -978,9 +978,10 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
     if (tid == 0) ptx::bulk_wait();   // the output stores are complete
 }
 
-// kHeadGate: one retention factor per (token, head), alpha [B, T, H] (Gated DeltaNet).
-// kRaw: the input preprocessing is fused into the staging (raw q, k and logits).
-template <bool kHeadGate, bool kRaw>
+// kGate: alpha per key channel [B, T, H, d_k], or one retention factor per (token, head),
+// alpha [B, T, H] (Gated DeltaNet), staged by TMA or read from memory.
+// kRaw: the input preprocessing is fused into the kernel (raw q, k and logits).
+template <int kGate, bool kRaw>
 __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs pa, const __grid_constant__ TcMaps maps)
 {
     extern __shared__ __align__(1024) uint8_t sm[];
@@ -995,8 +996,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs pa, const
         return;
     }
     // TMA coordinates: dense tensors by (batch, token); packed ones as one batch by token row
-    const TmaPos tp{pa.cu_seqlens ? 0 : bh / pa.H, h, pa.cu_seqlens ? (int)sp.tok0 : 0,
-                    pa.gate_per_head ? (maps.head_gate_tma ? 2 : 0) : 1};
+    const TmaPos tp{pa.cu_seqlens ? 0 : bh / pa.H, h, pa.cu_seqlens ? (int)sp.tok0 : 0};
     const int nchunks = (sp.len + C - 1) / C;
     if (nchunks == 0) {
         // an empty sequence: the final state is the initial one (or zeros)
@@ -1044,7 +1044,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs pa, const
     } else if (warp >= NCW) {
         prep_role<kRaw>(p, maps, sm, tmem, bars, tp, sp, h, nchunks, err_flag);
     } else {
-        chain_role<kHeadGate, kRaw>(p, maps, sm, tmem, bars, tp, sp, h, bh, nchunks, err_flag);
+        chain_role<kGate, kRaw>(p, maps, sm, tmem, bars, tp, sp, h, bh, nchunks, err_flag);
     }
     if (*err_flag && tid == 0 && p.status) atomicOr(p.status, 1u);
     ptx::tc_fence_before();
@@ -1142,22 +1142,23 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, int dk, int dv, cudaStream_t str
     if (encode_fn() == nullptr) return cudaErrorNotSupported;
     tc::TcMaps maps;
     const int mb = a.cu_seqlens ? 1 : a.B;   // packed sequences: one [1, T, H, d] tensor
-    maps.head_gate_tma = 0;
+    bool head_gate_tma = false;
     if (a.gate_per_head) {
         // [B][T][H] gates as boxes of 8 heads x 32 tokens when the layout allows a TMA box
         // (16-byte rows of heads and a 16-byte-aligned base); otherwise read per token
         memset(&maps.a, 0, sizeof(maps.a));
-        if (a.H % 8 == 0 && ((uintptr_t)a.alpha & 15u) == 0 && encode_head_gate(&maps.a, a.alpha, mb, a.T, a.H))
-            maps.head_gate_tma = 1;
+        head_gate_tma = a.H % 8 == 0 && ((uintptr_t)a.alpha & 15u) == 0 &&
+                        encode_head_gate(&maps.a, a.alpha, mb, a.T, a.H);
     }
     if (!encode_rows(&maps.q, a.q, mb, a.T, a.H) || !encode_rows(&maps.k, a.k, mb, a.T, a.H) ||
         (!a.gate_per_head && !encode_rows(&maps.a, a.alpha, mb, a.T, a.H)) || !encode_v(&maps.v, a.v, mb, a.T, a.H) ||
         !encode_out(&maps.o, a.o, mb, a.T, a.H, a.out_bf16))
         return cudaErrorInvalidValue;
     if (a.gate_per_head && a.raw_inputs) return cudaErrorInvalidValue;
-    auto kernel = a.gate_per_head ? tc::kda_chunk_tc_kernel<true, false>
-                  : a.raw_inputs  ? tc::kda_chunk_tc_kernel<false, true>
-                                  : tc::kda_chunk_tc_kernel<false, false>;
+    auto kernel = a.gate_per_head ? (head_gate_tma ? tc::kda_chunk_tc_kernel<tc::kGateHeadTma, false>
+                                                   : tc::kda_chunk_tc_kernel<tc::kGateHeadMem, false>)
+                  : a.raw_inputs  ? tc::kda_chunk_tc_kernel<tc::kGateChannel, true>
+                                  : tc::kda_chunk_tc_kernel<tc::kGateChannel, false>;
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     kernel<<<(unsigned)blocks, tc::NT, tc::SMEM_BYTES, stream>>>(a, maps);
