@@ -264,11 +264,11 @@ kda_status kda_decode_step_scalar_gate(const void *q, const void *k,
  *               divided by their L2 norms in the kernel (a zero row stays
  *               zero) -- "Notes on Linear Attention: From Linear Attention to
  *               KDA", section 5.3 "Why L2-normalize the key?" (and the
- *               query, as later DeltaNet-style models do: section 3)
+ *               query likewise, section 3)
  *   gate_logit  [B, T, H, d_k] gate_dtype: x with log alpha = -softplus(x),
- *               i.e. alpha = 1 / (1 + e^x) -- the log-decay g = log alpha <= 0
- *               that implementations keep ("Kimi Delta Attention (KDA)",
- *               brain.bigb.es), in the exp(-softplus) form of the gate
+ *               i.e. alpha = 1 / (1 + e^x) -- the stored log-decay
+ *               g = log alpha <= 0 of "Kimi Delta Attention (KDA)"
+ *               (brain.bigb.es), in the exp(-softplus) form of the gate
  *   beta_logit  [B, T, H] gate_dtype: y with beta = sigmoid(y) ("From Fast
  *               Weight Programmers to KDA", the delta rule's write strength)
  * Everything else (layouts, workspace, aliasing, status) is as kda_forward.

@@ -2,10 +2,10 @@
 
 "Notes on Linear Attention" section 5.3: with a unit key the read-back after a
 write interpolates exactly between the old prediction and the target, so the key
-is L2-normalised (and, in later DeltaNet-style models, the query too).  "Kimi
-Delta Attention (KDA)": implementations keep the log-decay g = log alpha <= 0;
-the workloads' gate is alpha = exp(-softplus(x)).  "From Fast Weight Programmers
-to KDA": beta = sigmoid of a projection.
+is L2-normalised (section 3: the query likewise).  "Kimi Delta Attention (KDA)":
+the log-decay g = log alpha <= 0 is what is stored; the workloads' gate is
+alpha = exp(-softplus(x)).  "From Fast Weight Programmers to KDA": beta = sigmoid
+of a projection.
 """
 import numpy as np
 
