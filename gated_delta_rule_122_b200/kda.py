@@ -146,7 +146,6 @@ _PIPELINED = ("kda_forward", "kda_forward_scalar_gate", "kda_forward_raw")
 
 def _prefill_host_pipelined(fn_name, q, k, v, alpha, beta, initial_state, scale, output_final_state,
                             out_dtype, out, final_state, check_status, gate_per_head):
-    dev = torch.device("cuda", torch.cuda.current_device())
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     a_shape = (B, T, H) if gate_per_head else (B, T, H, dk)
@@ -154,10 +153,15 @@ def _prefill_host_pipelined(fn_name, q, k, v, alpha, beta, initial_state, scale,
             or tuple(beta.shape) != (B, T, H):
         raise ValueError("shapes: q,k [B,T,H,dk], alpha " + ("[B,T,H]" if gate_per_head else "[B,T,H,dk]")
                          + ", v [B,T,H,dv], beta [B,T,H]")
+    for name, t in (("k", k), ("v", v), ("alpha", alpha), ("beta", beta), ("initial_state", initial_state),
+                    ("out", out), ("final_state", final_state)):
+        if t is not None and t.device.type != "cpu":
+            raise ValueError(f"{name} must be a host tensor like q")
+    if out is not None and tuple(out.shape) != (B, T, H, dv):
+        raise ValueError("out must be [B,T,H,dv]")
+    dev = torch.device("cuda", torch.cuda.current_device())
     if out is None:
         out = torch.empty((B, T, H, dv), dtype=out_dtype, pin_memory=True)
-    if tuple(out.shape) != (B, T, H, dv) or out.device.type != "cpu":
-        raise ValueError("out must be a host tensor [B,T,H,dv]")
     keep = []   # device tensors that must outlive the streams' work
     with torch.cuda.device(dev):
         compute = torch.cuda.current_stream(dev)
