@@ -93,3 +93,79 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(kda, "_lib", None)
     with pytest.raises(RuntimeError, match="not built"):
         kda.library()
+
+
+# ---- the further entry points: host-side rejections (nothing reaches the device) ----------
+
+def test_gdn2_rejects_bad_arguments(lib):
+    def g(q=0x10000, e=0x70000, w=0x80000, o=0x60000, dk=16, ws=0x90000):
+        return lib.kda_forward_gdn2(q, 0x20000, 0x30000, 0x40000, e, w, None, o, None, 1, 4, 1, dk, 16, 1.0,
+                                    0, 0, 0, ws, 16, None)
+    assert g(q=None) == ERR_NULL
+    assert g(w=None) == ERR_NULL
+    assert g(e=0x70004) == ERR_ALIGN
+    assert g(o=0x80000 + 64) == ERR_ALIAS                   # o overlaps the write gate
+    assert g(dk=48) == ERR_UNSUP
+    assert g(ws=None) == ERR_WS
+    d = lib.kda_decode_step_gdn2
+    assert d(0x10000, 0x20000, 0x30000, 0x40000, 0x70000, None, 0xA0000, 0x60000, 2, 1, 16, 16, 1.0,
+             0, 0, 0, None) == ERR_NULL
+
+
+def test_raw_and_scalar_gate_reject_bad_arguments(lib):
+    r = lib.kda_forward_raw
+    assert r(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, None, 0x60000, None, 1, 4, 1, 48, 16, 1.0,
+             0, 0, 0, 0x90000, 16, None) == ERR_UNSUP
+    assert r(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, None, 0x60000, None, 1, 4, 1, 16, 16, 1.0,
+             0, 0, 0, None, 0, None) == ERR_WS
+    s = lib.kda_forward_scalar_gate
+    # a per-head gate needs only its element alignment: fp32 at a 2-byte offset is rejected
+    assert s(0x10000, 0x20000, 0x30000, 0x40002, 0x50000, None, 0x60000, None, 1, 4, 1, 16, 16, 1.0,
+             0, 0, 0, 0x90000, 16, None) == ERR_ALIGN
+    assert lib.kda_decode_step_raw(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, None, 0x60000, 2, 1, 16, 16,
+                                   1.0, 0, 0, 0, None) == ERR_NULL
+
+
+def test_varlen_rejects_bad_arguments(lib):
+    def v(N=2, cu=0xB0000, T=8, dk=16):
+        return lib.kda_forward_varlen(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, cu, None, 0x60000, None,
+                                      N, T, 1, dk, 16, 1.0, 0, 0, 0, 0x90000, 16, None)
+    assert v(N=-1) == ERR_SHAPE
+    assert v(cu=None) == ERR_NULL
+    assert v(cu=0xB0002) == ERR_ALIGN
+    assert v(dk=48) == ERR_UNSUP
+
+
+def test_decode_tokens_rejects_bad_arguments(lib):
+    def d(state=0xA0000, slots=None, num_slots=4, o=0x60000, N=2, T=3, status=None, dk=16):
+        return lib.kda_decode_tokens(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, state, slots, num_slots, 1,
+                                     None, o, N, T, 1, dk, 16, 1.0, 0, 0, 0, status, None)
+    assert d(num_slots=1) == ERR_SHAPE                      # identity slots need num_slots >= N
+    assert d(num_slots=-1, slots=0xC0000) == ERR_SHAPE
+    assert d(state=0xA0004) == ERR_ALIGN
+    assert d(slots=0xC0002) == ERR_ALIGN
+    assert d(status=0x90004) == ERR_ALIGN
+    assert d(state=None) == ERR_NULL
+    assert d(o=0xA0000 + 256) == ERR_ALIAS                  # o inside the state pool
+    assert d(dk=48) == ERR_UNSUP
+    assert d(N=0) == OK                                     # nothing to do, nothing launched
+
+
+def test_state_copy_rejects_bad_arguments(lib):
+    def c(src=0x10000, si=None, ss=4, dst=0x80000, di=None, ds=4, count=2, H=1, dk=16, status=None):
+        return lib.kda_state_copy(src, si, ss, dst, di, ds, count, H, dk, 16, status, None)
+    assert c(count=-1) == ERR_SHAPE
+    assert c(dk=48) == ERR_UNSUP
+    assert c(count=5) == ERR_SHAPE                          # identity index past the source pool
+    assert c(count=5, si=0xC0000, ds=4) == ERR_SHAPE        # identity index past the destination pool
+    assert c(src=0x10008) == ERR_ALIGN
+    assert c(si=0xC0002) == ERR_ALIGN
+    assert c(src=None) == ERR_NULL
+    assert c(count=0) == OK and c(H=0) == OK                # nothing to copy, nothing launched
+
+
+def test_selftest_rejects_bad_arguments(lib):
+    assert lib.kda_selftest_bounded_wait(0, 1000, None, None) == ERR_NULL
+    assert lib.kda_selftest_bounded_wait(0, 1000, 0x90004, None) == ERR_ALIGN
+    assert lib.kda_selftest_bounded_wait(0, 0, 0x90000, None) == ERR_SHAPE
+    assert lib.kda_selftest_bounded_wait(0, 2000001, 0x90000, None) == ERR_SHAPE
