@@ -17,7 +17,8 @@ prefix) and ``state_copy`` the whole-state copy between slot pools, the two
 serving operations of "Module 03 -- KDA I", section 5 "State vs. checkpoint
 weights".  ``chunked.forward_chunked`` (numpy, fp64) is the second schedule of "Kimi Delta
 Attention (KDA)", "Two schedules for the same recurrence"; the tests pin it to
-the sequential loop.
+the sequential loop; ``chunked.forward_chunked_gdn2`` is the same schedule for
+GDN-2, pinned the same way.
 
 Every function here is pinned by ``tests/test_oracle_pins.py`` against values
 and identities the pages fix; no part is "parity unpinned".

@@ -76,3 +76,45 @@ def forward_chunked(q, k, v, alpha, beta, s0=None, scale=None, chunk=64):
                                                     alpha[b, :, h], beta[b, :, h], S,
                                                     scale, chunk)
     return o, s_final
+
+
+def _chunk_head_gdn2(q, k, v, a, er, wr, S, scale, C):
+    """GDN-2 in the same chunked form: with the erase gate b and write gate w in place of
+    beta, the in-chunk system is (I + R) E = w*V - ((g*b*K) S) with
+    R_ij = sum_d b_id k_id G[i,j,d] k_jd (j < i), and the outputs and the next state are
+    formed as for KDA ("From Fast Weight Programmers to KDA", section "Gated DeltaNet-2":
+    retrieve through b*k, write w*v minus the retrieval at k)."""
+    T = q.shape[0]
+    o = np.zeros((T, v.shape[1]))
+    for c0 in range(0, T, C):
+        sl = slice(c0, min(c0 + C, T))
+        qc, kc, vc, ac, bc, wc = q[sl], k[sl], v[sl], a[sl], er[sl], wr[sl]
+        L = qc.shape[0]
+        g = np.cumprod(ac, axis=0)
+        G = _pairwise_decay(ac)
+        ebar = wc * vc - (g * bc * kc) @ S
+        R = np.tril(np.einsum("id,ijd,jd->ij", bc * kc, G, kc), -1)
+        E = np.zeros((L, vc.shape[1]))
+        for i in range(L):
+            E[i] = ebar[i] - R[i, :i] @ E[:i]
+        chi = np.tril(np.einsum("id,ijd,jd->ij", qc, G, kc))
+        o[sl] = scale * ((g * qc) @ S + chi @ E)
+        S = g[-1][:, None] * S + (G[L - 1] * kc).T @ E
+    return o, S
+
+
+def forward_chunked_gdn2(q, k, v, alpha, erase, write, s0=None, scale=None, chunk=64):
+    """Chunkwise fp64 GDN-2 with the arguments and layouts of ``oracle.forward_gdn2``."""
+    q, k, v, alpha, erase, write = (np.asarray(x, dtype=np.float64) for x in (q, k, v, alpha, erase, write))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if scale is None:
+        scale = dk ** -0.5
+    o = np.zeros((B, T, H, dv))
+    s_final = np.zeros((B, H, dk, dv))
+    for b in range(B):
+        for h in range(H):
+            S = np.zeros((dk, dv)) if s0 is None else np.array(s0[b, h], dtype=np.float64)
+            o[b, :, h], s_final[b, h] = _chunk_head_gdn2(q[b, :, h], k[b, :, h], v[b, :, h], alpha[b, :, h],
+                                                         erase[b, :, h], write[b, :, h], S, scale, chunk)
+    return o, s_final

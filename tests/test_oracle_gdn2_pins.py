@@ -82,3 +82,14 @@ def test_gdn2_decoupled_gates_matter():
     o1, _ = oracle.forward_gdn2(q, k, v, a, np.full_like(k, 0.9), np.full_like(v, 0.1), s0=s0)
     o2, _ = oracle.forward_gdn2(q, k, v, a, np.full_like(k, 0.5), np.full_like(v, 0.5), s0=s0)
     assert np.abs(o1 - o2).max() > 1e-3
+
+
+@pytest.mark.parametrize("T,chunk", [(37, 8), (64, 32), (5, 16)])
+def test_gdn2_chunked_schedule_matches_sequential(T, chunk):
+    # the chunked form the CUDA-core kernel follows reaches the sequential recurrence
+    from oracle.chunked import forward_chunked_gdn2
+    q, k, v, a, s0, r = _rand(2, T, 2, 8, 6, 6)
+    b, w = r.uniform(0, 1, (2, T, 2, 8)), r.uniform(0, 1, (2, T, 2, 6))
+    o1, s1 = oracle.forward_gdn2(q, k, v, a, b, w, s0=s0)
+    o2, s2 = forward_chunked_gdn2(q, k, v, a, b, w, s0=s0, chunk=chunk)
+    assert np.allclose(o1, o2, rtol=0, atol=1e-12) and np.allclose(s1, s2, rtol=0, atol=1e-12)
