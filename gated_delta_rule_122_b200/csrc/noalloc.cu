@@ -17,7 +17,10 @@
 //  * The first call on a device looks up the array's device address with
 //    cudaGetSymbolAddress (a one-time set-up per device, made with that device
 //    current).  Make that first call before any stream capture begins.
-//  * The status the kernel records here is not readable through the C ABI.
+//  * The status word the kernel records in that array (a bounded wait that gave
+//    up, invalid offsets) is read back with kda_noalloc_status(), which reads
+//    the same array: call it after the call it should report on and before the
+//    next kda_forward_noalloc on that device, since each call clears it.
 #include <mutex>
 
 #include "common.cuh"
@@ -69,4 +72,11 @@ extern "C" kda_status kda_forward_noalloc(const void *q, const void *k, const vo
     if (!scratch) return KDA_ERR_LAUNCH;
     return kda_forward(q, k, v, alpha, beta, initial_state, o, final_state, B, T, H, d_k, d_v, scale,
                        qkv_dtype, gate_dtype, out_dtype, scratch, kKdaNoAllocScratchBytes, stream);
+}
+
+extern "C" kda_status kda_noalloc_status(cudaStream_t stream)
+{
+    void *scratch = scratch_for_current_device();
+    if (!scratch) return KDA_ERR_LAUNCH;
+    return kda_workspace_status(scratch, stream);
 }
