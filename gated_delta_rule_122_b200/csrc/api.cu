@@ -10,7 +10,7 @@ namespace {
 
 constexpr size_t kKdaWorkspaceBytes = 16;   // device status word (+ padding)
 
-bool head_size_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool head_size_ok(int d) { return d >= 16 && d <= 128 && d % 16 == 0; }
 bool dtype_ok(kda_dtype t) { return t == KDA_F32 || t == KDA_BF16; }
 size_t dsize(kda_dtype t) { return t == KDA_BF16 ? 2 : 4; }
 bool aligned16(const void *p) { return p == nullptr || ((uintptr_t)p & 15u) == 0; }
@@ -81,7 +81,7 @@ const char *kda_status_string(kda_status s)
     case KDA_ERR_SHAPE: return "a size is negative or too large";
     case KDA_ERR_DTYPE: return "unknown dtype code";
     case KDA_ERR_ALIGN: return "a pointer is not 16-byte aligned";
-    case KDA_ERR_UNSUPPORTED: return "head size must be 16, 32, 64 or 128";
+    case KDA_ERR_UNSUPPORTED: return "head size must be a multiple of 16 from 16 to 128";
     case KDA_ERR_WORKSPACE: return "workspace missing or too small";
     case KDA_ERR_LAUNCH: return "CUDA launch failed";
     case KDA_ERR_TIMEOUT: return "a bounded device-side wait timed out";

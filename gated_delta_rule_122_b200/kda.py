@@ -27,7 +27,7 @@ _lib = None
 _lock = threading.Lock()
 
 EXPORTED_SYMBOLS = ("kda_forward", "kda_forward_workspace_bytes", "kda_workspace_status",
-                    "kda_forward_noalloc", "kda_forward_varlen", "kda_forward_scalar_gate",
+                    "kda_forward_noalloc", "kda_noalloc_status", "kda_forward_varlen", "kda_forward_scalar_gate",
                     "kda_forward_gdn2", "kda_forward_raw", "kda_forward_sequential", "kda_decode_step",
                     "kda_decode_step_gdn2", "kda_decode_step_raw", "kda_decode_step_scalar_gate",
                     "kda_decode_tokens", "kda_state_copy", "kda_selftest_bounded_wait", "kda_status_string",
@@ -67,6 +67,8 @@ def library() -> ctypes.CDLL:
             lib.kda_forward_sequential.restype = _i
             lib.kda_forward_noalloc.argtypes = fwd_args + [_vp]
             lib.kda_forward_noalloc.restype = _i
+            lib.kda_noalloc_status.argtypes = [_vp]
+            lib.kda_noalloc_status.restype = _i
             lib.kda_forward_varlen.argtypes = [_vp] * 9 + [_i] * 5 + [_f] + [_i] * 3 + \
                 [_vp, ctypes.c_size_t, _vp]
             lib.kda_forward_varlen.restype = _i

@@ -26,7 +26,8 @@
  *    is launched; nothing is written then.  Launch failures return
  *    KDA_ERR_LAUNCH.  Calls are asynchronous on `stream` (0 = legacy default
  *    stream); no call synchronizes.  No exception crosses the ABI.
- *  - Supported head sizes: d_k, d_v in {16, 32, 64, 128}; otherwise
+ *  - Supported head sizes: d_k, d_v in {16, 32, 48, 64, 80, 96, 112, 128}
+ *    (every multiple of 16 up to 128), in any combination; otherwise
  *    KDA_ERR_UNSUPPORTED.
  *  - alpha is the linear retention factor in (0, 1] (alpha = 0 is accepted and
  *    treated as a retention of e^-80 ~ 1.8e-35); beta is the write strength in
@@ -52,7 +53,7 @@ typedef enum {
     KDA_ERR_SHAPE = 2,       /* a size is negative or a product overflows */
     KDA_ERR_DTYPE = 3,       /* unknown dtype code */
     KDA_ERR_ALIGN = 4,       /* a pointer is not 16-byte aligned */
-    KDA_ERR_UNSUPPORTED = 5, /* head size outside {16, 32, 64, 128} */
+    KDA_ERR_UNSUPPORTED = 5, /* head size not a multiple of 16 in [16, 128] */
     KDA_ERR_WORKSPACE = 6,   /* workspace too small or NULL when required */
     KDA_ERR_LAUNCH = 7,      /* the CUDA launch reported an error */
     KDA_ERR_TIMEOUT = 8,     /* a bounded device-side wait gave up */
@@ -123,7 +124,9 @@ kda_status kda_workspace_status(const void *workspace, cudaStream_t stream);
  * array and clears it at its start, so calls that overlap on the GPU race:
  * serialize them.  The first call on a device looks up the array's address
  * (once per device, with that device current); make it before any stream
- * capture.  The pages have no counterpart of this entry point.
+ * capture.  The kernel's status word (a bounded wait that gave up) lands in that
+ * array, not in a caller's workspace: read it with kda_noalloc_status().  The
+ * pages have no counterpart of this entry point.
  */
 kda_status kda_forward_noalloc(const void *q, const void *k, const void *v,
                                const void *alpha, const void *beta,
@@ -132,6 +135,17 @@ kda_status kda_forward_noalloc(const void *q, const void *k, const void *v,
                                int d_k, int d_v, float scale,
                                kda_dtype qkv_dtype, kda_dtype gate_dtype,
                                kda_dtype out_dtype, cudaStream_t stream);
+
+/*
+ * kda_noalloc_status -- synchronize `stream`, then read the status word that
+ * the last kda_forward_noalloc call on the current device left in the
+ * library's array: KDA_OK, or KDA_ERR_TIMEOUT when one of the kernel's bounded
+ * waits gave up (that call's outputs are then not valid); KDA_ERR_LAUNCH if
+ * the array cannot be reached or the read fails.  Allocates nothing.  Call it
+ * before the next kda_forward_noalloc on the device (each call clears the
+ * word).  Like kda_forward_noalloc, no counterpart on the pages.
+ */
+kda_status kda_noalloc_status(cudaStream_t stream);
 
 /*
  * kda_forward_varlen -- kda_forward over a packed batch of N sequences of

@@ -55,7 +55,8 @@ def _fwd(lib, q=0x10000, k=0x20000, v=0x30000, a=0x40000, b=0x50000, s0=None, o=
 def test_forward_rejects_bad_arguments_before_launch(lib):
     assert _fwd(lib, q=None) == ERR_NULL
     assert _fwd(lib, T=-1) == ERR_SHAPE
-    assert _fwd(lib, dk=48) == ERR_UNSUP
+    assert _fwd(lib, dk=40) == ERR_UNSUP                   # not a multiple of 16
+    assert _fwd(lib, dk=144) == ERR_UNSUP                  # above 128
     assert _fwd(lib, dv=256) == ERR_UNSUP
     assert _fwd(lib, qkv=7) == ERR_DTYPE
     assert _fwd(lib, k=0x20008) == ERR_ALIGN
@@ -65,6 +66,17 @@ def test_forward_rejects_bad_arguments_before_launch(lib):
     assert _fwd(lib, ws=None) == ERR_WS
     assert _fwd(lib, wsb=8) == ERR_WS
     assert _fwd(lib, ws=0x90008) == ERR_ALIGN
+
+
+@pytest.mark.parametrize("d", [16, 32, 48, 64, 80, 96, 112, 128])
+def test_every_multiple_of_16_head_size_is_accepted(lib, d):
+    # B = 0: the checks run, nothing is launched
+    assert _fwd(lib, dk=d, dv=d, B=0) == OK
+    assert _fwd(lib, dk=d, dv=16, B=0) == OK and _fwd(lib, dk=16, dv=d, B=0) == OK
+    assert lib.kda_forward_sequential(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, None, 0x60000, None,
+                                      0, 4, 1, d, d, 1.0, 0, 0, 0, None) == OK
+    assert lib.kda_decode_step(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 0x70000, 0x60000, 0, 2, d, d, 1.0,
+                               0, 0, 0, None) == OK
 
 
 def test_sequential_and_decode_reject_bad_arguments(lib):
@@ -105,7 +117,7 @@ def test_gdn2_rejects_bad_arguments(lib):
     assert g(w=None) == ERR_NULL
     assert g(e=0x70004) == ERR_ALIGN
     assert g(o=0x80000 + 64) == ERR_ALIAS                   # o overlaps the write gate
-    assert g(dk=48) == ERR_UNSUP
+    assert g(dk=40) == ERR_UNSUP
     assert g(ws=None) == ERR_WS
     d = lib.kda_decode_step_gdn2
     assert d(0x10000, 0x20000, 0x30000, 0x40000, 0x70000, None, 0xA0000, 0x60000, 2, 1, 16, 16, 1.0,
@@ -114,7 +126,7 @@ def test_gdn2_rejects_bad_arguments(lib):
 
 def test_raw_and_scalar_gate_reject_bad_arguments(lib):
     r = lib.kda_forward_raw
-    assert r(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, None, 0x60000, None, 1, 4, 1, 48, 16, 1.0,
+    assert r(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, None, 0x60000, None, 1, 4, 1, 56, 16, 1.0,
              0, 0, 0, 0x90000, 16, None) == ERR_UNSUP
     assert r(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, None, 0x60000, None, 1, 4, 1, 16, 16, 1.0,
              0, 0, 0, None, 0, None) == ERR_WS
@@ -133,7 +145,7 @@ def test_varlen_rejects_bad_arguments(lib):
     assert v(N=-1) == ERR_SHAPE
     assert v(cu=None) == ERR_NULL
     assert v(cu=0xB0002) == ERR_ALIGN
-    assert v(dk=48) == ERR_UNSUP
+    assert v(dk=40) == ERR_UNSUP
 
 
 def test_decode_tokens_rejects_bad_arguments(lib):
@@ -147,7 +159,7 @@ def test_decode_tokens_rejects_bad_arguments(lib):
     assert d(status=0x90004) == ERR_ALIGN
     assert d(state=None) == ERR_NULL
     assert d(o=0xA0000 + 256) == ERR_ALIAS                  # o inside the state pool
-    assert d(dk=48) == ERR_UNSUP
+    assert d(dk=40) == ERR_UNSUP
     assert d(N=0) == OK                                     # nothing to do, nothing launched
 
 
@@ -155,7 +167,7 @@ def test_state_copy_rejects_bad_arguments(lib):
     def c(src=0x10000, si=None, ss=4, dst=0x80000, di=None, ds=4, count=2, H=1, dk=16, status=None):
         return lib.kda_state_copy(src, si, ss, dst, di, ds, count, H, dk, 16, status, None)
     assert c(count=-1) == ERR_SHAPE
-    assert c(dk=48) == ERR_UNSUP
+    assert c(dk=40) == ERR_UNSUP
     assert c(count=5) == ERR_SHAPE                          # identity index past the source pool
     assert c(count=5, si=0xC0000, ds=4) == ERR_SHAPE        # identity index past the destination pool
     assert c(src=0x10008) == ERR_ALIGN

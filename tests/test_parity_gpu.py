@@ -134,6 +134,34 @@ def test_prefill_ragged_shapes_fp32(T, dk, dv):
         assert s_err(S, s_ref) < TOL_F32
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dk,dv", [(48, 48), (80, 80), (96, 96), (112, 112), (48, 112), (112, 48), (80, 32)])
+def test_prefill_multiple_of_16_head_sizes(dtype, dk, dv):
+    """Every multiple of 16 up to 128 is a supported head size: both schedules against the
+    oracle, a ragged last chunk and an initial state."""
+    w = WORKLOADS["tiny"].scaled(B=2, H=2, T=77, dk=dk, dv=dv, init_state=True, qkv_dtype=dtype,
+                                 gate_dtype=dtype)
+    x = make_inputs(w)
+    o_ref, s_ref = oracle_full(x)
+    tol = TOL_F32 if dtype == torch.float32 else TOL_BF16
+    for fn in PREFILL_FNS.values():
+        o, S = _run(fn, to_device(x))
+        assert o_err(o, o_ref) < tol
+        assert s_err(S, s_ref) < tol
+
+
+@pytest.mark.parametrize("dk,dv", [(48, 48), (112, 112), (80, 96)])
+def test_decode_multiple_of_16_head_sizes(dk, dv):
+    w = WORKLOADS["decode"].scaled(B=5, H=3, dk=dk, dv=dv)
+    x = make_decode_inputs(w)
+    o_ref, s_ref = oracle.decode_step(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["state"],
+                                      scale=x["scale"])
+    xd = to_device(x)
+    o = kda.decode_step(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta"], xd["state"], scale=x["scale"])
+    assert o_err(o, o_ref) < TOL_BF16
+    assert s_err(xd["state"], s_ref) < TOL_BF16
+
+
 @pytest.mark.parametrize("name", ["tiny", "small"])
 def test_chunked_agrees_with_sequential(name):
     x = to_device(make_inputs(name))
@@ -245,7 +273,7 @@ def test_host_buffers_pipelined_match_device(gate):
 
 
 def test_status_errors_raise():
-    x = to_device(make_inputs(WORKLOADS["tiny"].scaled(T=8, dk=48, dv=16)))
+    x = to_device(make_inputs(WORKLOADS["tiny"].scaled(T=8, dk=40, dv=16)))
     with pytest.raises(kda.KDAError, match="head size"):
         _run(kda.forward, x)
 
