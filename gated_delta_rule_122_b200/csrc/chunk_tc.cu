@@ -65,11 +65,21 @@ constexpr int NPW = 4;           // prep warps (A readout, solve, W' readout)
 constexpr int NPT = NPW * 32;
 constexpr int NT = NCT + NPT + 32;   // + the MMA-issuer warp
 constexpr int kIssuerWarp = NCW + NPW;
+// The chain thread that issues the staging loads, their L2 prefetches and the output
+// stores: lane 0 of the last chain warp, whose SM sub-partition does not also run the
+// MMA-issuer warp (warps are spread over the four sub-partitions by index mod 4).
+constexpr int kTmaThread = NCT - 32;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per bounded wait
 constexpr int kChainBar = 1, kPrepBar = 2;         // named barriers of the two roles
 constexpr int kCstSlots = 4;                       // per-chunk constants kept in flight
 constexpr float kMinAlpha = 1.8048513e-35f;        // e^-80: per-token retention floor
 constexpr float kMinScale = 2.3509887e-38f;        // 2^-125: floor of the anchored decays
+// A chunk in which some key channel decays by more than 2^-100 over one 16-token half
+// (about 69 nats) is outside the range in which the anchored factors e and 1/e, and
+// their products with the operands, are exact in fp32.  Such a chunk is computed token
+// by token instead (the sequential form of the recurrence, fp32, on the chain warps).
+constexpr float kExtremeDecay = 7.8886091e-31f;    // 2^-100
+constexpr float kExtremeInv = 1.2676506e30f;       // 2^100
 
 // ---- operand layouts ----------------------------------------------------------------
 // d-major slab (8 tokens x 128 channels, 2 KB): channel block d/8 at 128 B, channel
@@ -129,7 +139,11 @@ constexpr int NBARS = 7;
 constexpr int OFF_BAR = (OFF_TPU + C * C * 4 + 7) / 8 * 8;
 constexpr int OFF_SIG = OFF_BAR + NBARS * 8;           // 6 readiness counters (8 slots)
 constexpr int OFF_MISC = OFF_SIG + 32;                 // tmem base, error flag
-constexpr int SMEM_BYTES = OFF_MISC + 16;
+// Chunks whose decay leaves the range of the anchored factors: slot n % 4 holds n + 1
+// when chunk n is one (written by stage A, read by the chain warps after a barrier).
+constexpr int kXSlots = 4;
+constexpr int OFF_XF = OFF_MISC + 16;
+constexpr int SMEM_BYTES = OFF_XF + 4 * kXSlots;
 static_assert(SMEM_BYTES <= 232448, "shared memory plan exceeds the per-block limit");
 static_assert(OFF_AKK % 16 == 0 && OFF_LQR % 128 == 0 && OFF_TP % 128 == 0 && OFF_TPU % 128 == 0,
               "vector and operand alignment");
@@ -346,7 +360,7 @@ __device__ void issuer(uint8_t *sm, uint32_t tmem, const Bars &bars, int nchunks
                 return;
             }
         } else {
-            __nanosleep(20);
+            __nanosleep(20);   // polling without a pause slows every warp's shared-memory traffic
         }
     }
 }
@@ -427,6 +441,8 @@ __device__ void stage_a(const ChunkArgs &p, uint8_t *sm, const SeqSpan &sp, int 
             pr[i] = acc;                                     // e_r (raw: 1/e_r)
         }
         cst[D + d] = fmaxf(kRaw ? ptx::rcp(acc) : acc, kMinScale);   // exp(G_end - a)
+        if (kRaw ? !(acc <= kExtremeInv) : !(acc >= kExtremeDecay))
+            reinterpret_cast<volatile int *>(sm + OFF_XF)[n % kXSlots] = n + 1;
     } else {
 #pragma unroll
         for (int i = 15; i >= 0; --i) {
@@ -434,6 +450,8 @@ __device__ void stage_a(const ChunkArgs &p, uint8_t *sm, const SeqSpan &sp, int 
             acc *= (i < Lc) ? factor(i) : 1.f;
         }
         const float aexp = fmaxf(kRaw ? ptx::rcp(acc) : acc, kMinScale);   // exp(a)
+        if (kRaw ? !(acc <= kExtremeInv) : !(acc >= kExtremeDecay))
+            reinterpret_cast<volatile int *>(sm + OFF_XF)[n % kXSlots] = n + 1;
         cst[d] = aexp;
         cst[2 * D + d] = (n > 0) ? aexp * cst_prev[D + d] : 0.f;   // state-update factor
     }
@@ -499,6 +517,17 @@ __device__ __forceinline__ void load_qka(const TcMaps &maps, uint8_t *sm, const 
     if constexpr (kGate == kGateChannel) ptx::tma_load_4d(dst + STG_A, &maps.a, bars.stg, 0, tp.h, tp.t0 + n * C, tp.b);
     // heads h & ~7 .. (h & ~7) + 7 of 32 tokens: the x coordinate is a multiple of 8 elements
     if constexpr (kGate == kGateHeadTma) ptx::tma_load_3d(dst + STG_A, &maps.a, bars.stg, tp.h & ~7, tp.t0 + n * C, tp.b);
+}
+
+// L2 prefetch of chunk n's q, k, alpha rows (one thread), issued a few chunks before the
+// staging load of the same rows so that the load finds them in L2.
+template <int kGate>
+__device__ __forceinline__ void prefetch_qka(const TcMaps &maps, const TmaPos &tp, int n)
+{
+    ptx::tma_prefetch_4d(&maps.q, 0, tp.h, tp.t0 + n * C, tp.b);
+    ptx::tma_prefetch_4d(&maps.k, 0, tp.h, tp.t0 + n * C, tp.b);
+    if constexpr (kGate == kGateChannel) ptx::tma_prefetch_4d(&maps.a, 0, tp.h, tp.t0 + n * C, tp.b);
+    if constexpr (kGate == kGateHeadTma) ptx::tma_prefetch_3d(&maps.a, tp.h & ~7, tp.t0 + n * C, tp.b);
 }
 
 // TMA load of chunk n's v rows into V buffer n&1 (one thread).
@@ -699,12 +728,12 @@ __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, u
 // the fp32 values, write them back, and write the bf16 hi/lo planes of the M3
 // operand (two bf16 per TMEM column).
 __device__ __forceinline__ void write_state16(uint32_t tmem, uint32_t lane_base, int d0, float (&v)[16],
-                                              const float *scale_d)
+                                              const float *scale_d, bool unscaled = false)
 {
     uint32_t fw[16], hw[8], lw[8];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-        v[i] *= scale_d[i];
+        if (!unscaled) v[i] *= scale_d[i];
         fw[i] = __float_as_uint(v[i]);
     }
     ptx::tmem_st16(tmem + lane_base + TM_S + d0, fw);
@@ -772,13 +801,161 @@ __device__ __forceinline__ void chain_stage_b(const TcMaps &maps, uint8_t *sm, c
     ptx::fence_proxy_async_smem();
     warp_signal(bars.rc, lane);
     chain_bar();   // staging consumed, constants visible to every chain warp
-    if (tid == 0 && n + 1 < nchunks) load_qka<kGate>(maps, sm, bars, tp, n + 1);
+    if (tid == kTmaThread && n + 1 < nchunks) load_qka<kGate>(maps, sm, bars, tp, n + 1);
 }
 
 __device__ __forceinline__ void warp_signal_after_stage(const Bars &bars, int lane)
 {
     ptx::fence_proxy_async_smem();
     warp_signal(bars.rc, lane);
+}
+
+__device__ __forceinline__ bool chunk_is_extreme(const uint8_t *sm, int n)
+{
+    return reinterpret_cast<const volatile int *>(sm + OFF_XF)[n % kXSlots] == n + 1;
+}
+
+// Eight consecutive bf16 values (16 bytes) widened to fp32.
+__device__ __forceinline__ void ld_bf16x8(const void *p, float (&x)[8])
+{
+    const uint4 w = *reinterpret_cast<const uint4 *>(p);
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x[2 * i] = __uint_as_float(u[i] << 16);
+        x[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
+    }
+}
+
+// A chunk whose decay leaves the range of the anchored factors, token by token on the
+// chain warps: the five-step update of each token in fp32.  This thread's part of the
+// state, S[64 half + i][j] for i < 64 (key channels 64 half .. 64 half + 63 of value
+// channel j), stays in its TMEM lane at columns TM_S + 64 half + i and is walked in two
+// groups of 32 per pass.  The two predictions S~^T k, S~^T q and k.q are summed over the
+// two halves through shared memory, one barrier per token; o_t = scale (S~^T q + e (k.q))
+// is the read of S_t = S~ + k e^T.  Retention factors are used as they are (alpha = 0
+// clears a channel exactly).  xb: 2 x 2 x 4 x 128 floats of scratch.
+template <int kGate, bool kRaw>
+__device__ __forceinline__ void sequential_chunk(const ChunkArgs &p, const uint8_t *sm, uint32_t tcol,
+                                                 const SeqSpan &sp, int h, int c, int half, int j, float *xb)
+{
+    const int d0 = 64 * half;
+    const int Lc = min(C, sp.len - c * C);
+    const float *nrm = reinterpret_cast<const float *>(sm + OFF_NRM + (c % kNrmSlots) * NRM_BYTES);
+#pragma unroll 1
+    for (int r = 0; r < Lc; ++r) {
+        const size_t row = (sp.tok0 + (size_t)c * C + r) * p.H + h;
+        const __nv_bfloat16 *qr = (const __nv_bfloat16 *)p.q + row * D + d0;
+        const __nv_bfloat16 *kr = (const __nv_bfloat16 *)p.k + row * D + d0;
+        const __nv_bfloat16 *ar = (const __nv_bfloat16 *)p.alpha + row * D + d0;
+        float ah = 1.f;   // one gate per (token, head)
+        if constexpr (kGate != kGateChannel) ah = __bfloat162float(((const __nv_bfloat16 *)p.alpha)[row]);
+        float pv = 0.f, pq = 0.f, kq = 0.f;
+#pragma unroll 1
+        for (int q2 = 0; q2 < 2; ++q2) {
+            float sv[32];
+            ptx::tmem_ld32(tcol + 32 * q2, sv);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                float qv[8], kv[8], av[8];
+                ld_bf16x8(qr + 32 * q2 + 8 * g, qv);
+                ld_bf16x8(kr + 32 * q2 + 8 * g, kv);
+                if constexpr (kGate == kGateChannel) ld_bf16x8(ar + 32 * q2 + 8 * g, av);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    float al = (kGate == kGateChannel) ? av[i] : ah;
+                    if constexpr (kRaw) al = 1.f / (1.f + __expf(al));   // gate logit x: alpha = 1/(1 + e^x)
+                    float &x = sv[8 * g + i];
+                    x *= al;
+                    pv = fmaf(kv[i], x, pv);
+                    pq = fmaf(qv[i], x, pq);
+                    kq = fmaf(kv[i], qv[i], kq);
+                }
+            }
+            ptx::tmem_st32(tcol + 32 * q2, sv);
+        }
+        ptx::tmem_wait_st();
+        float *mine = xb + ((r & 1) * 2 + half) * 4 * D;
+        const float *other = xb + ((r & 1) * 2 + (1 - half)) * 4 * D;
+        mine[j] = pv;
+        mine[D + j] = pq;
+        mine[2 * D + j] = kq;
+        chain_bar();
+        const float nk = kRaw ? nrm[C + r] : 1.f, nq = kRaw ? nrm[r] : 1.f;
+        const float vh = (pv + other[j]) * nk;                  // S~^T k (unit key)
+        const float ph = (pq + other[D + j]) * nq;              // S~^T q (unit query)
+        const float kqs = (kq + other[2 * D + j]) * nk * nq;    // k . q
+        const float beta = load_beta<kRaw>(p, sp, h, c, r);
+        const float vj = __bfloat162float(((const __nv_bfloat16 *)p.v)[row * D + j]);
+        const float e = beta * (vj - vh);
+        if (half == 0) st_elem(p.o, row * D + j, p.scale * fmaf(e, kqs, ph), p.out_bf16);
+        const float ek = e * nk;
+#pragma unroll 1
+        for (int q2 = 0; q2 < 2; ++q2) {
+            float sv[32];
+            ptx::tmem_ld32(tcol + 32 * q2, sv);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                float kv[8];
+                ld_bf16x8(kr + 32 * q2 + 8 * g, kv);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) sv[8 * g + i] = fmaf(kv[i], ek, sv[8 * g + i]);
+            }
+            ptx::tmem_st32(tcol + 32 * q2, sv);
+        }
+        ptx::tmem_wait_st();
+    }
+}
+
+// Chain warps, a chunk that runs token by token (after its M3/M4 groups have completed;
+// the E phase saved the chunk's initial state in the S' plane columns): put the state
+// back into the fp32 state columns, run the tokens there, then write S'_{c+1}
+// (unscaled when chunk c+1 also runs token by token) with its bf16 planes and clear the
+// O accumulator, or store the final state.
+template <int kGate, bool kRaw>
+__device__ __forceinline__ void extreme_chunk(const ChunkArgs &p, uint8_t *sm, uint32_t tmem, uint32_t lane_base,
+                                              const SeqSpan &sp, int h, int c, int half, int j, size_t tile,
+                                              int nchunks, bool xn)
+{
+    const uint32_t tcol = tmem + lane_base + TM_S + 64 * half;
+#pragma unroll 1
+    for (int q2 = 0; q2 < 2; ++q2) {
+        float v[32];
+        ptx::tmem_ld32(tmem + lane_base + TM_SP + 64 * half + 32 * q2, v);
+        ptx::tmem_wait_ld();
+        ptx::tmem_st32(tcol + 32 * q2, v);
+    }
+    ptx::tmem_wait_st();
+    // E^T is free until chunk c+1's readout: scratch for the two halves' sums.  The
+    // barrier of the first token also orders every thread's read of the saved state
+    // before the plane writes below.
+    sequential_chunk<kGate, kRaw>(p, sm, tcol, sp, h, c, half, j, reinterpret_cast<float *>(sm + OFF_ET));
+    if (c + 1 < nchunks) {
+        const float *an = reinterpret_cast<const float *>(sm + OFF_CST + ((c + 1) % kCstSlots) * CST_BYTES);
+        ptx::tmem_st16_zero(tmem + lane_base + TM_O + 32 * half);
+        ptx::tmem_st16_zero(tmem + lane_base + TM_O + 32 * half + 16);
+#pragma unroll 1
+        for (int part = 0; part < 4; ++part) {
+            const int d0 = 64 * half + 16 * part;
+            float v[16];
+            ptx::tmem_ld16(tmem + lane_base + TM_S + d0, v);
+            ptx::tmem_wait_ld();
+            write_state16(tmem, lane_base, d0, v, an + d0, xn);
+        }
+        ptx::tmem_wait_st();
+    } else if (p.s_out) {
+#pragma unroll 1
+        for (int part = 0; part < 4; ++part) {
+            const int d0 = 64 * half + 16 * part;
+            float v[16];
+            ptx::tmem_ld16(tmem + lane_base + TM_S + d0, v);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) p.s_out[tile + (size_t)(d0 + i) * D + j] = v[i];
+        }
+    }
 }
 
 // ---- the chain warps: the serial recurrence over chunks --------------------------------
@@ -794,22 +971,26 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
     const size_t tile = (size_t)bh * D * D;
 
     uint32_t ie[16];   // R of the chunk being staged (split words), carried from part A to part B
-    if (tid == 0) load_qka<kGate>(maps, sm, bars, tp, 0);
+    if (tid == kTmaThread) {
+        load_qka<kGate>(maps, sm, bars, tp, 0);
+        for (int n = 1; n < 4 && n < nchunks; ++n) prefetch_qka<kGate>(maps, tp, n);
+    }
     int staged = 0;   // chunks whose rows have been waited for
     chain_stage_a<kGate, kRaw>(p, sm, bars, sp, h, 0, warp, lane, ie, err_flag);
     staged = 1;
     chain_stage_b<kGate>(maps, sm, bars, tp, 0, nchunks, tid, warp, lane, ie);
 
-    // S'_0 = Diag(exp(a_0)) S_0; cleared O accumulator
+    // S'_0 = Diag(exp(a_0)) S_0 (S_0 itself when chunk 0 runs token by token); cleared O
     {
         const float *cst0 = reinterpret_cast<const float *>(sm + OFF_CST);
+        const bool x0 = chunk_is_extreme(sm, 0);
 #pragma unroll 1
         for (int part = 0; part < 4; ++part) {
             const int d0 = 64 * half + 16 * part;
             float v[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) v[i] = p.s_in ? p.s_in[tile + (size_t)(d0 + i) * D + j] : 0.f;
-            write_state16(tmem, lane_base, d0, v, cst0 + d0);
+            write_state16(tmem, lane_base, d0, v, cst0 + d0, x0);
         }
         ptx::tmem_st16_zero(tmem + lane_base + TM_O + 32 * half);
         ptx::tmem_st16_zero(tmem + lane_base + TM_O + 32 * half + 16);
@@ -824,10 +1005,26 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
     }
 
     for (int c = 0; c < nchunks; ++c) {
+        // the rows of chunk c+4 into L2: their staging load (issued at the end of
+        // iteration c+1) then does not wait for HBM
+        if (tid == kTmaThread && c + 4 < nchunks) prefetch_qka<kGate>(maps, tp, c + 4);
         // ---- E: E^T = U^T - S'^T W'^T (hi and lo column groups) into the A operand of M4
         if (!ptx::mbar_wait(bars.e, (uint32_t)(c & 1), kWaitLimitNs)) *err_flag = 1;
         ptx::tc_fence_after();
-        {
+        const bool xc = chunk_is_extreme(sm, c);
+        if (xc) {
+            // the chunk runs token by token: keep its initial state (unscaled, written so by
+            // the previous chunk's rewrite) in the S' plane columns, which M3 has finished
+            // reading; the state update of M4 then changes nothing that is used
+#pragma unroll 1
+            for (int q2 = 0; q2 < 2; ++q2) {
+                float v[32];
+                ptx::tmem_ld32(tmem + lane_base + TM_S + 64 * half + 32 * q2, v);
+                ptx::tmem_wait_ld();
+                ptx::tmem_st32(tmem + lane_base + TM_SP + 64 * half + 32 * q2, v);
+            }
+            ptx::tmem_wait_st();
+        } else {
             // token blocks 2 half and 2 half + 1, each as [hi 8 | lo 8] columns
             float v0[16], v1[16];
             ptx::tmem_ld16(tmem + lane_base + TM_E + 32 * half, v0);
@@ -868,6 +1065,23 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
             stage_b(sm, c + 2, warp, lane, ie);
             warp_signal_after_stage(bars, lane);
         }
+        const bool xn = c + 1 < nchunks && chunk_is_extreme(sm, c + 1);
+        if (xc) {
+            // outputs stored token by token; the staging rows (read by every warp's stage A
+            // above, and by the previous chunk's output store) are then free for chunk c+3
+            extreme_chunk<kGate, kRaw>(p, sm, tmem, lane_base, sp, h, c, half, j, tile, nchunks, xn);
+            if (c + 1 < nchunks) {
+                ptx::tc_fence_before();
+                warp_signal(bars.rs, lane);
+            }
+            const bool stop = chain_bar_err(err_flag);
+            if (tid == kTmaThread && c + 3 < nchunks) {
+                ptx::bulk_wait_read();
+                load_qka<kGate>(maps, sm, bars, tp, c + 3);
+            }
+            if (stop) break;
+            continue;
+        }
         float ov[16];
         {
             float v0[16], v1[16];
@@ -886,8 +1100,10 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
             }
         }
         if (c + 1 < nchunks) {
-            // f(c+1) = exp(a_{c+1}) exp(G_end,c - a_c), written when chunk c+1 was staged
-            const float *f = reinterpret_cast<const float *>(sm + OFF_CST + ((c + 1) % kCstSlots) * CST_BYTES) + 2 * D;
+            // f(c+1) = exp(a_{c+1}) exp(G_end,c - a_c), written when chunk c+1 was staged; when
+            // chunk c+1 runs token by token its initial state is kept unscaled: exp(G_end,c - a_c)
+            const float *f = xn ? reinterpret_cast<const float *>(sm + OFF_CST + (c % kCstSlots) * CST_BYTES) + D
+                                : reinterpret_cast<const float *>(sm + OFF_CST + ((c + 1) % kCstSlots) * CST_BYTES) + 2 * D;
             ptx::tmem_st16_zero(tmem + lane_base + TM_O + 32 * half);
             ptx::tmem_st16_zero(tmem + lane_base + TM_O + 32 * half + 16);
 #pragma unroll 1
@@ -934,32 +1150,32 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
         // barrier.  The previous chunk's output store must also have read the rows: a
         // staging fill orders that (thread 0 issues it after the read); without one,
         // thread 0 waits for the read here, before the barrier.
-        if (c > 0 && c + 2 >= nchunks && tid == 0) ptx::bulk_wait_read();
+        if (c > 0 && c + 2 >= nchunks && tid == kTmaThread) ptx::bulk_wait_read();
         chain_bar();
         const bool full = (c + 1) * C <= sp.len;
         if (full) {
             const int esz = p.out_bf16 ? 2 : 4;
-            uint8_t *tile = sm + OFF_STG + (half ? STG_A : STG_Q) + j * esz;
+            uint8_t *otile = sm + OFF_STG + (half ? STG_A : STG_Q) + j * esz;
             if (p.out_bf16) {
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
-                    *reinterpret_cast<__nv_bfloat16 *>(tile + i * D * 2) = __float2bfloat16_rn(ov[i]);
+                    *reinterpret_cast<__nv_bfloat16 *>(otile + i * D * 2) = __float2bfloat16_rn(ov[i]);
             } else {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) *reinterpret_cast<float *>(tile + i * D * 4) = ov[i];
+                for (int i = 0; i < 16; ++i) *reinterpret_cast<float *>(otile + i * D * 4) = ov[i];
             }
         } else {
             // the sequence's last, partial chunk: only its own rows, one element per row
             // (a TMA box would also cover rows that belong to the next sequence)
             const size_t step = (size_t)p.H * D;
-            size_t idx = ((sp.tok0 + c * C + 16 * half) * p.H + h) * D + j;
+            size_t idx = ((sp.tok0 + (size_t)c * C + 16 * half) * p.H + h) * D + j;
 #pragma unroll
             for (int i = 0; i < 16; ++i, idx += step)
                 if (c * C + 16 * half + i < sp.len) st_elem(p.o, idx, ov[i], p.out_bf16);
         }
         ptx::fence_proxy_async_smem();
         const bool stop = chain_bar_err(err_flag);   // output tile written, staging rows consumed
-        if (tid == 0) {
+        if (tid == kTmaThread) {
             if (full) {
                 ptx::tma_store_4d(&maps.o, ptx::smem_u32(sm + OFF_STG + STG_Q), 0, h, tp.t0 + c * C, tp.b);
                 ptx::tma_store_4d(&maps.o, ptx::smem_u32(sm + OFF_STG + STG_A), 0, h, tp.t0 + c * C + 16, tp.b);
@@ -975,7 +1191,7 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
     // on an early exit, let a staging load still in flight land before the block ends
     if (staged < nchunks && staged > 0)
         (void)ptx::mbar_wait(bars.stg, (uint32_t)(staged & 1), kWaitLimitNs);
-    if (tid == 0) ptx::bulk_wait();   // the output stores are complete
+    if (tid == kTmaThread) ptx::bulk_wait();   // the output stores are complete
 }
 
 // kGate: alpha per key channel [B, T, H, d_k], or one retention factor per (token, head),
@@ -1028,6 +1244,8 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs pa, const
         ptx::fence_mbar_init();
 #pragma unroll
         for (int i = 0; i < 8; ++i) reinterpret_cast<uint32_t *>(sm + OFF_SIG)[i] = 0u;
+#pragma unroll
+        for (int i = 0; i < kXSlots; ++i) reinterpret_cast<int *>(sm + OFF_XF)[i] = 0;
         *err_flag = 0;
     }
     if (warp == 0) {

@@ -137,6 +137,23 @@ __device__ __forceinline__ void tma_load_5d(uint32_t dst, const void *tmap, uint
         : "memory");
 }
 
+// Prefetch the box at the given coordinates into L2 (no shared-memory destination, no
+// completion to wait for), so that a later load of the same box hits L2.
+__device__ __forceinline__ void tma_prefetch_3d(const void *tmap, int c0, int c1, int c2)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_4d(const void *tmap, int c0, int c1, int c2, int c3)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
+}
+
 // TMA tiled store of a box from shared memory (bulk-group completion).  The
 // box must start at a non-negative coordinate; rows past the tensor's end are
 // not written.
