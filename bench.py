@@ -67,6 +67,7 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true", help="skip the per-entry-point measurements")
+    ap.add_argument("--no-long", action="store_true", help="skip the long-prefill measurement")
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="run one kernel per step (for profiling); the JSON line is then partial")
     ap.add_argument("--prefill-seqs", type=int, default=None,
@@ -120,6 +121,28 @@ def time_call(torch, fn, reps=5, warmup=2):
     return e0.elapsed_time(e1) / reps
 
 
+def measure_long(torch, kda, device, hbm):
+    """The long prefill workload (B=1 H=64 T=65536 d=128, bf16 inputs, random initial
+    state, 30% strong-forget channels), device-timed with CUDA events on its own, with its
+    roofline against its algorithmic bytes (inputs, initial and final state, o)."""
+    from gated_delta_rule_122_b200.inputs import make_inputs, workload
+    w = workload("long")
+    xl = make_inputs(w, device=device)
+    ol = torch.empty((w.B, w.T, w.H, w.dv), device=device)
+    Sl = torch.empty((w.B, w.H, w.dk, w.dv), device=device)
+    fn = lambda: kda.forward(xl["q"], xl["k"], xl["v"], xl["alpha"], xl["beta"], initial_state=xl["s0"],
+                             scale=xl["scale"], out=ol, final_state=Sl)
+    ms = time_call(torch, fn, reps=5, warmup=2)
+    nbytes = prefill_bytes(w, True)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    del xl, ol, Sl
+    return {"workload": f"long prefill B={w.B} H={w.H} T={w.T} d_k=d_v={w.dk} bf16 q/k/v/alpha/beta, random "
+                        "initial state, 30% strong-forget channels", "ms": ms,
+            "mtokens_s": w.B * w.T / (ms * 1e-3) / 1e6,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "algorithmic_bytes": nbytes}}
+
+
 def measure_rows(torch, kda, x, y, wp, hbm):
     """Each further entry point once, at the scale of the prefill and decode workloads.
     Returns {row: {workload, ms, throughput, algorithmic bytes, fraction of hbm}}."""
@@ -137,6 +160,15 @@ def measure_rows(torch, kda, x, y, wp, hbm):
             r["mtokens_s"] = tokens / (ms * 1e-3) / 1e6
         rows[name] = r
 
+    # the small workload (B=1 H=4 T=2048 d=64, bf16 q/k/v, fp32 alpha/beta, random initial state)
+    from gated_delta_rule_122_b200.inputs import make_inputs, workload
+    ws_ = workload("small")
+    xs = make_inputs(ws_, device=dev)
+    ms = time_call(torch, lambda: kda.forward(xs["q"], xs["k"], xs["v"], xs["alpha"], xs["beta"],
+                                              initial_state=xs["s0"], scale=xs["scale"]))
+    row("small_prefill", f"B={ws_.B} T={ws_.T} H={ws_.H} d={ws_.dk}, bf16 q/k/v, fp32 alpha/beta, initial state",
+        ms, prefill_bytes(ws_, True), ws_.B * ws_.T)
+    del xs
     o = torch.empty((B, T, H, dv), device=dev)
     S = torch.empty((B, H, dk, dv), device=dev)
     # scalar gate: one retention factor per (token, head)
@@ -451,28 +483,47 @@ def main():
 
     e2e = None
     if not args.no_e2e:
+        # the whole step through the host-buffer C entry points: the prefill's inputs come
+        # from pinned host memory and its o and final state go back (kda_forward_host), and
+        # the decode step's token vectors come in and its o goes back with the state
+        # resident on the device (kda_decode_step_host)
         hx = {n: x[n].cpu().pin_memory() for n in ("q", "k", "v", "alpha", "beta")}
         ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
         hS = torch.empty(S.shape, dtype=S.dtype, pin_memory=True)
+        hy = {n: y[n].cpu().pin_memory() for n in ("q", "k", "v", "alpha", "beta")} if y is not None else None
+        hod = torch.empty(od.shape, dtype=od.dtype, pin_memory=True)
         h2d = sum(t.numel() * t.element_size() for t in hx.values())
         d2h = ho.numel() * ho.element_size() + hS.numel() * hS.element_size()
+        if hy is not None:
+            h2d += sum(t.numel() * t.element_size() for t in hy.values())
+            d2h += hod.numel() * hod.element_size()
+
+        def host_step():
+            kda.forward(hx["q"], hx["k"], hx["v"], hx["alpha"], hx["beta"], scale=x["scale"],
+                        out=ho, final_state=hS)
+            if hy is not None:
+                kda.decode_step(hy["q"], hy["k"], hy["v"], hy["alpha"], hy["beta"], y["state"],
+                                scale=y["scale"], out=hod)
+
         n_e2e = max(3, K // 4)
-        kda.forward(hx["q"], hx["k"], hx["v"], hx["alpha"], hx["beta"], scale=x["scale"],
-                    out=ho, final_state=hS)   # warm-up of the host path
+        host_step()   # warm-up of the host path
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier(pg)
         torch.cuda.synchronize()
         e0.record()
         for _ in range(n_e2e):
-            kda.forward(hx["q"], hx["k"], hx["v"], hx["alpha"], hx["beta"], scale=x["scale"],
-                        out=ho, final_state=hS)
+            host_step()
         e1.record()
         torch.cuda.synchronize()
         e2e_ms = reduce_max(pg, [e0.elapsed_time(e1) / n_e2e], device)[0]
         e2e = {"value": world * tokens / (e2e_ms * 1e-3) / 1e6, "unit": "Mtokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-               "steps": n_e2e}
+               "steps": n_e2e, "path": "kda_forward_host + kda_decode_step_host (C ABI, host buffers)"}
 
+    long_leg = None
+    if world == 1 and not args.no_long and args.only is None and args.prefill_seqs is None \
+            and args.prefill_len is None:
+        long_leg = measure_long(torch, kda, device, hbm)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_prefill(x, wp)
@@ -506,6 +557,7 @@ def main():
         "decode": None if args.only == "prefill" else {
             "value": dec_gbs, "unit": "GB/s", "us_per_step": dec_ms * 1e3, "algorithmic_bytes": db,
             "frac_of_measured_hbm": dec_gbs / hbm, "frac_of_8TBs": dec_gbs / 8000.0},
+        "long_prefill": long_leg,
         "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": (1 if args.only else 2) * K, "clocks": clocks,
         "next_rows": rows,
     }

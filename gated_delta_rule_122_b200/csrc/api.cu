@@ -71,6 +71,60 @@ kda_status empty_sequence(const float *s_in, float *s_out, int B, int H, int dk,
 
 }  // namespace
 
+namespace kda {
+
+// The dense prefill variants after the workspace handling: argument checks, T = 0, and
+// the launch on the tensor-core or CUDA-core kernel.  status: the device status word
+// (already cleared by the caller) or null.
+kda_status prefill_launch(int kind, const void *q, const void *k, const void *v, const void *alpha,
+                          const void *beta, const float *initial_state, void *o, float *final_state, int B,
+                          int T, int H, int d_k, int d_v, float scale, kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                          kda_dtype out_dtype, unsigned int *status, cudaStream_t stream)
+{
+    const bool per_head = kind == KDA_HOST_SCALAR_GATE;
+    kda_status st = check_forward(q, k, v, alpha, beta, initial_state, o, final_state, B, T, H, d_k, d_v,
+                                  qkv_dtype, gate_dtype, out_dtype, per_head);
+    if (st != KDA_OK) return st;
+    if (B * (long long)H == 0) return KDA_OK;
+    if (T == 0) return empty_sequence(initial_state, final_state, B, H, d_k, d_v, stream);
+    ChunkArgs a{q, k, v, alpha, beta, initial_state, final_state, o, B, T, H, scale,
+                qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16, status};
+    a.gate_per_head = per_head ? 1 : 0;
+    a.raw_inputs = kind == KDA_HOST_RAW ? 1 : 0;
+    cudaError_t err;
+    if (chunk_tc_supported(d_k, d_v, qkv_dtype, gate_dtype))
+        err = launch_chunk_tc(a, d_k, d_v, stream);
+    else
+        err = launch_chunk_simt(a, d_k, d_v, stream);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+}
+
+}  // namespace kda
+
+namespace {
+
+// Workspace handling of the dense prefill entry points: size and alignment, the status
+// word cleared on the stream, then the launch.
+kda_status prefill_with_workspace(int kind, const void *q, const void *k, const void *v, const void *alpha,
+                                  const void *beta, const float *initial_state, void *o, float *final_state,
+                                  int B, int T, int H, int d_k, int d_v, float scale, kda_dtype qkv_dtype,
+                                  kda_dtype gate_dtype, kda_dtype out_dtype, void *workspace,
+                                  size_t workspace_bytes, cudaStream_t stream)
+{
+    kda_status st = check_forward(q, k, v, alpha, beta, initial_state, o, final_state, B, T, H, d_k, d_v,
+                                  qkv_dtype, gate_dtype, out_dtype, kind == KDA_HOST_SCALAR_GATE);
+    if (st != KDA_OK) return st;
+    if (B * (long long)H == 0) return KDA_OK;
+    const size_t need = kda_forward_workspace_bytes(B, T, H, d_k, d_v);
+    if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return KDA_ERR_ALIGN;
+    if (cudaMemsetAsync(workspace, 0, need, stream) != cudaSuccess) return KDA_ERR_LAUNCH;
+    return kda::prefill_launch(kind, q, k, v, alpha, beta, initial_state, o, final_state, B, T, H, d_k, d_v, scale,
+                               qkv_dtype, gate_dtype, out_dtype, static_cast<unsigned int *>(workspace), stream);
+}
+
+}  // namespace
+
 extern "C" {
 
 const char *kda_status_string(kda_status s)
@@ -116,24 +170,9 @@ kda_status kda_forward(const void *q, const void *k, const void *v, const void *
                        kda_dtype gate_dtype, kda_dtype out_dtype, void *workspace,
                        size_t workspace_bytes, cudaStream_t stream)
 {
-    kda_status st = check_forward(q, k, v, alpha, beta, initial_state, o, final_state, B, T, H,
-                                  d_k, d_v, qkv_dtype, gate_dtype, out_dtype);
-    if (st != KDA_OK) return st;
-    if (B * (long long)H == 0) return KDA_OK;
-    const size_t need = kda_forward_workspace_bytes(B, T, H, d_k, d_v);
-    if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
-    if (!aligned16(workspace)) return KDA_ERR_ALIGN;
-    if (cudaMemsetAsync(workspace, 0, need, stream) != cudaSuccess) return KDA_ERR_LAUNCH;
-    if (T == 0) return empty_sequence(initial_state, final_state, B, H, d_k, d_v, stream);
-    kda::ChunkArgs a{q, k, v, alpha, beta, initial_state, final_state, o, B, T, H, scale,
-                     qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16,
-                     static_cast<unsigned int *>(workspace)};
-    cudaError_t err;
-    if (kda::chunk_tc_supported(d_k, d_v, qkv_dtype, gate_dtype))
-        err = kda::launch_chunk_tc(a, d_k, d_v, stream);
-    else
-        err = kda::launch_chunk_simt(a, d_k, d_v, stream);
-    return err == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+    return prefill_with_workspace(KDA_HOST_FORWARD, q, k, v, alpha, beta, initial_state, o, final_state, B, T, H,
+                                  d_k, d_v, scale, qkv_dtype, gate_dtype, out_dtype, workspace, workspace_bytes,
+                                  stream);
 }
 
 kda_status kda_forward_varlen(const void *q, const void *k, const void *v, const void *alpha,
@@ -185,24 +224,9 @@ kda_status kda_forward_scalar_gate(const void *q, const void *k, const void *v, 
                                    kda_dtype out_dtype, void *workspace, size_t workspace_bytes,
                                    cudaStream_t stream)
 {
-    kda_status st = check_forward(q, k, v, alpha, beta, initial_state, o, final_state, B, T, H,
-                                  d_k, d_v, qkv_dtype, gate_dtype, out_dtype, true);
-    if (st != KDA_OK) return st;
-    if (B * (long long)H == 0) return KDA_OK;
-    const size_t need = kda_forward_workspace_bytes(B, T, H, d_k, d_v);
-    if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
-    if (!aligned16(workspace)) return KDA_ERR_ALIGN;
-    if (cudaMemsetAsync(workspace, 0, need, stream) != cudaSuccess) return KDA_ERR_LAUNCH;
-    if (T == 0) return empty_sequence(initial_state, final_state, B, H, d_k, d_v, stream);
-    kda::ChunkArgs a{q, k, v, alpha, beta, initial_state, final_state, o, B, T, H, scale,
-                     qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16,
-                     static_cast<unsigned int *>(workspace), nullptr, 1};
-    cudaError_t err;
-    if (kda::chunk_tc_supported(d_k, d_v, qkv_dtype, gate_dtype))
-        err = kda::launch_chunk_tc(a, d_k, d_v, stream);
-    else
-        err = kda::launch_chunk_simt(a, d_k, d_v, stream);
-    return err == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+    return prefill_with_workspace(KDA_HOST_SCALAR_GATE, q, k, v, alpha, beta, initial_state, o, final_state, B, T,
+                                  H, d_k, d_v, scale, qkv_dtype, gate_dtype, out_dtype, workspace, workspace_bytes,
+                                  stream);
 }
 
 kda_status kda_forward_raw(const void *q, const void *k, const void *v, const void *gate_logit,
@@ -211,25 +235,9 @@ kda_status kda_forward_raw(const void *q, const void *k, const void *v, const vo
                            kda_dtype gate_dtype, kda_dtype out_dtype, void *workspace,
                            size_t workspace_bytes, cudaStream_t stream)
 {
-    kda_status st = check_forward(q, k, v, gate_logit, beta_logit, initial_state, o, final_state, B, T, H,
-                                  d_k, d_v, qkv_dtype, gate_dtype, out_dtype);
-    if (st != KDA_OK) return st;
-    if (B * (long long)H == 0) return KDA_OK;
-    const size_t need = kda_forward_workspace_bytes(B, T, H, d_k, d_v);
-    if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
-    if (!aligned16(workspace)) return KDA_ERR_ALIGN;
-    if (cudaMemsetAsync(workspace, 0, need, stream) != cudaSuccess) return KDA_ERR_LAUNCH;
-    if (T == 0) return empty_sequence(initial_state, final_state, B, H, d_k, d_v, stream);
-    kda::ChunkArgs a{q, k, v, gate_logit, beta_logit, initial_state, final_state, o, B, T, H, scale,
-                     qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16,
-                     static_cast<unsigned int *>(workspace)};
-    a.raw_inputs = 1;
-    cudaError_t err;
-    if (kda::chunk_tc_supported(d_k, d_v, qkv_dtype, gate_dtype))
-        err = kda::launch_chunk_tc(a, d_k, d_v, stream);
-    else
-        err = kda::launch_chunk_simt(a, d_k, d_v, stream);
-    return err == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+    return prefill_with_workspace(KDA_HOST_RAW, q, k, v, gate_logit, beta_logit, initial_state, o, final_state, B,
+                                  T, H, d_k, d_v, scale, qkv_dtype, gate_dtype, out_dtype, workspace,
+                                  workspace_bytes, stream);
 }
 
 kda_status kda_decode_step_raw(const void *q, const void *k, const void *v, const void *gate_logit,

@@ -89,4 +89,11 @@ cudaError_t launch_chunk_simt(const ChunkArgs &a, int dk, int dv, cudaStream_t s
 bool chunk_tc_supported(int dk, int dv, kda_dtype qkv, kda_dtype gate);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, int dk, int dv, cudaStream_t s);
 
+// The dense prefill (kind: KDA_HOST_FORWARD, KDA_HOST_SCALAR_GATE or KDA_HOST_RAW) after
+// the workspace handling: argument checks, T = 0, the launch; status cleared by the caller.
+kda_status prefill_launch(int kind, const void *q, const void *k, const void *v, const void *alpha,
+                          const void *beta, const float *initial_state, void *o, float *final_state, int B,
+                          int T, int H, int d_k, int d_v, float scale, kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                          kda_dtype out_dtype, unsigned int *status, cudaStream_t stream);
+
 }  // namespace kda

@@ -31,7 +31,8 @@ EXPORTED_SYMBOLS = ("kda_forward", "kda_forward_workspace_bytes", "kda_workspace
                     "kda_forward_gdn2", "kda_forward_raw", "kda_forward_sequential", "kda_decode_step",
                     "kda_decode_step_gdn2", "kda_decode_step_raw", "kda_decode_step_scalar_gate",
                     "kda_decode_tokens", "kda_state_copy", "kda_selftest_bounded_wait", "kda_status_string",
-                    "kda_version")
+                    "kda_version", "kda_forward_host", "kda_forward_host_workspace_bytes", "kda_decode_step_host",
+                    "kda_decode_step_host_workspace_bytes")
 
 _DT = {torch.float32: 0, torch.bfloat16: 1}
 _vp = ctypes.c_void_p
@@ -102,6 +103,14 @@ def library() -> ctypes.CDLL:
             lib.kda_status_string.restype = ctypes.c_char_p
             lib.kda_version.argtypes = []
             lib.kda_version.restype = _i
+            lib.kda_forward_host.argtypes = [_i] + fwd_args + [_vp, ctypes.c_size_t, _vp]
+            lib.kda_forward_host.restype = _i
+            lib.kda_forward_host_workspace_bytes.argtypes = [_i] * 9
+            lib.kda_forward_host_workspace_bytes.restype = ctypes.c_size_t
+            lib.kda_decode_step_host.argtypes = [_vp] * 7 + [_i] * 4 + [_f] + [_i] * 3 + [_vp, ctypes.c_size_t, _vp]
+            lib.kda_decode_step_host.restype = _i
+            lib.kda_decode_step_host_workspace_bytes.argtypes = [_i] * 7
+            lib.kda_decode_step_host_workspace_bytes.restype = ctypes.c_size_t
             _lib = lib
     return _lib
 
@@ -139,15 +148,13 @@ def _to_device(tensors, device):
     return [None if t is None else t.to(device, non_blocking=True) for t in tensors]
 
 
-# Host-buffer prefills of at least two segments run as a pipeline over token segments
-# of this many tokens: the copy of segment j+1 in and of segment j-1's outputs back
-# overlap the kernel on segment j, which continues from segment j-1's final state.
-_HOST_SEGMENT = 1024
-_PIPELINED = ("kda_forward", "kda_forward_scalar_gate", "kda_forward_raw")
+# Host-buffer prefills go through the library's host-buffer entry point, which moves the
+# inputs in and the results out itself (pipelined over token segments).
+_HOST_KIND = {"kda_forward": 0, "kda_forward_scalar_gate": 1, "kda_forward_raw": 2}
 
 
-def _prefill_host_pipelined(fn_name, q, k, v, alpha, beta, initial_state, scale, output_final_state,
-                            out_dtype, out, final_state, check_status, gate_per_head):
+def _prefill_host(fn_name, q, k, v, alpha, beta, initial_state, scale, output_final_state,
+                  out_dtype, out, final_state, check_status, gate_per_head):
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     a_shape = (B, T, H) if gate_per_head else (B, T, H, dk)
@@ -155,66 +162,51 @@ def _prefill_host_pipelined(fn_name, q, k, v, alpha, beta, initial_state, scale,
             or tuple(beta.shape) != (B, T, H):
         raise ValueError("shapes: q,k [B,T,H,dk], alpha " + ("[B,T,H]" if gate_per_head else "[B,T,H,dk]")
                          + ", v [B,T,H,dv], beta [B,T,H]")
-    for name, t in (("k", k), ("v", v), ("alpha", alpha), ("beta", beta), ("initial_state", initial_state),
-                    ("out", out), ("final_state", final_state)):
-        if t is not None and t.device.type != "cpu":
-            raise ValueError(f"{name} must be a host tensor like q")
-    if out is not None and tuple(out.shape) != (B, T, H, dv):
-        raise ValueError("out must be [B,T,H,dv]")
-    dev = torch.device("cuda", torch.cuda.current_device())
+    for name, t in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta", beta),
+                    ("initial_state", initial_state), ("out", out), ("final_state", final_state)):
+        if t is not None:
+            if t.device.type != "cpu":
+                raise ValueError(f"{name} must be a host tensor like q")
+            if not t.is_contiguous():
+                raise ValueError(f"{name} must be contiguous")
+    if k.dtype != q.dtype or v.dtype != q.dtype or alpha.dtype != beta.dtype:
+        raise TypeError("q/k/v and alpha/beta must each share a dtype")
+    if initial_state is not None and (initial_state.dtype != torch.float32
+                                      or tuple(initial_state.shape) != (B, H, dk, dv)):
+        raise ValueError("initial_state must be float32 [B,H,dk,dv]")
+    if scale is None:
+        scale = dk ** -0.5
     if out is None:
         out = torch.empty((B, T, H, dv), dtype=out_dtype, pin_memory=True)
-    keep = []   # device tensors that must outlive the streams' work
+    if tuple(out.shape) != (B, T, H, dv):
+        raise ValueError("out must be [B,T,H,dv]")
+    if final_state is None and output_final_state:
+        final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, pin_memory=True)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    lib = library()
+    kind = _HOST_KIND[fn_name]
+    qd, gd, od = _DT[q.dtype], _dt(alpha, "alpha"), _dt(out, "out")
+    ws_bytes = lib.kda_forward_host_workspace_bytes(B, T, H, dk, dv, qd, gd, od, kind)
     with torch.cuda.device(dev):
-        compute = torch.cuda.current_stream(dev)
-        h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        if initial_state is None:
-            state = torch.zeros((B, H, dk, dv), device=dev, dtype=torch.float32)
-        else:
-            state = torch.empty((B, H, dk, dv), device=dev, dtype=torch.float32)
-            state.copy_(initial_state, non_blocking=True)
-        for t0 in range(0, T, _HOST_SEGMENT):
-            t1 = min(T, t0 + _HOST_SEGMENT)
-            seg_in = []
-            with torch.cuda.stream(h2d):
-                for t in (q, k, v, alpha, beta):
-                    d = torch.empty((B, t1 - t0) + tuple(t.shape[2:]), device=dev, dtype=t.dtype)
-                    for b in range(B):   # one contiguous host run per sequence
-                        d[b].copy_(t[b, t0:t1], non_blocking=True)
-                    seg_in.append(d)
-                ready = torch.cuda.Event()
-                ready.record(h2d)
-            compute.wait_event(ready)
-            o_seg = torch.empty((B, t1 - t0, H, dv), device=dev, dtype=out.dtype)
-            _prefill(fn_name, *seg_in, state, scale, True, out_dtype, o_seg, state, None, check_status,
-                     gate_per_head)
-            done = torch.cuda.Event()
-            done.record(compute)
-            d2h.wait_event(done)
-            with torch.cuda.stream(d2h):
-                for b in range(B):
-                    out[b, t0:t1].copy_(o_seg[b], non_blocking=True)
-            keep.append((seg_in, o_seg))
-        if final_state is None and output_final_state:
-            final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, pin_memory=True)
-        if final_state is not None:
-            done = torch.cuda.Event()
-            done.record(compute)
-            d2h.wait_event(done)
-            with torch.cuda.stream(d2h):
-                final_state.copy_(state, non_blocking=True)
-        d2h.synchronize()
-        h2d.synchronize()
-        compute.synchronize()
+        ws = torch.empty(max(ws_bytes, 256), device=dev, dtype=torch.uint8)
+        stream = _vp(_stream_handle(dev))
+        code = lib.kda_forward_host(kind, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(initial_state),
+                                    _ptr(out), _ptr(final_state), B, T, H, dk, dv, float(scale), qd, gd, od,
+                                    _ptr(ws), ws.numel(), stream)
+        if code == 0 and check_status:
+            code = lib.kda_workspace_status(_ptr(ws), stream)
+        torch.cuda.current_stream(dev).synchronize()
+    if code != 0:
+        raise KDAError("kda_forward_host", code)
     return out, final_state
 
 
 def _prefill(fn_name, q, k, v, alpha, beta, initial_state, scale, output_final_state,
              out_dtype, out, final_state, workspace=None, check_status=False, gate_per_head=False):
     host = q.device.type == "cpu"
-    if host and fn_name in _PIPELINED and q.dim() == 4 and q.shape[1] >= 2 * _HOST_SEGMENT:
-        return _prefill_host_pipelined(fn_name, q, k, v, alpha, beta, initial_state, scale, output_final_state,
-                                       out_dtype, out, final_state, check_status, gate_per_head)
+    if host and fn_name in _HOST_KIND:
+        return _prefill_host(fn_name, q, k, v, alpha, beta, initial_state, scale, output_final_state,
+                             out_dtype, out, final_state, check_status, gate_per_head)
     host_out = host_state = None
     if host:
         # end-to-end path: host inputs are copied in (asynchronously when pinned),
@@ -338,6 +330,8 @@ def _decode(fn, q, k, v, alpha, beta, state, scale, out_dtype, out, gate_per_hea
     if device.type != "cuda":
         raise ValueError("the decode step needs the state on a CUDA device")
     N, H, dk, dv = state.shape
+    if fn == "kda_decode_step" and q.device.type == "cpu":
+        return _decode_host(q, k, v, alpha, beta, state, scale, out_dtype, out)
     for name, t in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta", beta),
                     ("state", state)):
         _check(name, t, device)
@@ -363,6 +357,40 @@ def _decode(fn, q, k, v, alpha, beta, state, scale, out_dtype, out, gate_per_hea
             _vp(_stream_handle(device)))
     if code != 0:
         raise KDAError(fn, code)
+    return out
+
+
+def _decode_host(q, k, v, alpha, beta, state, scale, out_dtype, out):
+    """Decode step with host token vectors and host o, the state resident on the device
+    (C entry point ``kda_decode_step_host``)."""
+    device = state.device
+    N, H, dk, dv = state.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta", beta)):
+        if t.device.type != "cpu" or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous host tensor like q")
+    _check("state", state, device)
+    if tuple(q.shape) != (N, H, dk) or tuple(k.shape) != (N, H, dk) or tuple(alpha.shape) != (N, H, dk) \
+            or tuple(v.shape) != (N, H, dv) or tuple(beta.shape) != (N, H):
+        raise ValueError("shapes: q,k,alpha [N,H,dk], v [N,H,dv], beta [N,H], state [N,H,dk,dv]")
+    if k.dtype != q.dtype or v.dtype != q.dtype or alpha.dtype != beta.dtype or state.dtype != torch.float32:
+        raise TypeError("q/k/v and alpha/beta must each share a dtype; the state is float32")
+    if scale is None:
+        scale = dk ** -0.5
+    if out is None:
+        out = torch.empty((N, H, dv), dtype=out_dtype, pin_memory=True)
+    if out.device.type != "cpu" or tuple(out.shape) != (N, H, dv):
+        raise ValueError("out must be a host tensor [N,H,dv]")
+    lib = library()
+    qd, gd, od = _DT[q.dtype], _dt(alpha, "alpha"), _dt(out, "out")
+    with torch.cuda.device(device):
+        nb = lib.kda_decode_step_host_workspace_bytes(N, H, dk, dv, qd, gd, od)
+        ws = torch.empty(max(nb, 256), device=device, dtype=torch.uint8)
+        code = lib.kda_decode_step_host(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(state), _ptr(out),
+                                        N, H, dk, dv, float(scale), qd, gd, od, _ptr(ws), ws.numel(),
+                                        _vp(_stream_handle(device)))
+        torch.cuda.current_stream(device).synchronize()
+    if code != 0:
+        raise KDAError("kda_decode_step_host", code)
     return out
 
 

@@ -321,6 +321,62 @@ kda_status kda_decode_step_gdn2(const void *q, const void *k, const void *v,
                                 kda_dtype out_dtype, cudaStream_t stream);
 
 /*
+ * Host-buffer entry points: for a caller whose tensors live in host memory (pinned
+ * memory lets the copies overlap the kernels; pageable memory works but copies
+ * synchronously).  The library copies the inputs in and the results out itself; not
+ * part of the recurrence, and the pages have no counterpart.
+ *
+ * kda_forward_host -- one prefill (kind KDA_HOST_FORWARD: kda_forward;
+ * KDA_HOST_SCALAR_GATE: kda_forward_scalar_gate, alpha [B, T, H]; KDA_HOST_RAW:
+ * kda_forward_raw) with q, k, v, alpha, beta, initial_state (or NULL), o and
+ * final_state (or NULL) all HOST pointers in the layouts of those entry points.
+ * The sequence is cut into segments of 1024 tokens: segment j+1 is copied in on an
+ * internal stream while the kernel runs segment j on `stream`, continuing from
+ * segment j-1's state, and segment j-1's outputs are copied back on another internal
+ * stream.  workspace: DEVICE memory of kda_forward_host_workspace_bytes() bytes,
+ * 256-byte aligned, owned by the caller: two slots of segment buffers, the carried
+ * state and, at offset 0, the status word (read it with kda_workspace_status()).
+ * Asynchronous: everything is ordered after the work already on `stream`, and work
+ * queued on `stream` afterwards (a synchronization included) starts only once the
+ * last result is back in host memory.  The host buffers must stay valid until then.
+ * Argument errors return before anything is queued; a failing segment returns its
+ * status (work already queued still runs).
+ */
+typedef enum { KDA_HOST_FORWARD = 0, KDA_HOST_SCALAR_GATE = 1, KDA_HOST_RAW = 2 } kda_host_kind;
+
+size_t kda_forward_host_workspace_bytes(int B, int T, int H, int d_k, int d_v,
+                                        kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                                        kda_dtype out_dtype, int kind);
+
+kda_status kda_forward_host(int kind, const void *q, const void *k,
+                            const void *v, const void *alpha, const void *beta,
+                            const float *initial_state, void *o,
+                            float *final_state, int B, int T, int H, int d_k,
+                            int d_v, float scale, kda_dtype qkv_dtype,
+                            kda_dtype gate_dtype, kda_dtype out_dtype,
+                            void *workspace, size_t workspace_bytes,
+                            cudaStream_t stream);
+
+/*
+ * kda_decode_step_host -- kda_decode_step with q, k, alpha [N, H, d_k], v [N, H, d_v],
+ * beta [N, H] and o [N, H, d_v] in HOST memory, and the state [N, H, d_k, d_v] fp32 in
+ * DEVICE memory (it stays resident between steps, like a KV cache), updated in place.
+ * The copies and the kernel run in order on `stream`; workspace: DEVICE memory of
+ * kda_decode_step_host_workspace_bytes() bytes, 256-byte aligned, for the token
+ * vectors and o.  Asynchronous like kda_forward_host.
+ */
+size_t kda_decode_step_host_workspace_bytes(int N, int H, int d_k, int d_v,
+                                            kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                                            kda_dtype out_dtype);
+
+kda_status kda_decode_step_host(const void *q, const void *k, const void *v,
+                                const void *alpha, const void *beta, float *state,
+                                void *o, int N, int H, int d_k, int d_v, float scale,
+                                kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                                kda_dtype out_dtype, void *workspace,
+                                size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Serving operations.  A recurrent state is request-scoped, like a KV-cache
  * slot: it is cached between turns and must be copied whenever a request is
  * forked, shares a prefix, migrates or is rolled back after a speculative

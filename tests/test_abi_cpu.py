@@ -181,3 +181,25 @@ def test_selftest_rejects_bad_arguments(lib):
     assert lib.kda_selftest_bounded_wait(0, 1000, 0x90004, None) == ERR_ALIGN
     assert lib.kda_selftest_bounded_wait(0, 0, 0x90000, None) == ERR_SHAPE
     assert lib.kda_selftest_bounded_wait(0, 2000001, 0x90000, None) == ERR_SHAPE
+
+
+def test_host_path_rejects_bad_arguments(lib):
+    def f(kind=0, q=0x10000, dk=16, B=1, T=4, ws=0x100000, wsb=1 << 20):
+        return lib.kda_forward_host(kind, q, 0x20000, 0x30000, 0x40000, 0x50000, None, 0x60000, None, B, T, 1, dk, 16,
+                                    1.0, 0, 0, 0, ws, wsb, None)
+    assert f(kind=3) == ERR_SHAPE
+    assert f(q=None) == ERR_NULL
+    assert f(dk=40) == ERR_UNSUP
+    assert f(ws=None) == ERR_WS
+    assert f(wsb=64) == ERR_WS
+    assert f(ws=0x100010) == ERR_ALIGN                      # the workspace needs 256-byte alignment
+    assert f(B=0) == OK
+    need = lib.kda_forward_host_workspace_bytes(2, 8192, 64, 128, 128, 1, 1, 0, 0)
+    # two slots of 1024-token segments and the carried state, plus the status word
+    seg = 2 * 1024 * 64 * (3 * 256 + 256 + 2 + 512)
+    assert need >= 2 * seg + 2 * 64 * 128 * 128 * 4
+    d = lib.kda_decode_step_host
+    assert d(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, None, 0x60000, 2, 1, 16, 16, 1.0, 0, 0, 0,
+             0x100000, 1 << 20, None) == ERR_NULL
+    assert d(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 0x70000, 0x60000, 2, 1, 16, 16, 1.0, 0, 0, 0,
+             None, 0, None) == ERR_WS

@@ -291,3 +291,17 @@ def test_full_size_prefill_sampled_heads(name):
     for (b, h), (o_ref, s_ref) in ref.items():
         assert o_err(o[b, :, h], o_ref) < TOL_BF16, (b, h)
         assert s_err(S[b, h], s_ref) < TOL_BF16, (b, h)
+
+
+def test_decode_step_host_inputs_match_device():
+    """Host token vectors and host o with the state resident on the device (the host-buffer
+    decode entry point) give the device path's results exactly."""
+    x = make_decode_inputs(WORKLOADS["decode"].scaled(B=5, H=3))
+    s_host_path = x["state"].cuda()
+    s_dev_path = x["state"].cuda()
+    hx = {n: x[n].pin_memory() for n in ("q", "k", "v", "alpha", "beta")}
+    o_h = kda.decode_step(hx["q"], hx["k"], hx["v"], hx["alpha"], hx["beta"], s_host_path, scale=x["scale"])
+    d = to_device(x)
+    o_d = kda.decode_step(d["q"], d["k"], d["v"], d["alpha"], d["beta"], s_dev_path, scale=x["scale"])
+    torch.cuda.synchronize()
+    assert o_h.device.type == "cpu" and torch.equal(o_h, o_d.cpu()) and torch.equal(s_host_path, s_dev_path)
