@@ -70,6 +70,9 @@ def parse_args():
     ap.add_argument("--no-long", action="store_true", help="skip the long-prefill measurement")
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="run one kernel per step (for profiling); the JSON line is then partial")
+    ap.add_argument("--prefill-workload", choices=["prefill", "long"], default="prefill",
+                    help="the prefill workload of each step (profiling the long workload; the JSON line "
+                         "then describes that workload)")
     ap.add_argument("--prefill-seqs", type=int, default=None,
                     help="sequences per rank of the prefill workload (profiling a smaller case; "
                          "the JSON line then describes that case, not the headline workload)")
@@ -410,7 +413,7 @@ def main():
     peaks, peak_kind = load_peaks()
 
     from gated_delta_rule_122_b200.shard import shard_bounds
-    wp, wd = workload("prefill"), workload("decode")
+    wp, wd = workload(args.prefill_workload), workload("decode")
     # the global batch is world x the workload's sequences; this rank's block of them
     p0, p1 = shard_bounds(world * wp.B, rank, world)
     d0, d1 = shard_bounds(world * wd.B, rank, world)
@@ -522,23 +525,23 @@ def main():
 
     long_leg = None
     if world == 1 and not args.no_long and args.only is None and args.prefill_seqs is None \
-            and args.prefill_len is None:
+            and args.prefill_len is None and args.prefill_workload == "prefill":
         long_leg = measure_long(torch, kda, device, hbm)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_prefill(x, wp)
     rows = None
     if world == 1 and not args.no_rows and args.only is None and args.prefill_seqs is None \
-            and args.prefill_len is None:
+            and args.prefill_len is None and args.prefill_workload == "prefill":
         rows = measure_rows(torch, kda, x, y, wp, float(peaks["hbm_gbs"]))
 
     clocks = sampler.summary()
     if rank != 0:
         return
-    headline = args.prefill_seqs is None and args.prefill_len is None
+    headline = args.prefill_seqs is None and args.prefill_len is None and args.prefill_workload == "prefill"
     traffic = PREFILL_TRAFFIC_BYTES if headline and kernel_sources_hash() == PREFILL_TRAFFIC_SOURCES else None
-    workload_desc = (f"prefill B={wp.B * world} H={wp.H} T={wp.T} d_k=d_v={wp.dk} bf16 q/k/v/alpha/beta, "
-                     "fp32 o and state")
+    workload_desc = (f"{wp.name} B={wp.B * world} H={wp.H} T={wp.T} d_k=d_v={wp.dk} bf16 q/k/v/alpha/beta, "
+                     "fp32 o and state" + (", random initial state" if wp.init_state else ""))
     if args.only != "prefill":
         workload_desc += f" (+ decode step N={wd.B * world} H={wd.H} d={wd.dk} in the same step)"
     line = {

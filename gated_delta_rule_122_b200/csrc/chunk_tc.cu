@@ -135,10 +135,9 @@ constexpr int kNrmSlots = 4;
 constexpr int NRM_BYTES = 2 * C * 4;
 constexpr int OFF_NRM = OFF_BETA + C * 4;
 constexpr int OFF_TPU = (OFF_NRM + kNrmSlots * NRM_BYTES + 127) / 128 * 128;   // raw: T Diag(beta), B of U
-constexpr int NBARS = 7;
+constexpr int NBARS = 14;
 constexpr int OFF_BAR = (OFF_TPU + C * C * 4 + 7) / 8 * 8;
-constexpr int OFF_SIG = OFF_BAR + NBARS * 8;           // 6 readiness counters (8 slots)
-constexpr int OFF_MISC = OFF_SIG + 32;                 // tmem base, error flag
+constexpr int OFF_MISC = OFF_BAR + NBARS * 8;          // tmem base, error flag
 // Chunks whose decay leaves the range of the anchored factors: slot n % 4 holds n + 1
 // when chunk n is one (written by stage A, read by the chain warps after a barrier).
 constexpr int kXSlots = 4;
@@ -224,19 +223,22 @@ constexpr int HG_ROW = 16;   // bytes per token row of a staged per-head gate bo
 // (token, head) staged by TMA as boxes of 8 heads x 32 tokens, or read from memory.
 constexpr int kGateChannel = 0, kGateHeadTma = 1, kGateHeadMem = 2;
 
-// Every warp of a role adds 1 to a readiness counter once its writes are visible
-// (the counter of chunk n's step reaches (n + 1) x the role's warps).
-__device__ __forceinline__ void warp_signal(uint32_t cnt, int lane)
+// Every warp of a role arrives once on a readiness mbarrier once its writes are visible
+// (release semantics; the barrier's phase for chunk n completes when all the role's
+// warps have arrived, and the MMA issuer waits on it with acquire semantics).
+__device__ __forceinline__ void warp_signal(uint32_t bar, int lane)
 {
     __syncwarp();
-    if (lane == 0) ptx::red_add_release(cnt, 1u);
+    if (lane == 0) ptx::mbar_arrive(bar);
 }
 
 struct Bars {
     uint32_t a, w, e, s;      // issuer -> warps (mbarriers, tcgen05.commit)
     uint32_t stg, v;          // TMA fills: q/k/alpha staging; V buffers (v and v + 8)
-    uint32_t rc, rs, re;      // chain -> issuer counters: operands staged, S' written, E^T written
-    uint32_t ra, rg, rj;      // prep -> issuer counters: A read, T' and A_qk written, -W' written
+    // warps -> issuer (mbarriers, one arrival per warp and chunk):
+    uint32_t rc;              // chain: operands of chunk n staged (rc + 8 (n & 1): one per parity of n)
+    uint32_t rs, re;          // chain: S' written, E^T written
+    uint32_t ra, rg, rj;      // prep: A read, T' and A_qk written, -W' written
 };
 
 // ---- the MMA-issuer warp (lane 0) -------------------------------------------------
@@ -310,10 +312,15 @@ __device__ __forceinline__ void issue_m2(uint8_t *sm, uint32_t tmem, const Bars 
     ptx::mma_commit(bars.w);
 }
 
-// Readiness of each group: M1(n) needs Lk, Lq, R of chunk n (rc) and A(n-1) read
-// (ra), so it runs while the prep warps solve chunk n-1; M2(n) needs T' and A_qk (rg; the prep warps signal it after reading
-// W'(n-1)) and M4(n-1) issued, since U goes into TM_E; M3(n) needs S'(n) (rs,
-// whose first count is the initial state) and -W'(n) (rj); M4(n) needs E^T(n) (re).
+// The issuer takes the groups in a fixed order, waiting on each group's readiness
+// mbarriers (the warp sleeps in the wait and wakes when the phase completes):
+//   M1(0), M1(1), M2(0), then for each chunk c: M3(c), M4(c), M2(c+1), M1(c+2).
+// M1(n) needs Lk, Lq, R of chunk n (rc) and A(n-1) read by the prep warps (ra, since
+// A(n) overwrites it); M2(n) needs T' and A_qk (rg, which the prep warps signal after
+// reading W'(n-1)) and the E readout of chunk n-1 (U(n) overwrites E in TMEM; implied
+// by M4(n-1) having been issued); M3(n) needs S'(n) (rs) and -W'(n) (rj); M4(n) needs
+// E^T(n) (re).  Each producer is at most one phase ahead of this order: every arrival
+// for chunk n+1 depends on a group of chunk n that is issued after the wait for chunk n.
 template <bool kRaw>
 __device__ void issuer(uint8_t *sm, uint32_t tmem, const Bars &bars, int nchunks, volatile int *err_flag)
 {
@@ -324,45 +331,31 @@ __device__ void issuer(uint8_t *sm, uint32_t tmem, const Bars &bars, int nchunks
     id.OE = ptx::idesc_bf16(128, 128, 0, 1, 0);   // S' (TMEM) x [Lq | -W'] (MN)
     id.O2 = ptx::idesc_bf16(128, 64, 0, 0, 0);    // E^T x A_qk
     id.dS = ptx::idesc_bf16(128, 128, 0, 0, 0);   // E^T x R (d x s)
-    int n1 = 0, n2 = 0, n3 = 0, n4 = 0;   // next chunk of each group
-    uint32_t idle = 0;                     // polls since the last issue
-    uint64_t t_idle = 0;
-    while (n4 < nchunks) {
-        const uint32_t c_rs = ptx::ld_relaxed(bars.rs), c_rj = ptx::ld_relaxed(bars.rj);
-        const uint32_t c_re = ptx::ld_relaxed(bars.re), c_rg = ptx::ld_relaxed(bars.rg);
-        const uint32_t c_rc = ptx::ld_relaxed(bars.rc), c_ra = ptx::ld_relaxed(bars.ra);
-        int g = 0;
-        if (n3 < n2 && n3 <= n4 && c_rs >= (uint32_t)(NCW * (n3 + 1)) && c_rj >= (uint32_t)(NPW * (n3 + 1)))
-            g = 3;
-        else if (n4 < n3 && c_re >= (uint32_t)(NCW * (n4 + 1)))
-            g = 4;
-        else if (n2 < n1 && n2 <= n4 && c_rg >= (uint32_t)(NPW * (n2 + 1)))
-            g = 2;
-        else if (n1 < nchunks && c_ra >= (uint32_t)(NPW * n1) && c_rc >= (uint32_t)(NCW * (n1 + 1)))
-            g = 1;
-        if (g != 0) {
-            // acquire the producers' writes (the counters only grow)
-            if (g == 3) { (void)ptx::ld_acquire(bars.rs); (void)ptx::ld_acquire(bars.rj); }
-            else if (g == 4) (void)ptx::ld_acquire(bars.re);
-            else if (g == 2) (void)ptx::ld_acquire(bars.rg);
-            else { (void)ptx::ld_acquire(bars.ra); (void)ptx::ld_acquire(bars.rc); }
-            if (g == 3) issue_m3(sm, tmem, bars, id, n3++);
-            else if (g == 4) issue_m4(sm, tmem, bars, id, n4++);
-            else if (g == 2) issue_m2<kRaw>(sm, tmem, bars, id, n2++);
-            else issue_m1(sm, tmem, bars, id, n1++);
-            idle = 0;
-        } else if ((++idle & 1023u) == 0) {
-            // nothing ready for a while: check the time limit and the error flag
-            const uint64_t now = ptx::global_timer_ns();
-            if (idle == 1024u) t_idle = now;
-            if (now - t_idle > kWaitLimitNs || *err_flag) {
-                *err_flag = 1;
-                return;
-            }
-        } else {
-            __nanosleep(20);   // polling without a pause slows every warp's shared-memory traffic
-        }
+    bool ok = true;
+    auto wait = [&](uint32_t bar, int phase) {
+        if (ok && !ptx::mbar_wait(bar, (uint32_t)(phase & 1), kWaitLimitNs)) ok = false;
+        return ok;
+    };
+    // M1(n): operands of chunk n staged (rc, one barrier per parity of n) and A(n-1) read
+    auto m1 = [&](int n) {
+        if (n > 0) wait(bars.ra, n - 1);
+        if (wait(bars.rc + 8 * (n & 1), n >> 1)) issue_m1(sm, tmem, bars, id, n);
+    };
+    auto m2 = [&](int n) {
+        if (wait(bars.rg, n)) issue_m2<kRaw>(sm, tmem, bars, id, n);
+    };
+    m1(0);
+    if (nchunks > 1) m1(1);
+    m2(0);
+    for (int c = 0; c < nchunks && ok; ++c) {
+        wait(bars.rs, c);
+        if (wait(bars.rj, c)) issue_m3(sm, tmem, bars, id, c);
+        if (wait(bars.re, c)) issue_m4(sm, tmem, bars, id, c);
+        if (c + 1 < nchunks) m2(c + 1);
+        if (c + 2 < nchunks) m1(c + 2);
+        if (*err_flag) ok = false;
     }
+    if (!ok) *err_flag = 1;
 }
 
 // ---- T' = (I + A_kk)^-1 Diag(beta), blocked over the four prep warps -------------
@@ -576,7 +569,8 @@ __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, u
         ptx::tc_fence_after();
         // raw inputs: the chain's stage A of chunk cn wrote its norms before adding to the
         // count rc, which M1(cn) waited for; acquiring rc makes them visible here
-        if constexpr (kRaw) (void)ptx::ld_acquire(bars.rc);
+        if constexpr (kRaw)
+            if (!ptx::mbar_wait(bars.rc + 8 * (cn & 1), (uint32_t)((cn >> 1) & 1), kWaitLimitNs)) *err_flag = 1;
         float a32[32];   // this plane's row r times R, summed over R's planes
 #pragma unroll
         for (int hs = 0; hs < 2; ++hs) {
@@ -799,15 +793,15 @@ __device__ __forceinline__ void chain_stage_b(const TcMaps &maps, uint8_t *sm, c
 {
     stage_b(sm, n, warp, lane, ie);
     ptx::fence_proxy_async_smem();
-    warp_signal(bars.rc, lane);
+    warp_signal(bars.rc + 8 * (n & 1), lane);
     chain_bar();   // staging consumed, constants visible to every chain warp
     if (tid == kTmaThread && n + 1 < nchunks) load_qka<kGate>(maps, sm, bars, tp, n + 1);
 }
 
-__device__ __forceinline__ void warp_signal_after_stage(const Bars &bars, int lane)
+__device__ __forceinline__ void warp_signal_after_stage(const Bars &bars, int n, int lane)
 {
     ptx::fence_proxy_async_smem();
-    warp_signal(bars.rc, lane);
+    warp_signal(bars.rc + 8 * (n & 1), lane);
 }
 
 __device__ __forceinline__ bool chunk_is_extreme(const uint8_t *sm, int n)
@@ -1063,7 +1057,7 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
         // chunk c+2 can then start while the state is rewritten
         if (c + 2 < nchunks) {
             stage_b(sm, c + 2, warp, lane, ie);
-            warp_signal_after_stage(bars, lane);
+            warp_signal_after_stage(bars, c + 2, lane);
         }
         const bool xn = c + 1 < nchunks && chunk_is_extreme(sm, c + 1);
         if (xc) {
@@ -1229,9 +1223,9 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs pa, const
     Bars bars;
     bars.a = bar0; bars.w = bar0 + 8; bars.e = bar0 + 16; bars.s = bar0 + 24;
     bars.stg = bar0 + 32; bars.v = bar0 + 40;   // v and v + 8
-    const uint32_t sig0 = ptx::smem_u32(sm + OFF_SIG);
-    bars.rc = sig0; bars.rs = sig0 + 4; bars.re = sig0 + 8;
-    bars.ra = sig0 + 12; bars.rg = sig0 + 16; bars.rj = sig0 + 20;
+    bars.rc = bar0 + 56;   // and bar0 + 64
+    bars.rs = bar0 + 72; bars.re = bar0 + 80;
+    bars.ra = bar0 + 88; bars.rg = bar0 + 96; bars.rj = bar0 + 104;
 
     if (tid == 0) {
         ptx::mbar_init(bars.a, 1);
@@ -1241,9 +1235,14 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs pa, const
         ptx::mbar_init(bars.stg, 1);
         ptx::mbar_init(bars.v, 1);
         ptx::mbar_init(bars.v + 8, 1);
+        ptx::mbar_init(bars.rc, NCW);
+        ptx::mbar_init(bars.rc + 8, NCW);
+        ptx::mbar_init(bars.rs, NCW);
+        ptx::mbar_init(bars.re, NCW);
+        ptx::mbar_init(bars.ra, NPW);
+        ptx::mbar_init(bars.rg, NPW);
+        ptx::mbar_init(bars.rj, NPW);
         ptx::fence_mbar_init();
-#pragma unroll
-        for (int i = 0; i < 8; ++i) reinterpret_cast<uint32_t *>(sm + OFF_SIG)[i] = 0u;
 #pragma unroll
         for (int i = 0; i < kXSlots; ++i) reinterpret_cast<int *>(sm + OFF_XF)[i] = 0;
         *err_flag = 0;

@@ -82,13 +82,16 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 }
 
 // Wait for the phase with the given parity to complete; give up after
-// limit_ns nanoseconds and return false (the caller records the timeout).
+// limit_ns nanoseconds and return false (the caller records the timeout).  Each
+// try_wait blocks for a hardware-chosen interval; without a suspend-time hint the
+// waiting warps resume sooner after the phase completes (measured: about 1.7 % of the
+// prefill's time against a 100 us hint).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
-        if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+        if (mbar_try_wait(bar, parity)) return true;
         if (global_timer_ns() - t0 > limit_ns) return false;
     }
 }
