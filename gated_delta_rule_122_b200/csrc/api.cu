@@ -294,8 +294,14 @@ kda_status kda_forward_gdn2(const void *q, const void *k, const void *v, const v
     kda::ChunkArgs a{q, k, v, alpha, nullptr, initial_state, final_state, o, B, T, H, scale,
                      qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16,
                      static_cast<unsigned int *>(workspace), nullptr, 0, erase, wgate};
-    // the CUDA-core chunk kernel serves every shape and dtype of GDN-2
-    return kda::launch_chunk_simt(a, d_k, d_v, stream) == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+    // the tensor-core kernel for d_k = d_v = 128 with bf16 inputs and gates, the CUDA-core
+    // chunk kernel for every other shape and dtype
+    cudaError_t err;
+    if (kda::chunk_tc_supported(d_k, d_v, qkv_dtype, gate_dtype))
+        err = kda::launch_chunk_tc(a, d_k, d_v, stream);
+    else
+        err = kda::launch_chunk_simt(a, d_k, d_v, stream);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
 }
 
 kda_status kda_forward_sequential(const void *q, const void *k, const void *v, const void *alpha,

@@ -200,11 +200,12 @@ __device__ __forceinline__ bool prep_bar_err(volatile int *err_flag)
     return ptx::named_bar_sync_or(kPrepBar, NPT, *err_flag != 0);
 }
 
-template <bool kRaw>
+template <bool kRaw, bool kGdn2 = false>
 __device__ __forceinline__ float load_beta(const ChunkArgs &p, const SeqSpan &sp, int h, int n, int r)
 {
     const int t = n * C + r;
     if (t >= sp.len) return 0.f;
+    if constexpr (kGdn2) return 1.f;   // GDN-2: the write gate takes beta's place, on v
     const float y = __bfloat162float(((const __nv_bfloat16 *)p.beta)[(sp.tok0 + t) * p.H + h]);
     if constexpr (kRaw) return ptx::rcp(1.f + __expf(-y));   // a beta logit: sigmoid(y)
     else return y;
@@ -215,13 +216,18 @@ __device__ __forceinline__ float load_beta(const ChunkArgs &p, const SeqSpan &sp
 // MN-major core-matrix layout of the U^T product; o as boxes of 16 token rows.
 struct TcMaps {
     CUtensorMap q, k, a, v, o;
+    CUtensorMap w, b;   // GDN-2: write gate (as v) and erase gate (as k, L2 prefetches only)
 };
 constexpr int HG_ROW = 16;   // bytes per token row of a staged per-head gate box
 
 // The gate kind is a template parameter of the kernel (a run-time choice inside stage A
 // costs the chain measurably): alpha rows per token and key channel, one gate per
 // (token, head) staged by TMA as boxes of 8 heads x 32 tokens, or read from memory.
-constexpr int kGateChannel = 0, kGateHeadTma = 1, kGateHeadMem = 2;
+// kGateGdn2: alpha per key channel plus GDN-2's erase gate b [B, T, H, d_k] (the
+// retrieval key is b * k) and write gate w [B, T, H, d_v] (the target is w * v), no beta
+// ("From Fast Weight Programmers to KDA", section "Gated DeltaNet-2").
+constexpr int kGateChannel = 0, kGateHeadTma = 1, kGateHeadMem = 2, kGateGdn2 = 3;
+__host__ __device__ constexpr bool per_channel(int g) { return g == kGateChannel || g == kGateGdn2; }
 
 // Every warp of a role arrives once on a readiness mbarrier once its writes are visible
 // (release semantics; the barrier's phase for chunk n completes when all the role's
@@ -292,13 +298,14 @@ __device__ __forceinline__ void issue_m1(uint8_t *sm, uint32_t tmem, const Bars 
     ptx::mma_commit(bars.a);
 }
 
-template <bool kRaw>
+template <int kGate, bool kRaw>
 __device__ __forceinline__ void issue_m2(uint8_t *sm, uint32_t tmem, const Bars &bars, const MmaIds &id, int n2)
 {
     ptx::tc_fence_after();
     const uint32_t base = ptx::smem_u32(sm + OFF_LQR + (n2 & 1) * LQR_BYTES);
     const uint32_t tp = ptx::smem_u32(sm + OFF_TP);
-    const uint32_t vv = ptx::smem_u32(sm + OFF_V + (n2 & 1) * V_BYTES);
+    // GDN-2: one V stage holding the hi and lo planes of w * v in the two V buffers
+    const uint32_t vv = ptx::smem_u32(sm + OFF_V + (kGate == kGateGdn2 ? 0 : (n2 & 1) * V_BYTES));
     for (int ks = 0; ks < C / 16; ++ks)
         for (int pl = 0; pl < 2; ++pl)
             // Lk plane pl as the K-major (M = d, K = s) operand: token blocks 2 slabs apart
@@ -306,9 +313,11 @@ __device__ __forceinline__ void issue_m2(uint8_t *sm, uint32_t tmem, const Bars 
                           ptx::smem_desc(base + (SL_LK + pl) * SLAB + 4 * SLAB * ks, 2 * SLAB, 128),
                           ptx::smem_desc(tp + 256 * ks, 128, 512), id.W, ks > 0 || pl > 0);
     const uint32_t tu = kRaw ? ptx::smem_u32(sm + OFF_TPU) : tp;   // raw inputs: T Diag(beta) for U
+    constexpr int kVPlanes = kGate == kGateGdn2 ? 2 : 1;
     for (int ks = 0; ks < C / 16; ++ks)
-        ptx::mma_bf16(tmem + TM_E, ptx::smem_desc(vv + 256 * ks, 128, (C / 8) * 128),
-                      ptx::smem_desc(tu + 256 * ks, 128, 512), id.U, ks > 0);
+        for (int pl = 0; pl < kVPlanes; ++pl)
+            ptx::mma_bf16(tmem + TM_E, ptx::smem_desc(vv + pl * V_BYTES + 256 * ks, 128, (C / 8) * 128),
+                          ptx::smem_desc(tu + 256 * ks, 128, 512), id.U, ks > 0 || pl > 0);
     ptx::mma_commit(bars.w);
 }
 
@@ -321,7 +330,7 @@ __device__ __forceinline__ void issue_m2(uint8_t *sm, uint32_t tmem, const Bars 
 // by M4(n-1) having been issued); M3(n) needs S'(n) (rs) and -W'(n) (rj); M4(n) needs
 // E^T(n) (re).  Each producer is at most one phase ahead of this order: every arrival
 // for chunk n+1 depends on a group of chunk n that is issued after the wait for chunk n.
-template <bool kRaw>
+template <int kGate, bool kRaw>
 __device__ void issuer(uint8_t *sm, uint32_t tmem, const Bars &bars, int nchunks, volatile int *err_flag)
 {
     MmaIds id;
@@ -342,7 +351,7 @@ __device__ void issuer(uint8_t *sm, uint32_t tmem, const Bars &bars, int nchunks
         if (wait(bars.rc + 8 * (n & 1), n >> 1)) issue_m1(sm, tmem, bars, id, n);
     };
     auto m2 = [&](int n) {
-        if (wait(bars.rg, n)) issue_m2<kRaw>(sm, tmem, bars, id, n);
+        if (wait(bars.rg, n)) issue_m2<kGate, kRaw>(sm, tmem, bars, id, n);
     };
     m1(0);
     if (nchunks > 1) m1(1);
@@ -449,9 +458,20 @@ __device__ void stage_a(const ChunkArgs &p, uint8_t *sm, const SeqSpan &sp, int 
         cst[2 * D + d] = (n > 0) ? aexp * cst_prev[D + d] : 0.f;   // state-update factor
     }
     const bool e_in_pr = (hf == 1) != kRaw;   // pr holds e (else 1/e)
+    // GDN-2: the erase gate of this channel for the chunk's rows, read from global memory
+    // (prefetched to L2 with the staged rows)
+    const __nv_bfloat16 *bcol =
+        kGate == kGateGdn2 ? (const __nv_bfloat16 *)p.erase + ((sp.tok0 + (size_t)n * C) * p.H + h) * D + d : nullptr;
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-        float lk[8], lq[8], ie[8];
+        float lk[8], lq[8], ie[8], bv[8];
+        if constexpr (kGate == kGateGdn2) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int r = 16 * hf + 8 * u + i;
+                bv[i] = (r < Lc) ? __bfloat162float(bcol[(size_t)r * p.H * D]) : 0.f;
+            }
+        }
         const uint64_t scale2 = ptx::pk2(p.scale, p.scale);
 #pragma unroll
         for (int i = 0; i < 8; i += 2) {
@@ -468,7 +488,10 @@ __device__ void stage_a(const ChunkArgs &p, uint8_t *sm, const SeqSpan &sp, int 
                 qv[t] = (r < Lc) ? ld_bf16(stg + STG_Q + stg_row(r) + 2 * d) : 0.f;
             }
             const uint64_t e2 = ptx::pk2(e[0], e[1]);
-            ptx::upk2(ptx::mul2(ptx::pk2(kv[0], kv[1]), e2), lk[i], lk[i + 1]);
+            if constexpr (kGate == kGateGdn2)   // the retrieval key b * k
+                ptx::upk2(ptx::mul2(ptx::mul2(ptx::pk2(kv[0], kv[1]), ptx::pk2(bv[i], bv[i + 1])), e2), lk[i], lk[i + 1]);
+            else
+                ptx::upk2(ptx::mul2(ptx::pk2(kv[0], kv[1]), e2), lk[i], lk[i + 1]);
             ptx::upk2(ptx::mul2(ptx::mul2(ptx::pk2(qv[0], qv[1]), scale2), e2), lq[i], lq[i + 1]);
             // R = K/e, kept split (hi words, lo words) until its slabs are free
             float r0, r1;
@@ -504,10 +527,10 @@ template <int kGate>
 __device__ __forceinline__ void load_qka(const TcMaps &maps, uint8_t *sm, const Bars &bars, const TmaPos &tp, int n)
 {
     const uint32_t dst = ptx::smem_u32(sm + OFF_STG);
-    ptx::mbar_arrive_expect_tx(bars.stg, 2 * STG_T + (kGate == kGateChannel ? STG_T : kGate == kGateHeadTma ? C * HG_ROW : 0));
+    ptx::mbar_arrive_expect_tx(bars.stg, 2 * STG_T + (per_channel(kGate) ? STG_T : kGate == kGateHeadTma ? C * HG_ROW : 0));
     ptx::tma_load_4d(dst + STG_Q, &maps.q, bars.stg, 0, tp.h, tp.t0 + n * C, tp.b);
     ptx::tma_load_4d(dst + STG_K, &maps.k, bars.stg, 0, tp.h, tp.t0 + n * C, tp.b);
-    if constexpr (kGate == kGateChannel) ptx::tma_load_4d(dst + STG_A, &maps.a, bars.stg, 0, tp.h, tp.t0 + n * C, tp.b);
+    if constexpr (per_channel(kGate)) ptx::tma_load_4d(dst + STG_A, &maps.a, bars.stg, 0, tp.h, tp.t0 + n * C, tp.b);
     // heads h & ~7 .. (h & ~7) + 7 of 32 tokens: the x coordinate is a multiple of 8 elements
     if constexpr (kGate == kGateHeadTma) ptx::tma_load_3d(dst + STG_A, &maps.a, bars.stg, tp.h & ~7, tp.t0 + n * C, tp.b);
 }
@@ -519,16 +542,38 @@ __device__ __forceinline__ void prefetch_qka(const TcMaps &maps, const TmaPos &t
 {
     ptx::tma_prefetch_4d(&maps.q, 0, tp.h, tp.t0 + n * C, tp.b);
     ptx::tma_prefetch_4d(&maps.k, 0, tp.h, tp.t0 + n * C, tp.b);
-    if constexpr (kGate == kGateChannel) ptx::tma_prefetch_4d(&maps.a, 0, tp.h, tp.t0 + n * C, tp.b);
+    if constexpr (per_channel(kGate)) ptx::tma_prefetch_4d(&maps.a, 0, tp.h, tp.t0 + n * C, tp.b);
+    if constexpr (kGate == kGateGdn2) ptx::tma_prefetch_4d(&maps.b, 0, tp.h, tp.t0 + n * C, tp.b);
     if constexpr (kGate == kGateHeadTma) ptx::tma_prefetch_3d(&maps.a, tp.h & ~7, tp.t0 + n * C, tp.b);
 }
 
-// TMA load of chunk n's v rows into V buffer n&1 (one thread).
+// TMA load of chunk n's v rows into V buffer n&1 (one thread).  GDN-2: v into the first
+// buffer and the write gate w into the second (one stage, refilled once M2 has read it;
+// the prep warps turn the pair into the hi and lo planes of w * v in place).
+template <int kGate>
 __device__ __forceinline__ void load_v(const TcMaps &maps, uint8_t *sm, const Bars &bars, const TmaPos &tp, int n)
 {
-    const uint32_t bar = bars.v + 8 * (n & 1);
-    ptx::mbar_arrive_expect_tx(bar, V_BYTES);
-    ptx::tma_load_5d(ptx::smem_u32(sm + OFF_V + (n & 1) * V_BYTES), &maps.v, bar, 0, tp.t0 + n * C, 0, tp.h, tp.b);
+    if constexpr (kGate == kGateGdn2) {
+        ptx::mbar_arrive_expect_tx(bars.v, 2 * V_BYTES);
+        ptx::tma_load_5d(ptx::smem_u32(sm + OFF_V), &maps.v, bars.v, 0, tp.t0 + n * C, 0, tp.h, tp.b);
+        ptx::tma_load_5d(ptx::smem_u32(sm + OFF_V + V_BYTES), &maps.w, bars.v, 0, tp.t0 + n * C, 0, tp.h, tp.b);
+    } else {
+        const uint32_t bar = bars.v + 8 * (n & 1);
+        ptx::mbar_arrive_expect_tx(bar, V_BYTES);
+        ptx::tma_load_5d(ptx::smem_u32(sm + OFF_V + (n & 1) * V_BYTES), &maps.v, bar, 0, tp.t0 + n * C, 0, tp.h, tp.b);
+    }
+}
+// The mbarrier and phase parity of chunk n's V load.
+template <int kGate>
+__device__ __forceinline__ void v_bar(const Bars &bars, int n, uint32_t &bar, uint32_t &parity)
+{
+    if constexpr (kGate == kGateGdn2) {
+        bar = bars.v;
+        parity = (uint32_t)(n & 1);
+    } else {
+        bar = bars.v + 8 * (n & 1);
+        parity = (uint32_t)((n >> 1) & 1);
+    }
 }
 
 // ---- the prep warps: A readout, the solve, W' readout, V loads ---------------------
@@ -536,7 +581,7 @@ __device__ __forceinline__ void load_v(const TcMaps &maps, uint8_t *sm, const Ba
 // Lq_lo times R: warps 0 and 2 hand their partial sums to warps 1 and 3 through
 // shared memory; warp 1 forms A_kk and solves its diagonal blocks, warp 3 writes
 // A_qk, and all four finish the off-diagonal block of T and write T'.
-template <bool kRaw>
+template <int kGate, bool kRaw>
 __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, uint32_t tmem, const Bars &bars,
                           const TmaPos &tp, const SeqSpan &sp, int h, int nchunks, volatile int *err_flag)
 {
@@ -553,16 +598,18 @@ __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, u
     const int pl = (lane >> 3) & 1;
     const int r = 16 * (pw & 1) + 8 * (lane >> 4) + (lane & 7);
 
+    constexpr bool kGdn2 = kGate == kGateGdn2;
+    constexpr int kVAhead = kGdn2 ? 1 : 2;   // V stages: GDN-2 uses both buffers for one chunk
     int v_loaded = 0, v_seen = 0;   // V loads issued (thread pt 0) and waited for
     if (pt == 0) {
-        load_v(maps, sm, bars, tp, 0);
-        if (nchunks > 1) load_v(maps, sm, bars, tp, 1);
+        load_v<kGate>(maps, sm, bars, tp, 0);
+        if (!kGdn2 && nchunks > 1) load_v<kGate>(maps, sm, bars, tp, 1);
     }
-    v_loaded = nchunks > 1 ? 2 : 1;
-    float beta = (pw < 2) ? load_beta<kRaw>(p, sp, h, 0, r) : 0.f;   // beta of row r
+    v_loaded = min(kVAhead, nchunks);
+    float beta = (pw < 2) ? load_beta<kRaw, kGdn2>(p, sp, h, 0, r) : 0.f;   // beta of row r
 
     for (int cn = 0; cn < nchunks; ++cn) {
-        const float beta_next = (pw < 2 && cn + 1 < nchunks) ? load_beta<kRaw>(p, sp, h, cn + 1, r) : 0.f;
+        const float beta_next = (pw < 2 && cn + 1 < nchunks) ? load_beta<kRaw, kGdn2>(p, sp, h, cn + 1, r) : 0.f;
 
         // ---- G(cn): A_kk / A_qk from TMEM; the solve; T'
         if (!ptx::mbar_wait(bars.a, (uint32_t)(cn & 1), kWaitLimitNs)) *err_flag = 1;
@@ -593,16 +640,42 @@ __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, u
             ar[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
         }
         // V(cn) has landed (every warp observes it before it signals M2's readiness)
-        if (!ptx::mbar_wait(bars.v + 8 * (cn & 1), (uint32_t)((cn >> 1) & 1), kWaitLimitNs)) *err_flag = 1;
+        {
+            uint32_t vbar, vpar;
+            v_bar<kGate>(bars, cn, vbar, vpar);
+            if (!ptx::mbar_wait(vbar, vpar, kWaitLimitNs)) *err_flag = 1;
+        }
         v_seen = cn + 1;
+        uint8_t *vb = sm + OFF_V + (kGdn2 ? 0 : (cn & 1) * V_BYTES);
         if (sp.len - cn * C < C) {
             // rows past the sequence's end hold zeros (dense layout) or the next
             // sequence's tokens (packed): clear them, T' does not see them anyway
             const int Lc = sp.len - cn * C;
-            uint8_t *vb = sm + OFF_V + (cn & 1) * V_BYTES;
             for (int i = pt; i < (C - Lc) * (D / 8); i += NPT) {
                 const int r = Lc + i / (D / 8), jb = i % (D / 8);
                 *reinterpret_cast<uint4 *>(vb + mnmaj(8 * jb, r, C)) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            if (kGdn2) prep_bar();   // the cleared rows before the products below read them
+            ptx::fence_proxy_async_smem();
+        }
+        if constexpr (kGdn2) {
+            // w * v in place: the first buffer holds v, the second w (the same MN-major
+            // layout); they become the hi plane (w v truncated to bf16) and the lo plane
+            // (bf16 of the rest), the two A operands of U
+            for (int i = pt; i < V_BYTES / 16; i += NPT) {
+                uint4 &hv = reinterpret_cast<uint4 *>(vb)[i];
+                uint4 &lw = reinterpret_cast<uint4 *>(vb + V_BYTES)[i];
+                const uint4 vv = hv, ww = lw;
+                const uint32_t va[4] = {vv.x, vv.y, vv.z, vv.w}, wa[4] = {ww.x, ww.y, ww.z, ww.w};
+                uint32_t ho[4], lo[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float x0 = __uint_as_float(va[q] << 16) * __uint_as_float(wa[q] << 16);
+                    const float x1 = __uint_as_float(va[q] & 0xFFFF0000u) * __uint_as_float(wa[q] & 0xFFFF0000u);
+                    split_pair(x0, x1, ho[q], lo[q]);
+                }
+                hv = make_uint4(ho[0], ho[1], ho[2], ho[3]);
+                lw = make_uint4(lo[0], lo[1], lo[2], lo[3]);
             }
             ptx::fence_proxy_async_smem();
         }
@@ -706,16 +779,19 @@ __device__ void prep_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, u
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         warp_signal(bars.rj, lane);
-        // M2(cn) has completed: its V buffer can take chunk cn+2
-        if (cn + 2 < nchunks) {
-            if (pt == 0) load_v(maps, sm, bars, tp, cn + 2);
-            v_loaded = cn + 3;
+        // M2(cn) has completed: its V buffer can take chunk cn+2 (GDN-2: the one stage, cn+1)
+        if (cn + kVAhead < nchunks) {
+            if (pt == 0) load_v<kGate>(maps, sm, bars, tp, cn + kVAhead);
+            v_loaded = cn + kVAhead + 1;
         }
         if (stop) break;
     }
     // on an early exit, let the V loads still in flight land before the block ends
-    for (int n = v_seen; n < v_loaded; ++n)
-        (void)ptx::mbar_wait(bars.v + 8 * (n & 1), (uint32_t)((n >> 1) & 1), kWaitLimitNs);
+    for (int n = v_seen; n < v_loaded; ++n) {
+        uint32_t vbar, vpar;
+        v_bar<kGate>(bars, n, vbar, vpar);
+        (void)ptx::mbar_wait(vbar, vpar, kWaitLimitNs);
+    }
 }
 
 // 16 columns of S'^T in this thread's row j, starting at key channel d0: scale
@@ -842,8 +918,9 @@ __device__ __forceinline__ void sequential_chunk(const ChunkArgs &p, const uint8
         const __nv_bfloat16 *qr = (const __nv_bfloat16 *)p.q + row * D + d0;
         const __nv_bfloat16 *kr = (const __nv_bfloat16 *)p.k + row * D + d0;
         const __nv_bfloat16 *ar = (const __nv_bfloat16 *)p.alpha + row * D + d0;
+        const __nv_bfloat16 *br = (const __nv_bfloat16 *)p.erase + row * D + d0;   // GDN-2 erase gate
         float ah = 1.f;   // one gate per (token, head)
-        if constexpr (kGate != kGateChannel) ah = __bfloat162float(((const __nv_bfloat16 *)p.alpha)[row]);
+        if constexpr (!per_channel(kGate)) ah = __bfloat162float(((const __nv_bfloat16 *)p.alpha)[row]);
         float pv = 0.f, pq = 0.f, kq = 0.f;
 #pragma unroll 1
         for (int q2 = 0; q2 < 2; ++q2) {
@@ -852,17 +929,19 @@ __device__ __forceinline__ void sequential_chunk(const ChunkArgs &p, const uint8
             ptx::tmem_wait_ld();
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
-                float qv[8], kv[8], av[8];
+                float qv[8], kv[8], av[8], bv[8];
                 ld_bf16x8(qr + 32 * q2 + 8 * g, qv);
                 ld_bf16x8(kr + 32 * q2 + 8 * g, kv);
-                if constexpr (kGate == kGateChannel) ld_bf16x8(ar + 32 * q2 + 8 * g, av);
+                if constexpr (per_channel(kGate)) ld_bf16x8(ar + 32 * q2 + 8 * g, av);
+                if constexpr (kGate == kGateGdn2) ld_bf16x8(br + 32 * q2 + 8 * g, bv);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    float al = (kGate == kGateChannel) ? av[i] : ah;
+                    float al = per_channel(kGate) ? av[i] : ah;
                     if constexpr (kRaw) al = 1.f / (1.f + __expf(al));   // gate logit x: alpha = 1/(1 + e^x)
                     float &x = sv[8 * g + i];
                     x *= al;
-                    pv = fmaf(kv[i], x, pv);
+                    // the retrieval key: b * k for GDN-2
+                    pv = fmaf(kGate == kGateGdn2 ? bv[i] * kv[i] : kv[i], x, pv);
                     pq = fmaf(qv[i], x, pq);
                     kq = fmaf(kv[i], qv[i], kq);
                 }
@@ -880,9 +959,12 @@ __device__ __forceinline__ void sequential_chunk(const ChunkArgs &p, const uint8
         const float vh = (pv + other[j]) * nk;                  // S~^T k (unit key)
         const float ph = (pq + other[D + j]) * nq;              // S~^T q (unit query)
         const float kqs = (kq + other[2 * D + j]) * nk * nq;    // k . q
-        const float beta = load_beta<kRaw>(p, sp, h, c, r);
         const float vj = __bfloat162float(((const __nv_bfloat16 *)p.v)[row * D + j]);
-        const float e = beta * (vj - vh);
+        float e;
+        if constexpr (kGate == kGateGdn2)   // e = w * v - S~^T (b * k)
+            e = __bfloat162float(((const __nv_bfloat16 *)p.wgate)[row * D + j]) * vj - vh;
+        else
+            e = load_beta<kRaw>(p, sp, h, c, r) * (vj - vh);
         if (half == 0) st_elem(p.o, row * D + j, p.scale * fmaf(e, kqs, ph), p.out_bf16);
         const float ek = e * nk;
 #pragma unroll 1
@@ -1257,9 +1339,9 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs pa, const
     const uint32_t tmem = *tmem_slot;
 
     if (warp == kIssuerWarp) {
-        if (lane == 0) issuer<kRaw>(sm, tmem, bars, nchunks, err_flag);
+        if (lane == 0) issuer<kGate, kRaw>(sm, tmem, bars, nchunks, err_flag);
     } else if (warp >= NCW) {
-        prep_role<kRaw>(p, maps, sm, tmem, bars, tp, sp, h, nchunks, err_flag);
+        prep_role<kGate, kRaw>(p, maps, sm, tmem, bars, tp, sp, h, nchunks, err_flag);
     } else {
         chain_role<kGate, kRaw>(p, maps, sm, tmem, bars, tp, sp, h, bh, nchunks, err_flag);
     }
@@ -1367,15 +1449,22 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, int dk, int dv, cudaStream_t str
         head_gate_tma = a.H % 8 == 0 && ((uintptr_t)a.alpha & 15u) == 0 &&
                         encode_head_gate(&maps.a, a.alpha, mb, a.T, a.H);
     }
+    const bool gdn2 = a.erase != nullptr;
+    if (gdn2 && (!a.wgate || a.gate_per_head || a.raw_inputs)) return cudaErrorInvalidValue;
+    memset(&maps.w, 0, sizeof(maps.w));
+    memset(&maps.b, 0, sizeof(maps.b));
+    if (gdn2 && (!encode_v(&maps.w, a.wgate, mb, a.T, a.H) || !encode_rows(&maps.b, a.erase, mb, a.T, a.H)))
+        return cudaErrorInvalidValue;
     if (!encode_rows(&maps.q, a.q, mb, a.T, a.H) || !encode_rows(&maps.k, a.k, mb, a.T, a.H) ||
         (!a.gate_per_head && !encode_rows(&maps.a, a.alpha, mb, a.T, a.H)) || !encode_v(&maps.v, a.v, mb, a.T, a.H) ||
         !encode_out(&maps.o, a.o, mb, a.T, a.H, a.out_bf16))
         return cudaErrorInvalidValue;
     if (a.gate_per_head && a.raw_inputs) return cudaErrorInvalidValue;
-    auto kernel = a.gate_per_head ? (head_gate_tma ? tc::kda_chunk_tc_kernel<tc::kGateHeadTma, false>
-                                                   : tc::kda_chunk_tc_kernel<tc::kGateHeadMem, false>)
-                  : a.raw_inputs  ? tc::kda_chunk_tc_kernel<tc::kGateChannel, true>
-                                  : tc::kda_chunk_tc_kernel<tc::kGateChannel, false>;
+    auto kernel = gdn2            ? tc::kda_chunk_tc_kernel<tc::kGateGdn2, false>
+                  : a.gate_per_head ? (head_gate_tma ? tc::kda_chunk_tc_kernel<tc::kGateHeadTma, false>
+                                                     : tc::kda_chunk_tc_kernel<tc::kGateHeadMem, false>)
+                  : a.raw_inputs    ? tc::kda_chunk_tc_kernel<tc::kGateChannel, true>
+                                    : tc::kda_chunk_tc_kernel<tc::kGateChannel, false>;
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     kernel<<<(unsigned)blocks, tc::NT, tc::SMEM_BYTES, stream>>>(a, maps);

@@ -79,3 +79,49 @@ def test_gdn2_empty_sequence_copies_state():
     o, S = kda.forward_gdn2(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["alpha"]), sl(b), sl(torch.ones_like(x["v"])),
                             initial_state=x["s0"], scale=x["scale"], check_status=True)
     assert o.numel() == 0 and torch.equal(S, x["s0"])
+
+
+# --- the tensor-core prefill (d_k = d_v = 128, bf16 inputs and gates) ----------------------
+@pytest.mark.parametrize("name", ["prefill", "long"])
+@pytest.mark.parametrize("B,H,T", [(1, 1, 1), (1, 2, 31), (2, 2, 64), (1, 3, 100), (2, 1, 257)])
+def test_gdn2_tc_prefill_matches_oracle(name, B, H, T):
+    x = make_inputs(WORKLOADS[name].scaled(B=B, H=H, T=T))
+    b, wr = _gates(x["k"].shape, x["v"].shape, x["alpha"].dtype, 21 + T)
+    o_ref, s_ref = oracle.forward_gdn2(x["q"], x["k"], x["v"], x["alpha"], b, wr, s0=x["s0"], scale=x["scale"])
+    d = to_device(x)
+    o, S = kda.forward_gdn2(d["q"], d["k"], d["v"], d["alpha"], b.cuda(), wr.cuda(), initial_state=d["s0"],
+                            scale=x["scale"], check_status=True)
+    eo, es = o_err(o, o_ref), s_err(S, s_ref)
+    assert eo < TOL_BF16 and es < TOL_BF16, f"o {eo:.3e} state {es:.3e}"
+
+
+def test_gdn2_tc_strong_decay_runs_token_by_token():
+    """alpha = 0 on two tokens of one half chunk and a small retention held on some
+    channels: those chunks run token by token with the erase and write gates."""
+    x = make_inputs(WORKLOADS["long"].scaled(B=1, H=2, T=130))
+    x["alpha"][0, 40, :, :] = 0.0
+    x["alpha"][0, 44, :, :] = 0.0
+    x["alpha"][0, 80:112, 1, 5:30] = 1e-3
+    b, wr = _gates(x["k"].shape, x["v"].shape, x["alpha"].dtype, 31)
+    o_ref, s_ref = oracle.forward_gdn2(x["q"], x["k"], x["v"], x["alpha"], b, wr, s0=x["s0"], scale=x["scale"])
+    d = to_device(x)
+    o, S = kda.forward_gdn2(d["q"], d["k"], d["v"], d["alpha"], b.cuda(), wr.cuda(), initial_state=d["s0"],
+                            scale=x["scale"], check_status=True)
+    eo, es = o_err(o, o_ref), s_err(S, s_ref)
+    assert eo < TOL_BF16 and es < TOL_BF16, f"o {eo:.3e} state {es:.3e}"
+
+
+def test_gdn2_tc_tied_gates_match_kda():
+    """b = w = beta on the tensor-core path equals the KDA prefill up to the rounding of the
+    split operands (beta enters the products at different points)."""
+    x = make_inputs(WORKLOADS["long"].scaled(B=1, H=2, T=100))
+    beta = x["beta"]
+    b = beta.unsqueeze(-1).expand(*x["k"].shape).contiguous()
+    wr = beta.unsqueeze(-1).expand(*x["v"].shape).contiguous()
+    d = to_device(x)
+    o1, s1 = kda.forward_gdn2(d["q"], d["k"], d["v"], d["alpha"], b.cuda(), wr.cuda(), initial_state=d["s0"],
+                              scale=x["scale"], check_status=True)
+    o2, s2 = kda.forward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], initial_state=d["s0"],
+                         scale=x["scale"], check_status=True)
+    assert o_err(o1, o2.cpu().double().numpy()) < 1e-3
+    assert s_err(s1, s2.cpu().double().numpy()) < 1e-3
