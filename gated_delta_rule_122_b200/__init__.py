@@ -1,7 +1,9 @@
 """B200-native KDA (Kimi Delta Attention): a CUDA library for sm_100a with a C ABI.
 
 Entry points (see include/kda.h): ``forward`` (chunkwise prefill),
-``forward_varlen`` (prefill over packed sequences of different lengths),
+``forward_varlen`` / ``forward_varlen_raw`` / ``forward_varlen_gdn2`` (prefill over
+packed sequences of different lengths), the same calls on host tensors go through the
+host-buffer entry points,
 ``forward_scalar_gate`` / ``decode_step_scalar_gate`` (one retention factor per
 head: Gated DeltaNet), ``forward_gdn2`` / ``decode_step_gdn2`` (decoupled erase
 and write gates: GDN-2), ``forward_raw`` / ``decode_step_raw`` (input
@@ -15,10 +17,11 @@ draws the seeded synthetic workloads.  All arithmetic runs in
 """
 from .kda import (EXPORTED_SYMBOLS, KDAError, decode_step, decode_step_gdn2, decode_step_raw,
                   decode_step_scalar_gate, decode_tokens, forward, forward_gdn2, forward_raw,
-                  forward_scalar_gate, forward_sequential, forward_varlen, library, library_path,
+                  forward_scalar_gate, forward_sequential, forward_varlen, forward_varlen_gdn2,
+                  forward_varlen_raw, library, library_path,
                   selftest_bounded_wait, state_copy, status_string, version)
 
-__all__ = ["forward", "forward_varlen", "forward_scalar_gate", "forward_gdn2", "forward_raw",
+__all__ = ["forward", "forward_varlen", "forward_varlen_raw", "forward_varlen_gdn2", "forward_scalar_gate", "forward_gdn2", "forward_raw",
            "forward_sequential", "decode_step", "decode_step_scalar_gate", "decode_step_gdn2",
            "decode_step_raw", "decode_tokens", "state_copy", "selftest_bounded_wait", "KDAError", "library",
            "library_path",

@@ -55,6 +55,11 @@ kda_status check_forward(const void *q, const void *k, const void *v, const void
     return KDA_OK;
 }
 
+constexpr int kVarlenKda = 0, kVarlenRaw = 1, kVarlenGdn2 = 2;
+kda_status check_gdn2(const void *q, const void *k, const void *v, const void *alpha, const void *erase,
+                      const void *wgate, const float *s_in, const void *o, const float *s_out, int B, int T, int H,
+                      int dk, int dv, kda_dtype qkv, kda_dtype gate, kda_dtype out);
+
 // T = 0: the final state is the initial state (or zeros).
 kda_status empty_sequence(const float *s_in, float *s_out, int B, int H, int dk, int dv,
                           cudaStream_t stream)
@@ -175,17 +180,25 @@ kda_status kda_forward(const void *q, const void *k, const void *v, const void *
                                   stream);
 }
 
-kda_status kda_forward_varlen(const void *q, const void *k, const void *v, const void *alpha,
-                              const void *beta, const int *cu_seqlens, const float *initial_state,
-                              void *o, float *final_state, int N, int total_T, int H, int d_k,
-                              int d_v, float scale, kda_dtype qkv_dtype, kda_dtype gate_dtype,
-                              kda_dtype out_dtype, void *workspace, size_t workspace_bytes,
-                              cudaStream_t stream)
+}  // extern "C"
+
+namespace {
+
+// The packed-sequence prefill for every kind (KDA, raw inputs, GDN-2): checks, workspace,
+// then the launch.  For GDN-2, `beta` is the erase gate and `wgate` the write gate.
+kda_status varlen_prefill(int kind, const void *q, const void *k, const void *v, const void *alpha,
+                          const void *beta, const void *wgate, const int *cu_seqlens, const float *initial_state,
+                          void *o, float *final_state, int N, int total_T, int H, int d_k, int d_v, float scale,
+                          kda_dtype qkv_dtype, kda_dtype gate_dtype, kda_dtype out_dtype, void *workspace,
+                          size_t workspace_bytes, cudaStream_t stream)
 {
     if (N < 0) return KDA_ERR_SHAPE;
+    const bool gdn2 = kind == kVarlenGdn2;
     // the token tensors are one [1, total_T, H, d] batch; the states are per sequence
-    kda_status st = check_forward(q, k, v, alpha, beta, nullptr, o, nullptr, 1, total_T, H, d_k, d_v,
-                                  qkv_dtype, gate_dtype, out_dtype);
+    kda_status st = gdn2 ? check_gdn2(q, k, v, alpha, beta, wgate, nullptr, o, nullptr, 1, total_T, H, d_k, d_v,
+                                      qkv_dtype, gate_dtype, out_dtype)
+                         : check_forward(q, k, v, alpha, beta, nullptr, o, nullptr, 1, total_T, H, d_k, d_v,
+                                         qkv_dtype, gate_dtype, out_dtype);
     if (st != KDA_OK) return st;
     if (N * (long long)H == 0) return KDA_OK;
     if (!cu_seqlens) return KDA_ERR_NULL;
@@ -206,15 +219,58 @@ kda_status kda_forward_varlen(const void *q, const void *k, const void *v, const
     if (cudaMemsetAsync(workspace, 0, need, stream) != cudaSuccess) return KDA_ERR_LAUNCH;
     // no tokens at all: every sequence is empty (the offsets are all zero)
     if (total_T == 0) return empty_sequence(initial_state, final_state, N, H, d_k, d_v, stream);
-    kda::ChunkArgs a{q, k, v, alpha, beta, initial_state, final_state, o, N, total_T, H, scale,
+    kda::ChunkArgs a{q, k, v, alpha, gdn2 ? nullptr : beta, initial_state, final_state, o, N, total_T, H, scale,
                      qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16,
                      static_cast<unsigned int *>(workspace), cu_seqlens};
+    if (gdn2) {
+        a.erase = beta;
+        a.wgate = wgate;
+    }
+    a.raw_inputs = kind == kVarlenRaw ? 1 : 0;
     cudaError_t err;
     if (kda::chunk_tc_supported(d_k, d_v, qkv_dtype, gate_dtype))
         err = kda::launch_chunk_tc(a, d_k, d_v, stream);
     else
         err = kda::launch_chunk_simt(a, d_k, d_v, stream);
     return err == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status kda_forward_varlen(const void *q, const void *k, const void *v, const void *alpha,
+                              const void *beta, const int *cu_seqlens, const float *initial_state,
+                              void *o, float *final_state, int N, int total_T, int H, int d_k,
+                              int d_v, float scale, kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                              kda_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                              cudaStream_t stream)
+{
+    return varlen_prefill(kVarlenKda, q, k, v, alpha, beta, nullptr, cu_seqlens, initial_state, o, final_state, N,
+                          total_T, H, d_k, d_v, scale, qkv_dtype, gate_dtype, out_dtype, workspace, workspace_bytes,
+                          stream);
+}
+
+kda_status kda_forward_varlen_raw(const void *q, const void *k, const void *v, const void *gate_logit,
+                                  const void *beta_logit, const int *cu_seqlens, const float *initial_state,
+                                  void *o, float *final_state, int N, int total_T, int H, int d_k, int d_v,
+                                  float scale, kda_dtype qkv_dtype, kda_dtype gate_dtype, kda_dtype out_dtype,
+                                  void *workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    return varlen_prefill(kVarlenRaw, q, k, v, gate_logit, beta_logit, nullptr, cu_seqlens, initial_state, o,
+                          final_state, N, total_T, H, d_k, d_v, scale, qkv_dtype, gate_dtype, out_dtype, workspace,
+                          workspace_bytes, stream);
+}
+
+kda_status kda_forward_varlen_gdn2(const void *q, const void *k, const void *v, const void *alpha,
+                                   const void *erase, const void *write, const int *cu_seqlens,
+                                   const float *initial_state, void *o, float *final_state, int N, int total_T,
+                                   int H, int d_k, int d_v, float scale, kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                                   kda_dtype out_dtype, void *workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    return varlen_prefill(kVarlenGdn2, q, k, v, alpha, erase, write, cu_seqlens, initial_state, o, final_state, N,
+                          total_T, H, d_k, d_v, scale, qkv_dtype, gate_dtype, out_dtype, workspace, workspace_bytes,
+                          stream);
 }
 
 kda_status kda_forward_scalar_gate(const void *q, const void *k, const void *v, const void *alpha,
@@ -256,8 +312,12 @@ kda_status kda_decode_step_raw(const void *q, const void *k, const void *v, cons
     return kda::launch_recurrent(a, d_k, d_v, stream) == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
 }
 
+}  // extern "C"
+
+namespace {
+
 // GDN-2 entry points: the erase and write gates take the place of beta.
-static kda_status check_gdn2(const void *q, const void *k, const void *v, const void *alpha,
+kda_status check_gdn2(const void *q, const void *k, const void *v, const void *alpha,
                              const void *erase, const void *wgate, const float *s_in, const void *o,
                              const float *s_out, int B, int T, int H, int dk, int dv, kda_dtype qkv,
                              kda_dtype gate, kda_dtype out)
@@ -275,6 +335,10 @@ static kda_status check_gdn2(const void *q, const void *k, const void *v, const 
         return KDA_ERR_ALIAS;
     return KDA_OK;
 }
+
+}  // namespace
+
+extern "C" {
 
 kda_status kda_forward_gdn2(const void *q, const void *k, const void *v, const void *alpha,
                             const void *erase, const void *wgate, const float *initial_state, void *o,

@@ -15,7 +15,7 @@ import threading
 
 import torch
 
-__all__ = ["KDAError", "forward", "forward_varlen", "forward_scalar_gate", "forward_gdn2",
+__all__ = ["KDAError", "forward", "forward_varlen", "forward_varlen_raw", "forward_varlen_gdn2", "forward_scalar_gate", "forward_gdn2",
            "forward_raw", "forward_sequential", "decode_step", "decode_step_raw",
            "decode_step_scalar_gate", "decode_step_gdn2", "decode_tokens", "state_copy",
            "selftest_bounded_wait", "library",
@@ -27,7 +27,8 @@ _lib = None
 _lock = threading.Lock()
 
 EXPORTED_SYMBOLS = ("kda_forward", "kda_forward_workspace_bytes", "kda_workspace_status",
-                    "kda_forward_noalloc", "kda_noalloc_status", "kda_forward_varlen", "kda_forward_scalar_gate",
+                    "kda_forward_noalloc", "kda_noalloc_status", "kda_forward_varlen", "kda_forward_varlen_raw",
+                    "kda_forward_varlen_gdn2", "kda_forward_scalar_gate",
                     "kda_forward_gdn2", "kda_forward_raw", "kda_forward_sequential", "kda_decode_step",
                     "kda_decode_step_gdn2", "kda_decode_step_raw", "kda_decode_step_scalar_gate",
                     "kda_decode_tokens", "kda_state_copy", "kda_selftest_bounded_wait", "kda_status_string",
@@ -73,6 +74,11 @@ def library() -> ctypes.CDLL:
             lib.kda_forward_varlen.argtypes = [_vp] * 9 + [_i] * 5 + [_f] + [_i] * 3 + \
                 [_vp, ctypes.c_size_t, _vp]
             lib.kda_forward_varlen.restype = _i
+            lib.kda_forward_varlen_raw.argtypes = lib.kda_forward_varlen.argtypes
+            lib.kda_forward_varlen_raw.restype = _i
+            lib.kda_forward_varlen_gdn2.argtypes = [_vp] * 10 + [_i] * 5 + [_f] + [_i] * 3 + \
+                [_vp, ctypes.c_size_t, _vp]
+            lib.kda_forward_varlen_gdn2.restype = _i
             lib.kda_forward_scalar_gate.argtypes = fwd_args + [_vp, ctypes.c_size_t, _vp]
             lib.kda_forward_scalar_gate.restype = _i
             lib.kda_forward_raw.argtypes = fwd_args + [_vp, ctypes.c_size_t, _vp]
@@ -416,37 +422,38 @@ def decode_step_raw(q, k, v, gate_logit, beta_logit, state, scale=None, out_dtyp
     return _decode("kda_decode_step_raw", q, k, v, gate_logit, beta_logit, state, scale, out_dtype, out)
 
 
-def forward_varlen(q, k, v, alpha, beta, cu_seqlens, initial_state=None, scale=None,
-                   output_final_state=True, out_dtype=torch.float32, out=None, final_state=None,
-                   workspace=None, check_status=False):
-    """Prefill over packed sequences of different lengths (C entry point ``kda_forward_varlen``).
-
-    q, k, alpha: [total_T,H,dk] (or [1,total_T,H,dk]); v: [total_T,H,dv]; beta: [total_T,H];
-    cu_seqlens: int32 [N+1] on the same device (0, then cumulative lengths).  initial_state:
-    float32 [N,H,dk,dv] or None.  check_status=True synchronizes and raises KDAError on
-    invalid offsets or a timed-out device wait.  Returns (o [total_T,H,dv], final_state or None).
-    """
+def _varlen(fn, q, k, v, alpha, beta, write, cu_seqlens, initial_state, scale, output_final_state, out_dtype,
+            out, final_state, workspace, check_status):
+    """Shared marshalling of the packed-sequence prefills (C function ``fn``); for GDN-2
+    ``beta`` is the erase gate and ``write`` the write gate."""
     device = q.device
     if device.type != "cuda":
         raise ValueError("KDA runs on CUDA devices only")
+    gdn2 = write is not None
     squeeze = q.dim() == 4
     if squeeze:
         if q.shape[0] != 1:
             raise ValueError("packed tensors are [total_T,H,d] or [1,total_T,H,d]")
         q, k, v, alpha, beta = (t[0] for t in (q, k, v, alpha, beta))
+        if gdn2:
+            write = write[0]
     total_T, H, dk = q.shape
     dv = v.shape[-1]
     for name, t in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta", beta),
-                    ("cu_seqlens", cu_seqlens)):
+                    ("cu_seqlens", cu_seqlens)) + ((("write", write),) if gdn2 else ()):
         _check(name, t, device)
     if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
         raise ValueError("cu_seqlens must be a 1-D int32 tensor [N+1]")
     N = cu_seqlens.numel() - 1
+    b_shape = (total_T, H, dk) if gdn2 else (total_T, H)
     if tuple(k.shape) != (total_T, H, dk) or tuple(alpha.shape) != (total_T, H, dk) or \
-            tuple(v.shape) != (total_T, H, dv) or tuple(beta.shape) != (total_T, H):
-        raise ValueError("shapes: q,k,alpha [total_T,H,dk], v [total_T,H,dv], beta [total_T,H]")
-    if k.dtype != q.dtype or v.dtype != q.dtype or alpha.dtype != beta.dtype:
-        raise TypeError("q/k/v and alpha/beta must each share a dtype")
+            tuple(v.shape) != (total_T, H, dv) or tuple(beta.shape) != b_shape or \
+            (gdn2 and tuple(write.shape) != (total_T, H, dv)):
+        raise ValueError("shapes: q,k,alpha [total_T,H,dk], v [total_T,H,dv], " +
+                         ("erase [total_T,H,dk], write [total_T,H,dv]" if gdn2 else "beta [total_T,H]"))
+    if k.dtype != q.dtype or v.dtype != q.dtype or alpha.dtype != beta.dtype or \
+            (gdn2 and write.dtype != alpha.dtype):
+        raise TypeError("q/k/v and the gates must each share a dtype")
     if initial_state is not None:
         _check("initial_state", initial_state, device)
         if initial_state.dtype != torch.float32 or tuple(initial_state.shape) != (N, H, dk, dv):
@@ -467,16 +474,49 @@ def forward_varlen(q, k, v, alpha, beta, cu_seqlens, initial_state=None, scale=N
         ws = workspace
         if ws is None or ws.numel() * ws.element_size() < ws_bytes:
             ws = torch.empty(max(ws_bytes, 16), device=device, dtype=torch.uint8)
-        code = lib.kda_forward_varlen(
-            _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(cu_seqlens),
+        gates = (_ptr(alpha), _ptr(beta), _ptr(write)) if gdn2 else (_ptr(alpha), _ptr(beta))
+        code = getattr(lib, fn)(
+            _ptr(q), _ptr(k), _ptr(v), *gates, _ptr(cu_seqlens),
             _ptr(initial_state), _ptr(out), _ptr(final_state), N, total_T, H, dk, dv,
             float(scale), _DT[q.dtype], _dt(alpha, "alpha"), _dt(out, "out"), _ptr(ws),
             ws.numel() * ws.element_size(), stream)
         if code == 0 and check_status:
             code = lib.kda_workspace_status(_ptr(ws), stream)
     if code != 0:
-        raise KDAError("kda_forward_varlen", code)
+        raise KDAError(fn, code)
     return (out.unsqueeze(0) if squeeze else out), final_state
+
+
+def forward_varlen(q, k, v, alpha, beta, cu_seqlens, initial_state=None, scale=None,
+                   output_final_state=True, out_dtype=torch.float32, out=None, final_state=None,
+                   workspace=None, check_status=False):
+    """Prefill over packed sequences of different lengths (C entry point ``kda_forward_varlen``).
+
+    q, k, alpha: [total_T,H,dk] (or [1,total_T,H,dk]); v: [total_T,H,dv]; beta: [total_T,H];
+    cu_seqlens: int32 [N+1] on the same device (0, then cumulative lengths).  initial_state:
+    float32 [N,H,dk,dv] or None.  check_status=True synchronizes and raises KDAError on
+    invalid offsets or a timed-out device wait.  Returns (o [total_T,H,dv], final_state or None).
+    """
+    return _varlen("kda_forward_varlen", q, k, v, alpha, beta, None, cu_seqlens, initial_state, scale,
+                   output_final_state, out_dtype, out, final_state, workspace, check_status)
+
+
+def forward_varlen_raw(q, k, v, gate_logit, beta_logit, cu_seqlens, initial_state=None, scale=None,
+                       output_final_state=True, out_dtype=torch.float32, out=None, final_state=None,
+                       workspace=None, check_status=False):
+    """Packed-sequence prefill on raw inputs (C entry point ``kda_forward_varlen_raw``): the
+    preprocessing of ``forward_raw`` with the layouts of ``forward_varlen``."""
+    return _varlen("kda_forward_varlen_raw", q, k, v, gate_logit, beta_logit, None, cu_seqlens, initial_state,
+                   scale, output_final_state, out_dtype, out, final_state, workspace, check_status)
+
+
+def forward_varlen_gdn2(q, k, v, alpha, erase, write, cu_seqlens, initial_state=None, scale=None,
+                        output_final_state=True, out_dtype=torch.float32, out=None, final_state=None,
+                        workspace=None, check_status=False):
+    """Packed-sequence GDN-2 prefill (C entry point ``kda_forward_varlen_gdn2``): erase
+    [total_T,H,dk] and write [total_T,H,dv] gates in place of beta; otherwise ``forward_varlen``."""
+    return _varlen("kda_forward_varlen_gdn2", q, k, v, alpha, erase, write, cu_seqlens, initial_state, scale,
+                   output_final_state, out_dtype, out, final_state, workspace, check_status)
 
 
 def forward_gdn2(q, k, v, alpha, erase, write, initial_state=None, scale=None, output_final_state=True,

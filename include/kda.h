@@ -180,6 +180,37 @@ kda_status kda_forward_varlen(const void *q, const void *k, const void *v,
                               size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * kda_forward_varlen_raw -- kda_forward_varlen on raw inputs: the preprocessing of
+ * kda_forward_raw (q, k divided by their row norms in the kernel, gate logits
+ * [total_T, H, d_k] with alpha = 1 / (1 + e^x), beta logits [total_T, H] with beta =
+ * sigmoid(y)) over packed sequences.  Other arguments, layouts and errors as
+ * kda_forward_varlen.
+ */
+kda_status kda_forward_varlen_raw(const void *q, const void *k, const void *v,
+                                  const void *gate_logit, const void *beta_logit,
+                                  const int *cu_seqlens, const float *initial_state,
+                                  void *o, float *final_state, int N, int total_T,
+                                  int H, int d_k, int d_v, float scale,
+                                  kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                                  kda_dtype out_dtype, void *workspace,
+                                  size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * kda_forward_varlen_gdn2 -- kda_forward_gdn2 over packed sequences: erase [total_T, H,
+ * d_k] and write [total_T, H, d_v] gates (16-byte aligned) in place of beta.  Other
+ * arguments, layouts and errors as kda_forward_varlen.
+ */
+kda_status kda_forward_varlen_gdn2(const void *q, const void *k, const void *v,
+                                   const void *alpha, const void *erase,
+                                   const void *write, const int *cu_seqlens,
+                                   const float *initial_state, void *o,
+                                   float *final_state, int N, int total_T, int H,
+                                   int d_k, int d_v, float scale,
+                                   kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                                   kda_dtype out_dtype, void *workspace,
+                                   size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * kda_forward_scalar_gate -- kda_forward with one retention factor per (token,
  * head): Gated DeltaNet, S~_t = alpha_t S_{t-1} with a scalar alpha_t, which is
  * KDA with alpha_t broadcast over the key channels ("From Fast Weight
@@ -212,8 +243,9 @@ kda_status kda_forward_scalar_gate(const void *q, const void *k, const void *v,
  * w_t = beta_t 1 give kda_forward.  Arguments as kda_forward with
  *   erase [B, T, H, d_k] and write [B, T, H, d_v]  (gate_dtype, 16-byte
  *   aligned) in place of beta.
- * Computed by the chunkwise schedule on CUDA cores, fp32, every supported head
- * size and dtype.
+ * Computed by the chunkwise schedule on the tensor cores for d_k = d_v = 128 with
+ * bf16 inputs and gates, on CUDA cores in fp32 for every other supported shape and
+ * dtype.
  */
 kda_status kda_forward_gdn2(const void *q, const void *k, const void *v,
                             const void *alpha, const void *erase,

@@ -203,3 +203,22 @@ def test_host_path_rejects_bad_arguments(lib):
              0x100000, 1 << 20, None) == ERR_NULL
     assert d(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 0x70000, 0x60000, 2, 1, 16, 16, 1.0, 0, 0, 0,
              None, 0, None) == ERR_WS
+
+
+def test_varlen_raw_and_gdn2_reject_bad_arguments(lib):
+    def r(N=2, cu=0xB0000, dk=16, ws=0x90000):
+        return lib.kda_forward_varlen_raw(0x10000, 0x20000, 0x30000, 0x40000, 0x50000, cu, None, 0x60000, None,
+                                          N, 8, 1, dk, 16, 1.0, 0, 0, 0, ws, 16, None)
+    assert r(N=-1) == ERR_SHAPE
+    assert r(cu=None) == ERR_NULL
+    assert r(dk=40) == ERR_UNSUP
+    assert r(ws=None) == ERR_WS
+    assert r(N=0) == OK
+
+    def g(w=0x70000, e=0x50000, o=0x60000, cu=0xB0000):
+        return lib.kda_forward_varlen_gdn2(0x10000, 0x20000, 0x30000, 0x40000, e, w, cu, None, o, None,
+                                           2, 8, 1, 16, 16, 1.0, 0, 0, 0, 0x90000, 16, None)
+    assert g(w=None) == ERR_NULL
+    assert g(e=0x50004) == ERR_ALIGN                        # the erase gate needs 16-byte rows
+    assert g(o=0x70000 + 64) == ERR_ALIAS                   # o overlaps the write gate
+    assert g(cu=None) == ERR_NULL

@@ -107,3 +107,66 @@ def test_varlen_invalid_offsets_reported(bad):
                            torch.tensor(bad, dtype=torch.int32, device="cuda"), initial_state=s0.cuda(),
                            scale=scale, check_status=True)
     assert e.value.code == 2   # KDA_ERR_SHAPE
+
+
+def _packed_extra(name, lengths, H, seed, **over):
+    p, cu, s0, scale = _packed(name, lengths, H, **over)
+    g = torch.Generator().manual_seed(seed)
+    return p, cu, s0, scale, g
+
+
+@pytest.mark.parametrize("name,lengths,over,tol", [
+    ("long", [40, 0, 33, 1, 96, 31], {}, TOL_BF16),                          # tensor cores
+    ("small", [20, 0, 33, 5], dict(qkv_dtype=torch.float32), TOL_F32),       # CUDA cores
+])
+def test_varlen_raw_matches_oracle(name, lengths, over, tol):
+    """Raw inputs over packed sequences: rows of q, k rescaled, gate and beta logits whose
+    maps give the workload's alpha and beta; each sequence against the oracle's fp64
+    preprocessing and recurrence."""
+    p, cu, s0, scale, g = _packed_extra(name, lengths, 3, 41, **over)
+    cq = torch.exp(torch.randn(*p["q"].shape[:-1], 1, generator=g))
+    ck = torch.exp(torch.randn(*p["k"].shape[:-1], 1, generator=g))
+    a = p["alpha"].double().clamp(1e-30, 1 - 1e-7)
+    bb = p["beta"].double().clamp(1e-7, 1 - 1e-7)
+    r = dict(q=(cq * p["q"].float()).to(p["q"].dtype), k=(ck * p["k"].float()).to(p["k"].dtype), v=p["v"],
+             x=torch.log((1 - a) / a).to(p["alpha"].dtype), y=torch.log(bb / (1 - bb)).to(p["beta"].dtype))
+    outs, states = [], []
+    for i in range(len(cu) - 1):
+        lo, hi = int(cu[i]), int(cu[i + 1])
+        sl = lambda t: t[lo:hi].unsqueeze(0)
+        o_i, S_i = oracle.forward_raw(sl(r["q"]), sl(r["k"]), sl(r["v"]), sl(r["x"]), sl(r["y"]),
+                                      s0=s0[i:i + 1], scale=scale)
+        outs.append(o_i[0])
+        states.append(S_i[0])
+    o_ref, s_ref = np.concatenate(outs, 0), np.stack(states, 0)
+    c = lambda t: t.cuda()
+    o, S = kda.forward_varlen_raw(c(r["q"]), c(r["k"]), c(r["v"]), c(r["x"]), c(r["y"]),
+                                  torch.from_numpy(cu).cuda(), initial_state=s0.cuda(), scale=scale,
+                                  check_status=True)
+    eo, es = o_err(o, o_ref), s_err(S, s_ref)
+    assert eo < tol and es < tol, f"o {eo:.3e} state {es:.3e}"
+
+
+@pytest.mark.parametrize("name,lengths,over,tol", [
+    ("long", [50, 0, 32, 1, 100, 7], {}, TOL_BF16),                          # tensor cores
+    ("small", [20, 0, 33, 5], dict(qkv_dtype=torch.float32), TOL_F32),       # CUDA cores
+])
+def test_varlen_gdn2_matches_oracle(name, lengths, over, tol):
+    p, cu, s0, scale, g = _packed_extra(name, lengths, 2, 43, **over)
+    er = torch.sigmoid(torch.randn(*p["k"].shape, generator=g)).to(p["alpha"].dtype)
+    wr = torch.sigmoid(torch.randn(*p["v"].shape, generator=g)).to(p["alpha"].dtype)
+    outs, states = [], []
+    for i in range(len(cu) - 1):
+        lo, hi = int(cu[i]), int(cu[i + 1])
+        sl = lambda t: t[lo:hi].unsqueeze(0)
+        o_i, S_i = oracle.forward_gdn2(sl(p["q"]), sl(p["k"]), sl(p["v"]), sl(p["alpha"]), sl(er), sl(wr),
+                                       s0=s0[i:i + 1], scale=scale)
+        outs.append(o_i[0])
+        states.append(S_i[0])
+    o_ref, s_ref = np.concatenate(outs, 0), np.stack(states, 0)
+    d = {n: t.cuda() for n, t in p.items()}
+    o, S = kda.forward_varlen_gdn2(d["q"], d["k"], d["v"], d["alpha"], er.cuda(), wr.cuda(),
+                                   torch.from_numpy(cu).cuda(), initial_state=s0.cuda(), scale=scale,
+                                   check_status=True)
+    eo, es = o_err(o, o_ref), s_err(S, s_ref)
+    assert eo < tol and es < tol, f"o {eo:.3e} state {es:.3e}"
