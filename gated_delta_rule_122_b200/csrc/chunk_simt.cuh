@@ -60,8 +60,9 @@ struct SimtLayout {
     static constexpr int oV = oW + C * PK;
     static constexpr int oE = oV + C * PV;
     static constexpr int oS = oE + C * PV;
-    static constexpr int oAkk = oS + DK * DV;
-    static constexpr int oAqk = oAkk + C * PC;
+    static constexpr int PT = C + 4;              // row pitch of A_kk^T (16-byte rows)
+    static constexpr int oAkk = oS + DK * DV;     // A_kk^T: column s of A_kk as row s
+    static constexpr int oAqk = oAkk + C * PT;
     static constexpr int oBeta = oAqk + C * PC;
     static constexpr int oNrm = oBeta + C;      // 1/||q_r||, 1/||k_r|| (raw inputs)
     static constexpr int floats = oNrm + 2 * C;
@@ -163,19 +164,19 @@ kda_chunk_simt_kernel(ChunkArgs a)
             float akk = 0.f, aqk = 0.f;
             if (s <= r) {
                 for (int d = 0; d < DK; ++d) {
-                    const float ks = K[s * PK + d] * expf(G[r * PK + d] - G[s * PK + d]);
+                    const float ks = K[s * PK + d] * __expf(G[r * PK + d] - G[s * PK + d]);
                     akk = fmaf(kGdn2 ? W[r * PK + d] : K[r * PK + d], ks, akk);
                     aqk = fmaf(Q[r * PK + d], ks, aqk);
                 }
             }
-            Akk[r * PC + s] = (s < r) ? (kGdn2 ? akk : Bt[r] * akk) : 0.f;
+            Akk[s * Ly::PT + r] = (s < r) ? (kGdn2 ? akk : Bt[r] * akk) : 0.f;
             Aqk[r * PC + s] = aqk;
         }
         if constexpr (kGdn2) __syncthreads();   // the Akk loop above read W
         for (int idx = tid; idx < C * DK; idx += NT) {
             const int r = idx / DK, d = idx % DK;
-            if constexpr (kGdn2) W[r * PK + d] *= expf(G[r * PK + d]);
-            else W[r * PK + d] = Bt[r] * K[r * PK + d] * expf(G[r * PK + d]);
+            if constexpr (kGdn2) W[r * PK + d] *= __expf(G[r * PK + d]);
+            else W[r * PK + d] = Bt[r] * K[r * PK + d] * __expf(G[r * PK + d]);
         }
         for (int idx = tid; idx < C * DV; idx += NT) {
             const int r = idx / DV, j = idx % DV;
@@ -188,8 +189,11 @@ kda_chunk_simt_kernel(ChunkArgs a)
         }
         __syncthreads();
 
-        // 4. forward substitution (I + Akk) X = RHS, one column per thread;
-        //    then the decay-scaled operands of the inter-chunk products
+        // 4. forward substitution (I + Akk) X = RHS, one column per thread, right-looking:
+        //    once x_j is final it is subtracted from every later row, so the 31 updates of
+        //    a step are independent and column j of A_kk is read as 16-byte vectors (row j
+        //    of the transposed copy); then the decay-scaled operands of the inter-chunk
+        //    products
         for (int col = tid; col < DK + DV; col += NT) {
             float *X = (col < DK) ? (W + col) : (V + (col - DK));
             const int stride = (col < DK) ? PK : PV;
@@ -197,11 +201,16 @@ kda_chunk_simt_kernel(ChunkArgs a)
 #pragma unroll
             for (int i = 0; i < C; ++i) x[i] = X[i * stride];
 #pragma unroll
-            for (int i = 1; i < C; ++i) {
-                float acc = x[i];
+            for (int j = 0; j < C - 1; ++j) {
+                const float xj = x[j];
 #pragma unroll
-                for (int j = 0; j < i; ++j) acc = fmaf(-Akk[i * PC + j], x[j], acc);
-                x[i] = acc;
+                for (int i4 = (j + 1) / 4; i4 < C / 4; ++i4) {
+                    const float4 a = *reinterpret_cast<const float4 *>(Akk + j * Ly::PT + 4 * i4);
+                    if (4 * i4 + 0 > j) x[4 * i4 + 0] = fmaf(-a.x, xj, x[4 * i4 + 0]);
+                    if (4 * i4 + 1 > j) x[4 * i4 + 1] = fmaf(-a.y, xj, x[4 * i4 + 1]);
+                    if (4 * i4 + 2 > j) x[4 * i4 + 2] = fmaf(-a.z, xj, x[4 * i4 + 2]);
+                    if (4 * i4 + 3 > j) x[4 * i4 + 3] = fmaf(-a.w, xj, x[4 * i4 + 3]);
+                }
             }
 #pragma unroll
             for (int i = 0; i < C; ++i) X[i * stride] = x[i];
@@ -210,8 +219,8 @@ kda_chunk_simt_kernel(ChunkArgs a)
         for (int idx = tid; idx < C * DK; idx += NT) {
             const int r = idx / DK, d = idx % DK;
             const float g = G[r * PK + d];
-            Q[r * PK + d] *= expf(g);                              // q * gamma_r
-            K[r * PK + d] *= expf(G[(C - 1) * PK + d] - g);        // k * gamma_end / gamma_r
+            Q[r * PK + d] *= __expf(g);                            // q * gamma_r
+            K[r * PK + d] *= __expf(G[(C - 1) * PK + d] - g);      // k * gamma_end / gamma_r
         }
         __syncthreads();
 
@@ -255,7 +264,7 @@ kda_chunk_simt_kernel(ChunkArgs a)
 #pragma unroll
             for (int g = 0; g < SG; ++g) {
                 const int i = rgrp + NRG * (m0 + g);
-                acc[g] = S[i * DV + jcol] * expf(G[(C - 1) * PK + i]);
+                acc[g] = S[i * DV + jcol] * __expf(G[(C - 1) * PK + i]);
             }
             for (int r = 0; r < C; ++r) {
                 const float erj = E[r * PV + jcol];
