@@ -40,12 +40,14 @@ if ROOT not in sys.path:
 
 METRIC = "KDA prefill Mtokens/s (H=64,d=128); decode-step HBM GB/s vs ~8 TB/s peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of the prefill
-# kernel (1.08 GB read + 0.5087 GB written), from the capture summarised under
-# profiles/, with the hash of the kernel sources it was taken for: once the
-# sources change, the line reports traffic as null until it is captured again.
-PREFILL_TRAFFIC_BYTES = 1_588_670_000
-PREFILL_TRAFFIC_SOURCES = "01c9f9f2031d0f2b"
+# ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch of the prefill
+# kernel on the prefill workload (1.0831 GB read + 0.5106 GB written) and on the long
+# workload (4.3137 GB + 2.1217 GB), from the captures summarised under profiles/, with
+# the hash of the kernel sources they were taken for: once the sources change, the
+# line reports traffic as null until it is captured again.
+PREFILL_TRAFFIC_BYTES = 1_083_118_080 + 510_573_312
+LONG_TRAFFIC_BYTES = 4_313_738_240 + 2_121_667_840
+PREFILL_TRAFFIC_SOURCES = "f31e3e424745f84e"
 
 
 def kernel_sources_hash() -> str:
@@ -143,6 +145,7 @@ def measure_long(torch, kda, device, hbm):
                         "initial state, 30% strong-forget channels", "ms": ms,
             "mtokens_s": w.B * w.T / (ms * 1e-3) / 1e6,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "traffic": LONG_TRAFFIC_BYTES if kernel_sources_hash() == PREFILL_TRAFFIC_SOURCES else None,
                          "algorithmic_bytes": nbytes}}
 
 
