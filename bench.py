@@ -170,10 +170,17 @@ def measure_rows(torch, kda, x, y, wp, hbm):
     from gated_delta_rule_122_b200.inputs import make_inputs, workload
     ws_ = workload("small")
     xs = make_inputs(ws_, device=dev)
-    ms = time_call(torch, lambda: kda.forward(xs["q"], xs["k"], xs["v"], xs["alpha"], xs["beta"],
-                                              initial_state=xs["s0"], scale=xs["scale"]))
-    row("small_prefill", f"B={ws_.B} T={ws_.T} H={ws_.H} d={ws_.dk}, bf16 q/k/v, fp32 alpha/beta, initial state",
-        ms, prefill_bytes(ws_, True), ws_.B * ws_.T)
+    small = f"B={ws_.B} T={ws_.T} H={ws_.H} d={ws_.dk}, bf16 q/k/v, fp32 alpha/beta, initial state"
+    run_small = lambda: kda.forward(xs["q"], xs["k"], xs["v"], xs["alpha"], xs["beta"],
+                                    initial_state=xs["s0"], scale=xs["scale"])
+    # the library's own choice for 4 (sequence, head) pairs: the column scan
+    ms = time_call(torch, run_small)
+    row("small_prefill", small + f", schedule {kda.get_schedule()} (column scan)", ms,
+        prefill_bytes(ws_, True), ws_.B * ws_.T)
+    with kda.schedule("chunked"):   # the CUDA-core chunk kernel on the same input
+        ms = time_call(torch, run_small)
+    row("small_prefill_chunked", small + ", chunkwise schedule (CUDA-core chunk kernel)", ms,
+        prefill_bytes(ws_, True), ws_.B * ws_.T)
     del xs
     o = torch.empty((B, T, H, dv), device=dev)
     S = torch.empty((B, H, dk, dv), device=dev)
@@ -206,13 +213,13 @@ def measure_rows(torch, kda, x, y, wp, hbm):
                                                      scale=x["scale"], out=ov, final_state=Sv))
     row("varlen_prefill", f"{B * T} tokens as sequences {lengths}, H={H} d={dk} bf16", ms,
         tok_heads * 1538 + len(lengths) * H * dk * dv * 4, B * T)
-    # GDN-2 (CUDA-core chunk kernel): erase [.., d_k] and write [.., d_v] gates in place of beta
+    # GDN-2 (tensor-core chunk kernel): erase [.., d_k] and write [.., d_v] gates in place of beta
     g = torch.Generator(device=dev).manual_seed(7)
     er = torch.sigmoid(torch.randn(x["k"].shape, generator=g, device=dev)).to(torch.bfloat16)
     wr = torch.sigmoid(torch.randn(x["v"].shape, generator=g, device=dev)).to(torch.bfloat16)
     ms = time_call(torch, lambda: kda.forward_gdn2(x["q"], x["k"], x["v"], x["alpha"], er, wr, scale=x["scale"],
-                                                   out=o, final_state=S), reps=2, warmup=1)
-    row("gdn2_prefill", f"B={B} T={T} H={H} d={dk} bf16, erase/write gates (CUDA-core kernel)", ms,
+                                                   out=o, final_state=S))
+    row("gdn2_prefill", f"B={B} T={T} H={H} d={dk} bf16, erase/write gates (tensor-core kernel)", ms,
         tok_heads * (6 * 256 + 512) + state, B * T)
     del er, wr
     if y is not None:

@@ -2,6 +2,8 @@
 // caller's stream.  Nothing here allocates, synchronizes or throws.
 #include <stdint.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -9,6 +11,9 @@
 namespace {
 
 constexpr size_t kKdaWorkspaceBytes = 16;   // device status word (+ padding)
+
+// The process-wide prefill schedule (kda_set_schedule).
+std::atomic<int> g_schedule{KDA_SCHEDULE_AUTO};
 
 bool head_size_ok(int d) { return d >= 16 && d <= 128 && d % 16 == 0; }
 bool dtype_ok(kda_dtype t) { return t == KDA_F32 || t == KDA_BF16; }
@@ -96,12 +101,17 @@ kda_status prefill_launch(int kind, const void *q, const void *k, const void *v,
                 qkv_dtype == KDA_BF16, gate_dtype == KDA_BF16, out_dtype == KDA_BF16, status};
     a.gate_per_head = per_head ? 1 : 0;
     a.raw_inputs = kind == KDA_HOST_RAW ? 1 : 0;
-    cudaError_t err;
-    if (chunk_tc_supported(d_k, d_v, qkv_dtype, gate_dtype))
-        err = launch_chunk_tc(a, d_k, d_v, stream);
-    else
-        err = launch_chunk_simt(a, d_k, d_v, stream);
-    return err == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+    return launch_prefill(a, d_k, d_v, qkv_dtype, gate_dtype, stream) == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+}
+
+cudaError_t launch_prefill(const ChunkArgs &a, int dk, int dv, kda_dtype qkv, kda_dtype gate, cudaStream_t s)
+{
+    const int sched = g_schedule.load(std::memory_order_relaxed);
+    const bool tc = chunk_tc_supported(dk, dv, qkv, gate);
+    if (sched != KDA_SCHEDULE_CHUNKED && scan_supported(a) &&
+        (sched == KDA_SCHEDULE_SCAN || scan_preferred(a, dk, dv, tc)))
+        return launch_scan(a, dk, dv, s);
+    return tc ? launch_chunk_tc(a, dk, dv, s) : launch_chunk_simt(a, dk, dv, s);
 }
 
 }  // namespace kda
@@ -145,11 +155,22 @@ const char *kda_status_string(kda_status s)
     case KDA_ERR_LAUNCH: return "CUDA launch failed";
     case KDA_ERR_TIMEOUT: return "a bounded device-side wait timed out";
     case KDA_ERR_ALIAS: return "an output overlaps an input";
+    case KDA_ERR_VALUE: return "an enumerated argument has an unknown value";
     }
     return "unknown status";
 }
 
 int kda_version(void) { return 100; }
+
+kda_status kda_set_schedule(int schedule)
+{
+    if (schedule != KDA_SCHEDULE_AUTO && schedule != KDA_SCHEDULE_CHUNKED && schedule != KDA_SCHEDULE_SCAN)
+        return KDA_ERR_VALUE;
+    g_schedule.store(schedule, std::memory_order_relaxed);
+    return KDA_OK;
+}
+
+int kda_get_schedule(void) { return g_schedule.load(std::memory_order_relaxed); }
 
 size_t kda_forward_workspace_bytes(int B, int T, int H, int d_k, int d_v)
 {
@@ -227,12 +248,7 @@ kda_status varlen_prefill(int kind, const void *q, const void *k, const void *v,
         a.wgate = wgate;
     }
     a.raw_inputs = kind == kVarlenRaw ? 1 : 0;
-    cudaError_t err;
-    if (kda::chunk_tc_supported(d_k, d_v, qkv_dtype, gate_dtype))
-        err = kda::launch_chunk_tc(a, d_k, d_v, stream);
-    else
-        err = kda::launch_chunk_simt(a, d_k, d_v, stream);
-    return err == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
+    return kda::launch_prefill(a, d_k, d_v, qkv_dtype, gate_dtype, stream) == cudaSuccess ? KDA_OK : KDA_ERR_LAUNCH;
 }
 
 }  // namespace

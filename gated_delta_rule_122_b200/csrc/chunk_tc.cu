@@ -1135,13 +1135,13 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
         // ---- I: X = S' + E^T R -> the next S' (or the final state); outputs of chunk c
         if (!ptx::mbar_wait(bars.s, (uint32_t)(c & 1), kWaitLimitNs)) *err_flag = 1;
         ptx::tc_fence_after();
-        // R of chunk c+2 first (the update of chunk c has read R(c)): the A product of
-        // chunk c+2 can then start while the state is rewritten
-        if (c + 2 < nchunks) {
+        const bool xn = c + 1 < nchunks && chunk_is_extreme(sm, c + 1);
+        // R of chunk c+2 (the update of chunk c has read R(c)) is written after the state
+        // rewrite below, which is on the chain; before a token-by-token chunk, here
+        if (xc && c + 2 < nchunks) {
             stage_b(sm, c + 2, warp, lane, ie);
             warp_signal_after_stage(bars, c + 2, lane);
         }
-        const bool xn = c + 1 < nchunks && chunk_is_extreme(sm, c + 1);
         if (xc) {
             // outputs stored token by token; the staging rows (read by every warp's stage A
             // above, and by the previous chunk's output store) are then free for chunk c+3
@@ -1207,6 +1207,10 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             warp_signal(bars.rs, lane);
+            if (c + 2 < nchunks) {   // R of chunk c+2, once S' is out
+                stage_b(sm, c + 2, warp, lane, ie);
+                warp_signal_after_stage(bars, c + 2, lane);
+            }
         } else if (p.s_out) {
             const float *cend = reinterpret_cast<const float *>(sm + OFF_CST + (c % kCstSlots) * CST_BYTES) + D;
 #pragma unroll 1

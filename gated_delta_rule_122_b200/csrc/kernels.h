@@ -88,6 +88,16 @@ cudaError_t launch_chunk_simt(const ChunkArgs &a, int dk, int dv, cudaStream_t s
 // (both take GDN-2 gates when a.erase is set)
 bool chunk_tc_supported(int dk, int dv, kda_dtype qkv, kda_dtype gate);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, int dk, int dv, cudaStream_t s);
+// The column-scan prefill (one 8-lane group per value column, token by token): plain KDA
+// and the per-head gate, no raw inputs or GDN-2 gates.  scan_preferred: the automatic
+// schedule takes the scan over the chunk kernel that would run otherwise (tc: the
+// tensor-core one).
+bool scan_supported(const ChunkArgs &a);
+bool scan_preferred(const ChunkArgs &a, int dk, int dv, bool tc);
+cudaError_t launch_scan(const ChunkArgs &a, int dk, int dv, cudaStream_t s);
+// The prefill launch chosen for a's variant and shape under the process-wide schedule
+// setting: the column scan, the tensor-core chunk kernel or the CUDA-core one.
+cudaError_t launch_prefill(const ChunkArgs &a, int dk, int dv, kda_dtype qkv, kda_dtype gate, cudaStream_t s);
 
 // The dense prefill (kind: KDA_HOST_FORWARD, KDA_HOST_SCALAR_GATE or KDA_HOST_RAW) after
 // the workspace handling: argument checks, T = 0, the launch; status cleared by the caller.

@@ -18,7 +18,7 @@ import torch
 __all__ = ["KDAError", "forward", "forward_varlen", "forward_varlen_raw", "forward_varlen_gdn2", "forward_scalar_gate", "forward_gdn2",
            "forward_raw", "forward_sequential", "decode_step", "decode_step_raw",
            "decode_step_scalar_gate", "decode_step_gdn2", "decode_tokens", "state_copy",
-           "selftest_bounded_wait", "library",
+           "selftest_bounded_wait", "set_schedule", "get_schedule", "schedule", "library",
            "library_path", "status_string", "version", "EXPORTED_SYMBOLS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -33,7 +33,7 @@ EXPORTED_SYMBOLS = ("kda_forward", "kda_forward_workspace_bytes", "kda_workspace
                     "kda_decode_step_gdn2", "kda_decode_step_raw", "kda_decode_step_scalar_gate",
                     "kda_decode_tokens", "kda_state_copy", "kda_selftest_bounded_wait", "kda_status_string",
                     "kda_version", "kda_forward_host", "kda_forward_host_workspace_bytes", "kda_decode_step_host",
-                    "kda_decode_step_host_workspace_bytes")
+                    "kda_decode_step_host_workspace_bytes", "kda_set_schedule", "kda_get_schedule")
 
 _DT = {torch.float32: 0, torch.bfloat16: 1}
 _vp = ctypes.c_void_p
@@ -117,6 +117,10 @@ def library() -> ctypes.CDLL:
             lib.kda_decode_step_host.restype = _i
             lib.kda_decode_step_host_workspace_bytes.argtypes = [_i] * 7
             lib.kda_decode_step_host_workspace_bytes.restype = ctypes.c_size_t
+            lib.kda_set_schedule.argtypes = [_i]
+            lib.kda_set_schedule.restype = _i
+            lib.kda_get_schedule.argtypes = []
+            lib.kda_get_schedule.restype = _i
             _lib = lib
     return _lib
 
@@ -127,6 +131,42 @@ def status_string(code: int) -> str:
 
 def version() -> int:
     return library().kda_version()
+
+
+_SCHEDULES = {"auto": 0, "chunked": 1, "scan": 2}
+
+
+def set_schedule(name: str) -> None:
+    """Process-wide prefill schedule (kda_set_schedule): "auto" (the tensor-core chunk
+    kernel where it applies, the column scan otherwise), "chunked" or "scan"."""
+    if name not in _SCHEDULES:
+        raise ValueError(f"unknown schedule {name!r}; expected one of {sorted(_SCHEDULES)}")
+    code = library().kda_set_schedule(_SCHEDULES[name])
+    if code != 0:
+        raise KDAError("kda_set_schedule", code)
+
+
+def get_schedule() -> str:
+    code = library().kda_get_schedule()
+    return {v: k for k, v in _SCHEDULES.items()}[code]
+
+
+class schedule:
+    """Context manager: ``with schedule("chunked"): ...`` sets the prefill schedule for
+    the block and restores the previous one after it."""
+
+    def __init__(self, name: str):
+        self.name = name
+        self.prev = None
+
+    def __enter__(self):
+        self.prev = get_schedule()
+        set_schedule(self.name)
+        return self
+
+    def __exit__(self, *exc):
+        set_schedule(self.prev)
+        return False
 
 
 def _ptr(t):

@@ -57,12 +57,42 @@ typedef enum {
     KDA_ERR_WORKSPACE = 6,   /* workspace too small or NULL when required */
     KDA_ERR_LAUNCH = 7,      /* the CUDA launch reported an error */
     KDA_ERR_TIMEOUT = 8,     /* a bounded device-side wait gave up */
-    KDA_ERR_ALIAS = 9        /* an output overlaps an input it must not alias */
+    KDA_ERR_ALIAS = 9,       /* an output overlaps an input it must not alias */
+    KDA_ERR_VALUE = 10       /* an enumerated argument has an unknown value */
 } kda_status;
 
 /*
+ * Prefill schedule, process-wide (every prefill entry point that runs plain
+ * KDA or the per-head gate: kda_forward, kda_forward_scalar_gate, the packed
+ * kda_forward_varlen, their no-alloc and host-buffer forms).
+ *   KDA_SCHEDULE_AUTO     (default) the tensor-core chunk kernel where it
+ *                         applies (d_k = d_v = 128, bf16 inputs and gates),
+ *                         otherwise the column scan (it is faster than the
+ *                         CUDA-core chunk kernel at every size measured).
+ *   KDA_SCHEDULE_CHUNKED  always the chunkwise schedule.
+ *   KDA_SCHEDULE_SCAN     always the column scan where it applies.
+ * The column scan is the token-by-token recurrence with every value column of
+ * the state run as a chain of its own (column j of S depends only on k, q,
+ * alpha, beta and v_j): "Kimi Delta Attention (KDA)" (brain.bigb.es), "Two
+ * schedules for the same recurrence", the fused recurrent form.  It does not
+ * take raw inputs or GDN-2 gates; those always run chunkwise.  Both schedules
+ * give the recurrence's result up to rounding.
+ */
+typedef enum { KDA_SCHEDULE_AUTO = 0, KDA_SCHEDULE_CHUNKED = 1, KDA_SCHEDULE_SCAN = 2 } kda_schedule;
+
+/* Set the prefill schedule for later calls (KDA_ERR_VALUE for an unknown
+ * value; the setting is then unchanged).  Affects calls made after it returns,
+ * on any thread. */
+kda_status kda_set_schedule(int schedule);
+
+/* The current prefill schedule. */
+int kda_get_schedule(void);
+
+/*
  * kda_forward -- prefill: run the recurrence over T tokens for B sequences and
- * H heads with the chunkwise-parallel schedule.
+ * H heads with the chunkwise-parallel schedule on the tensor cores (d_k = d_v
+ * = 128, bf16 inputs and gates), or with the column scan for other shapes and
+ * dtypes (see kda_set_schedule).
  *
  * Defined by: "Kimi Delta Attention (KDA)" (brain.bigb.es), "Two schedules for
  * the same recurrence" (provisional errors, the unit-lower-triangular

@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_status_strings(lib):
     assert kda.status_string(OK) == "ok"
-    for code in range(1, 10):
+    for code in range(1, 11):
         assert kda.status_string(code) not in ("ok", "unknown status")
     assert kda.version() >= 100
 
@@ -222,3 +222,22 @@ def test_varlen_raw_and_gdn2_reject_bad_arguments(lib):
     assert g(e=0x50004) == ERR_ALIGN                        # the erase gate needs 16-byte rows
     assert g(o=0x70000 + 64) == ERR_ALIAS                   # o overlaps the write gate
     assert g(cu=None) == ERR_NULL
+
+
+def test_schedule_setting_round_trip_and_rejection(lib):
+    """The process-wide prefill schedule: every known value round-trips, an unknown one
+    returns KDA_ERR_VALUE (10) and leaves the setting as it was."""
+    prev = lib.kda_get_schedule()
+    try:
+        for value in (1, 2, 0):
+            assert lib.kda_set_schedule(value) == OK
+            assert lib.kda_get_schedule() == value
+        assert lib.kda_set_schedule(3) == 10 and lib.kda_get_schedule() == 0
+        assert lib.kda_set_schedule(-1) == 10 and lib.kda_get_schedule() == 0
+        with kda.schedule("scan"):
+            assert kda.get_schedule() == "scan"
+        assert kda.get_schedule() == "auto"
+        with pytest.raises(ValueError):
+            kda.set_schedule("fastest")
+    finally:
+        lib.kda_set_schedule(prev)
