@@ -20,11 +20,11 @@ bool scan_supported(const ChunkArgs &a)
 }
 
 // Measured on a B200 (T = 2048, CUDA events): the scan is faster than the CUDA-core chunk
-// kernel at every size tried (d = 64: 4 heads 0.39 against 1.32 ms, 1184 heads 5.8
-// against 12.5 ms; d = 128 fp32: 128 heads 2.6 against 3.5 ms), and slower than the
-// tensor-core chunk kernel even for one head (d = 128 bf16: 0.57 against 0.24 ms).  So
-// the scan replaces the CUDA-core chunk kernel wherever it applies and never the
-// tensor-core one.
+// kernel at every size tried (d = 64: 4 heads 0.37 against 1.32 ms, 1184 heads 4.4
+// against 12.5 ms; d = 128 fp32: 128 heads 2.7 against 3.5 ms; d = 16: 0.25 against
+// 0.37 ms), and slower than the tensor-core chunk kernel even for few heads (d = 128
+// bf16, 4 heads: 0.46 against 0.24 ms).  So the scan replaces the CUDA-core chunk kernel
+// wherever it applies and never the tensor-core one.
 bool scan_preferred(const ChunkArgs &a, int dk, int dv, bool tc)
 {
     (void)dk;

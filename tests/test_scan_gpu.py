@@ -73,11 +73,12 @@ def test_ragged_lengths_and_head_sizes(T, dk, dv):
     assert o_err(o, o_ref) < TOL_F32 and s_err(S, s_ref) < TOL_F32
 
 
-@pytest.mark.parametrize("H", [4, 20, 40])
-def test_block_widths(H):
-    """1, 2 and 4 warps per block (the launch picks them from the warp count: 4 H d/4
-    against 2 and 4 times the 148 SMs)."""
-    w = WORKLOADS["small"].scaled(T=45, H=H)
+@pytest.mark.parametrize("H,d", [(4, 64), (4, 32), (20, 64), (40, 64)])
+def test_launch_forms(H, d):
+    """The launch forms: one column a group of 16 lanes (d = 64: H d/2 = 128 warps, within
+    4 a SM) or 8 lanes (d = 32), two columns a group of 8 lanes with one warp a block
+    (H d/8 = 160 warps) and with two (320 warps, at least two a SM)."""
+    w = WORKLOADS["small"].scaled(T=45, H=H, dk=d, dv=d)
     x = make_inputs(w)
     o_ref, s_ref = oracle_full(x)
     with kda.schedule("scan"):
