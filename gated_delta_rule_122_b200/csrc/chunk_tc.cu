@@ -1035,7 +1035,7 @@ __device__ __forceinline__ void extreme_chunk(const ChunkArgs &p, uint8_t *sm, u
 }
 
 // ---- the chain warps: the serial recurrence over chunks --------------------------------
-template <int kGate, bool kRaw>
+template <int kGate, bool kRaw, bool kLateB>
 __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, uint32_t tmem, const Bars &bars,
                            const TmaPos &tp, const SeqSpan &sp, int h, int bh, int nchunks, volatile int *err_flag)
 {
@@ -1136,9 +1136,11 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
         if (!ptx::mbar_wait(bars.s, (uint32_t)(c & 1), kWaitLimitNs)) *err_flag = 1;
         ptx::tc_fence_after();
         const bool xn = c + 1 < nchunks && chunk_is_extreme(sm, c + 1);
-        // R of chunk c+2 (the update of chunk c has read R(c)) is written after the state
-        // rewrite below, which is on the chain; before a token-by-token chunk, here
-        if (xc && c + 2 < nchunks) {
+        // R of chunk c+2 (the update of chunk c has read R(c)): here, or (kLateB) after the
+        // state rewrite below, which is on the chain -- measured faster when the grid has
+        // more blocks than half the SMs, slower when it has fewer; before a token-by-token
+        // chunk always here
+        if ((xc || !kLateB) && c + 2 < nchunks) {
             stage_b(sm, c + 2, warp, lane, ie);
             warp_signal_after_stage(bars, c + 2, lane);
         }
@@ -1207,7 +1209,7 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             warp_signal(bars.rs, lane);
-            if (c + 2 < nchunks) {   // R of chunk c+2, once S' is out
+            if (kLateB && c + 2 < nchunks) {   // R of chunk c+2, once S' is out
                 stage_b(sm, c + 2, warp, lane, ie);
                 warp_signal_after_stage(bars, c + 2, lane);
             }
@@ -1277,7 +1279,7 @@ __device__ void chain_role(const ChunkArgs &p, const TcMaps &maps, uint8_t *sm, 
 // kGate: alpha per key channel [B, T, H, d_k], or one retention factor per (token, head),
 // alpha [B, T, H] (Gated DeltaNet), staged by TMA or read from memory.
 // kRaw: the input preprocessing is fused into the kernel (raw q, k and logits).
-template <int kGate, bool kRaw>
+template <int kGate, bool kRaw, bool kLateB>
 __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs pa, const __grid_constant__ TcMaps maps)
 {
     extern __shared__ __align__(1024) uint8_t sm[];
@@ -1347,7 +1349,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs pa, const
     } else if (warp >= NCW) {
         prep_role<kGate, kRaw>(p, maps, sm, tmem, bars, tp, sp, h, nchunks, err_flag);
     } else {
-        chain_role<kGate, kRaw>(p, maps, sm, tmem, bars, tp, sp, h, bh, nchunks, err_flag);
+        chain_role<kGate, kRaw, kLateB>(p, maps, sm, tmem, bars, tp, sp, h, bh, nchunks, err_flag);
     }
     if (*err_flag && tid == 0 && p.status) atomicOr(p.status, 1u);
     ptx::tc_fence_before();
@@ -1464,11 +1466,25 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, int dk, int dv, cudaStream_t str
         !encode_out(&maps.o, a.o, mb, a.T, a.H, a.out_bf16))
         return cudaErrorInvalidValue;
     if (a.gate_per_head && a.raw_inputs) return cudaErrorInvalidValue;
-    auto kernel = gdn2            ? tc::kda_chunk_tc_kernel<tc::kGateGdn2, false>
-                  : a.gate_per_head ? (head_gate_tma ? tc::kda_chunk_tc_kernel<tc::kGateHeadTma, false>
-                                                     : tc::kda_chunk_tc_kernel<tc::kGateHeadMem, false>)
-                  : a.raw_inputs    ? tc::kda_chunk_tc_kernel<tc::kGateChannel, true>
-                                    : tc::kda_chunk_tc_kernel<tc::kGateChannel, false>;
+    // R of the chunk two ahead staged after the state rewrite when the grid fills more than
+    // half the SMs (prefill workload, 128 blocks: 2 % faster), before it otherwise (long
+    // workload, 64 blocks: 3 % faster); measured on a B200.  A compile-time choice: as a
+    // run-time flag the two placements in one kernel made the first 3.5 % slower.
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const bool late_b = 2 * blocks > sms;
+    auto pick = [&](auto k_late, auto k_early) { return late_b ? k_late : k_early; };
+    using tc::kda_chunk_tc_kernel;
+    auto kernel = gdn2 ? pick(kda_chunk_tc_kernel<tc::kGateGdn2, false, true>, kda_chunk_tc_kernel<tc::kGateGdn2, false, false>)
+                  : a.gate_per_head
+                      ? (head_gate_tma ? pick(kda_chunk_tc_kernel<tc::kGateHeadTma, false, true>,
+                                              kda_chunk_tc_kernel<tc::kGateHeadTma, false, false>)
+                                       : pick(kda_chunk_tc_kernel<tc::kGateHeadMem, false, true>,
+                                              kda_chunk_tc_kernel<tc::kGateHeadMem, false, false>))
+                  : a.raw_inputs ? pick(kda_chunk_tc_kernel<tc::kGateChannel, true, true>,
+                                        kda_chunk_tc_kernel<tc::kGateChannel, true, false>)
+                                 : pick(kda_chunk_tc_kernel<tc::kGateChannel, false, true>,
+                                        kda_chunk_tc_kernel<tc::kGateChannel, false, false>);
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     kernel<<<(unsigned)blocks, tc::NT, tc::SMEM_BYTES, stream>>>(a, maps);
