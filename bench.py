@@ -41,13 +41,13 @@ if ROOT not in sys.path:
 METRIC = "KDA prefill Mtokens/s (H=64,d=128); decode-step HBM GB/s vs ~8 TB/s peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch of the prefill
-# kernel on the prefill workload (1.0831 GB read + 0.5106 GB written) and on the long
-# workload (4.3137 GB + 2.1217 GB), from the captures summarised under profiles/, with
+# kernel on the prefill workload (1.0760 GB read + 0.5088 GB written) and on the long
+# workload (4.3124 GB + 2.1222 GB), from the captures summarised under profiles/, with
 # the hash of the kernel sources they were taken for: once the sources change, the
 # line reports traffic as null until it is captured again.
-PREFILL_TRAFFIC_BYTES = 1_083_118_080 + 510_573_312
-LONG_TRAFFIC_BYTES = 4_313_738_240 + 2_121_667_840
-PREFILL_TRAFFIC_SOURCES = "f31e3e424745f84e"
+PREFILL_TRAFFIC_BYTES = 1_075_956_736 + 508_817_664
+LONG_TRAFFIC_BYTES = 4_312_354_048 + 2_122_153_728
+PREFILL_TRAFFIC_SOURCES = "57896cee10ccb20d"
 
 
 def kernel_sources_hash() -> str:
@@ -72,9 +72,9 @@ def parse_args():
     ap.add_argument("--no-long", action="store_true", help="skip the long-prefill measurement")
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="run one kernel per step (for profiling); the JSON line is then partial")
-    ap.add_argument("--prefill-workload", choices=["prefill", "long"], default="prefill",
-                    help="the prefill workload of each step (profiling the long workload; the JSON line "
-                         "then describes that workload)")
+    ap.add_argument("--prefill-workload", choices=["prefill", "long", "small"], default="prefill",
+                    help="the prefill workload of each step (profiling the long or the small workload; the "
+                         "JSON line then describes that workload)")
     ap.add_argument("--prefill-seqs", type=int, default=None,
                     help="sequences per rank of the prefill workload (profiling a smaller case; "
                          "the JSON line then describes that case, not the headline workload)")
@@ -550,8 +550,10 @@ def main():
         return
     headline = args.prefill_seqs is None and args.prefill_len is None and args.prefill_workload == "prefill"
     traffic = PREFILL_TRAFFIC_BYTES if headline and kernel_sources_hash() == PREFILL_TRAFFIC_SOURCES else None
-    workload_desc = (f"{wp.name} B={wp.B * world} H={wp.H} T={wp.T} d_k=d_v={wp.dk} bf16 q/k/v/alpha/beta, "
-                     "fp32 o and state" + (", random initial state" if wp.init_state else ""))
+    dt = {torch.bfloat16: "bf16", torch.float32: "fp32"}
+    workload_desc = (f"{wp.name} B={wp.B * world} H={wp.H} T={wp.T} d_k=d_v={wp.dk} {dt[wp.qkv_dtype]} q/k/v, "
+                     f"{dt[wp.gate_dtype]} alpha/beta, fp32 o and state"
+                     + (", random initial state" if wp.init_state else ""))
     if args.only != "prefill":
         workload_desc += f" (+ decode step N={wd.B * world} H={wd.H} d={wd.dk} in the same step)"
     line = {
