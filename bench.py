@@ -47,7 +47,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # line reports traffic as null until it is captured again.
 PREFILL_TRAFFIC_BYTES = 1_075_956_736 + 508_817_664
 LONG_TRAFFIC_BYTES = 4_312_354_048 + 2_122_153_728
-PREFILL_TRAFFIC_SOURCES = "57896cee10ccb20d"
+PREFILL_TRAFFIC_SOURCES = "354174ffce65341e"
 
 
 def kernel_sources_hash() -> str:

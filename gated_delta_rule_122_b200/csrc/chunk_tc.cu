@@ -1466,25 +1466,23 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, int dk, int dv, cudaStream_t str
         !encode_out(&maps.o, a.o, mb, a.T, a.H, a.out_bf16))
         return cudaErrorInvalidValue;
     if (a.gate_per_head && a.raw_inputs) return cudaErrorInvalidValue;
-    // R of the chunk two ahead staged after the state rewrite when the grid fills more than
-    // half the SMs (prefill workload, 128 blocks: 2 % faster), before it otherwise (long
-    // workload, 64 blocks: 3 % faster); measured on a B200.  A compile-time choice: as a
-    // run-time flag the two placements in one kernel made the first 3.5 % slower.
+    // The plain kernel stages R of the chunk two ahead after the state rewrite when the grid
+    // fills more than half the SMs (prefill workload, 128 blocks: 2 % faster), before it
+    // otherwise (long workload, 64 blocks: 3 % faster); the other gate kinds and the raw
+    // inputs always before it (at 128 blocks the late form made them 3.4-5.5 % slower).
+    // Measured on a B200, two builds timed alternately in one process.  A compile-time
+    // choice: as a run-time flag the two placements in one kernel made the late one 3.5 %
+    // slower.
     int sms = 148, dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const bool late_b = 2 * blocks > sms;
-    auto pick = [&](auto k_late, auto k_early) { return late_b ? k_late : k_early; };
     using tc::kda_chunk_tc_kernel;
-    auto kernel = gdn2 ? pick(kda_chunk_tc_kernel<tc::kGateGdn2, false, true>, kda_chunk_tc_kernel<tc::kGateGdn2, false, false>)
-                  : a.gate_per_head
-                      ? (head_gate_tma ? pick(kda_chunk_tc_kernel<tc::kGateHeadTma, false, true>,
-                                              kda_chunk_tc_kernel<tc::kGateHeadTma, false, false>)
-                                       : pick(kda_chunk_tc_kernel<tc::kGateHeadMem, false, true>,
-                                              kda_chunk_tc_kernel<tc::kGateHeadMem, false, false>))
-                  : a.raw_inputs ? pick(kda_chunk_tc_kernel<tc::kGateChannel, true, true>,
-                                        kda_chunk_tc_kernel<tc::kGateChannel, true, false>)
-                                 : pick(kda_chunk_tc_kernel<tc::kGateChannel, false, true>,
-                                        kda_chunk_tc_kernel<tc::kGateChannel, false, false>);
+    auto kernel = gdn2            ? kda_chunk_tc_kernel<tc::kGateGdn2, false, false>
+                  : a.gate_per_head ? (head_gate_tma ? kda_chunk_tc_kernel<tc::kGateHeadTma, false, false>
+                                                     : kda_chunk_tc_kernel<tc::kGateHeadMem, false, false>)
+                  : a.raw_inputs    ? kda_chunk_tc_kernel<tc::kGateChannel, true, false>
+                  : late_b          ? kda_chunk_tc_kernel<tc::kGateChannel, false, true>
+                                    : kda_chunk_tc_kernel<tc::kGateChannel, false, false>;
     cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES);
     if (err != cudaSuccess) return err;
     kernel<<<(unsigned)blocks, tc::NT, tc::SMEM_BYTES, stream>>>(a, maps);
