@@ -216,3 +216,26 @@ def test_unknown_schedule_rejected():
     with pytest.raises(ValueError):
         kda.set_schedule("fastest")
     assert kda.library().kda_set_schedule(3) == 10   # KDA_ERR_VALUE, setting unchanged
+
+
+def test_variants_without_a_scan_stay_chunkwise():
+    """Raw inputs and GDN-2 gates have no column-scan form: with the scan forced they run
+    the chunk kernels, bit-identical to the chunkwise schedule."""
+    x = to_device(make_inputs(WORKLOADS["small"].scaled(T=70, H=2)))
+    a = x["alpha"].float().clamp(1e-30, 1 - 1e-7)
+    gl = torch.log((1 - a) / a).to(x["alpha"].dtype)
+    bt = x["beta"].float().clamp(1e-7, 1 - 1e-7)
+    bl = torch.log(bt / (1 - bt)).to(x["beta"].dtype)
+    er = torch.sigmoid(torch.randn(x["k"].shape, generator=torch.Generator().manual_seed(3))).to(x["alpha"].dtype).cuda()
+    wr = torch.sigmoid(torch.randn(x["v"].shape, generator=torch.Generator().manual_seed(4))).to(x["alpha"].dtype).cuda()
+    res = {}
+    for sched in ("scan", "chunked"):
+        with kda.schedule(sched):
+            raw = kda.forward_raw(x["q"], x["k"], x["v"], gl, bl, initial_state=x["s0"], scale=x["scale"],
+                                  check_status=True)
+            g2 = kda.forward_gdn2(x["q"], x["k"], x["v"], x["alpha"], er, wr, initial_state=x["s0"],
+                                  scale=x["scale"], check_status=True)
+        res[sched] = (raw, g2)
+    for i in range(2):
+        for j in range(2):
+            assert torch.equal(res["scan"][i][j], res["chunked"][i][j])
