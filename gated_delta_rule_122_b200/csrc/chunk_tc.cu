@@ -257,34 +257,45 @@ struct MmaIds {
     uint32_t A, W, U, OE, O2, dS;
 };
 
+// Descriptor of the operand bytes further on than desc's: the start address field holds
+// address / 16 in its low 14 bits, and every operand here lies below 256 KB of shared
+// memory, so the step is a plain add (built once per group, not once per MMA).
+__device__ __forceinline__ uint64_t desc_at(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
+
 __device__ __forceinline__ void issue_m3(uint8_t *sm, uint32_t tmem, const Bars &bars, const MmaIds &id, int n3)
 {
     ptx::tc_fence_after();
-    const uint32_t b0 = ptx::smem_u32(sm + OFF_LQR + (n3 & 1) * LQR_BYTES) + SL_LQ * SLAB;
+    const uint64_t lq = ptx::smem_desc(ptx::smem_u32(sm + OFF_LQR + (n3 & 1) * LQR_BYTES) + SL_LQ * SLAB, 128, SLAB);
+#pragma unroll
     for (int ks = 0; ks < D / 16; ++ks)
+#pragma unroll
         for (int pl = 0; pl < 2; ++pl)
-            ptx::mma_bf16_ts(tmem + TM_O, tmem + TM_SP + 64 * pl + 8 * ks,
-                             ptx::smem_desc(b0 + 256 * ks, 128, SLAB), id.OE, 1);
+            ptx::mma_bf16_ts(tmem + TM_O, tmem + TM_SP + 64 * pl + 8 * ks, desc_at(lq, 256 * ks), id.OE, 1);
     ptx::mma_commit(bars.e);
 }
 
 __device__ __forceinline__ void issue_m4(uint8_t *sm, uint32_t tmem, const Bars &bars, const MmaIds &id, int n4)
 {
     ptx::tc_fence_after();
-    const uint32_t et = ptx::smem_u32(sm + OFF_ET);
-    const uint32_t aq = ptx::smem_u32(sm + OFF_AQ + (n4 & 1) * AQ_BYTES);
-    const uint32_t rr = ptx::smem_u32(sm + OFF_LQR + (n4 & 1) * LQR_BYTES) + SL_R * SLAB;
+    const uint64_t et = ptx::smem_desc(ptx::smem_u32(sm + OFF_ET), 128, C * 32);
+    const uint64_t aq = ptx::smem_desc(ptx::smem_u32(sm + OFF_AQ + (n4 & 1) * AQ_BYTES), 128, 512);
+    const uint64_t rr =
+        ptx::smem_desc(ptx::smem_u32(sm + OFF_LQR + (n4 & 1) * LQR_BYTES) + SL_R * SLAB, 2 * SLAB, 128);
+#pragma unroll
     for (int ks = 0; ks < C / 16; ++ks)
+#pragma unroll
         for (int pl = 0; pl < 2; ++pl)
-            ptx::mma_bf16(tmem + TM_O, ptx::smem_desc(et + C * 16 * pl + 256 * ks, 128, C * 32),
-                          ptx::smem_desc(aq + 256 * ks, 128, 512), id.O2, 1);
+            ptx::mma_bf16(tmem + TM_O, desc_at(et, C * 16 * pl + 256 * ks), desc_at(aq, 256 * ks), id.O2, 1);
+#pragma unroll
     for (int ks = 0; ks < C / 16; ++ks)
+#pragma unroll
         for (int pa = 0; pa < 2; ++pa)
+#pragma unroll
             for (int pb = 0; pb < 2 - pa; ++pb)
                 // R as the K-major (N = d, K = s) operand: token blocks 2 slabs apart.  The
                 // E_lo R_lo term (2^-16 of the product) is left out: three cross terms.
-                ptx::mma_bf16(tmem + TM_S, ptx::smem_desc(et + C * 16 * pa + 256 * ks, 128, C * 32),
-                              ptx::smem_desc(rr + SLAB * pb + 4 * SLAB * ks, 2 * SLAB, 128), id.dS, 1);
+                ptx::mma_bf16(tmem + TM_S, desc_at(et, C * 16 * pa + 256 * ks),
+                              desc_at(rr, SLAB * pb + 4 * SLAB * ks), id.dS, 1);
     ptx::mma_commit(bars.s);
 }
 
@@ -292,9 +303,10 @@ __device__ __forceinline__ void issue_m1(uint8_t *sm, uint32_t tmem, const Bars 
 {
     ptx::tc_fence_after();
     const uint32_t base = ptx::smem_u32(sm + OFF_LQR + (n1 & 1) * LQR_BYTES);
+    const uint64_t lk = ptx::smem_desc(base + SL_LK * SLAB, 128, SLAB), r = ptx::smem_desc(base + SL_R * SLAB, 128, SLAB);
+#pragma unroll
     for (int ks = 0; ks < D / 16; ++ks)
-        ptx::mma_bf16(tmem + TM_A, ptx::smem_desc(base + SL_LK * SLAB + 256 * ks, 128, SLAB),
-                      ptx::smem_desc(base + SL_R * SLAB + 256 * ks, 128, SLAB), id.A, ks > 0);
+        ptx::mma_bf16(tmem + TM_A, desc_at(lk, 256 * ks), desc_at(r, 256 * ks), id.A, ks > 0);
     ptx::mma_commit(bars.a);
 }
 
@@ -302,22 +314,27 @@ template <int kGate, bool kRaw>
 __device__ __forceinline__ void issue_m2(uint8_t *sm, uint32_t tmem, const Bars &bars, const MmaIds &id, int n2)
 {
     ptx::tc_fence_after();
-    const uint32_t base = ptx::smem_u32(sm + OFF_LQR + (n2 & 1) * LQR_BYTES);
-    const uint32_t tp = ptx::smem_u32(sm + OFF_TP);
+    const uint64_t lk = ptx::smem_desc(ptx::smem_u32(sm + OFF_LQR + (n2 & 1) * LQR_BYTES) + SL_LK * SLAB, 2 * SLAB, 128);
+    const uint64_t tp = ptx::smem_desc(ptx::smem_u32(sm + OFF_TP), 128, 512);
     // GDN-2: one V stage holding the hi and lo planes of w * v in the two V buffers
-    const uint32_t vv = ptx::smem_u32(sm + OFF_V + (kGate == kGateGdn2 ? 0 : (n2 & 1) * V_BYTES));
+    const uint64_t vv = ptx::smem_desc(ptx::smem_u32(sm + OFF_V + (kGate == kGateGdn2 ? 0 : (n2 & 1) * V_BYTES)), 128,
+                                       (C / 8) * 128);
+#pragma unroll
     for (int ks = 0; ks < C / 16; ++ks)
+#pragma unroll
         for (int pl = 0; pl < 2; ++pl)
             // Lk plane pl as the K-major (M = d, K = s) operand: token blocks 2 slabs apart
-            ptx::mma_bf16(tmem + TM_W,
-                          ptx::smem_desc(base + (SL_LK + pl) * SLAB + 4 * SLAB * ks, 2 * SLAB, 128),
-                          ptx::smem_desc(tp + 256 * ks, 128, 512), id.W, ks > 0 || pl > 0);
-    const uint32_t tu = kRaw ? ptx::smem_u32(sm + OFF_TPU) : tp;   // raw inputs: T Diag(beta) for U
+            ptx::mma_bf16(tmem + TM_W, desc_at(lk, pl * SLAB + 4 * SLAB * ks), desc_at(tp, 256 * ks), id.W,
+                          ks > 0 || pl > 0);
+    // raw inputs: T Diag(beta) for U
+    const uint64_t tu = kRaw ? ptx::smem_desc(ptx::smem_u32(sm + OFF_TPU), 128, 512) : tp;
     constexpr int kVPlanes = kGate == kGateGdn2 ? 2 : 1;
+#pragma unroll
     for (int ks = 0; ks < C / 16; ++ks)
+#pragma unroll
         for (int pl = 0; pl < kVPlanes; ++pl)
-            ptx::mma_bf16(tmem + TM_E, ptx::smem_desc(vv + pl * V_BYTES + 256 * ks, 128, (C / 8) * 128),
-                          ptx::smem_desc(tu + 256 * ks, 128, 512), id.U, ks > 0 || pl > 0);
+            ptx::mma_bf16(tmem + TM_E, desc_at(vv, pl * V_BYTES + 256 * ks), desc_at(tu, 256 * ks), id.U,
+                          ks > 0 || pl > 0);
     ptx::mma_commit(bars.w);
 }
 
