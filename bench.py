@@ -42,12 +42,12 @@ METRIC = "KDA prefill Mtokens/s (H=64,d=128); decode-step HBM GB/s vs ~8 TB/s pe
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch of the prefill
 # kernel on the prefill workload (1.0760 GB read + 0.5088 GB written) and on the long
-# workload (4.3124 GB + 2.1222 GB), from the captures summarised under profiles/, with
+# workload (4.3134 GB + 2.1216 GB), from the captures summarised under profiles/, with
 # the hash of the kernel sources they were taken for: once the sources change, the
 # line reports traffic as null until it is captured again.
-PREFILL_TRAFFIC_BYTES = 1_075_956_736 + 508_817_664
-LONG_TRAFFIC_BYTES = 4_312_354_048 + 2_122_153_728
-PREFILL_TRAFFIC_SOURCES = "354174ffce65341e"
+PREFILL_TRAFFIC_BYTES = 1_075_952_128 + 508_771_072
+LONG_TRAFFIC_BYTES = 4_313_396_736 + 2_121_649_920
+PREFILL_TRAFFIC_SOURCES = "ac2c07ca88d4093f"
 
 
 def kernel_sources_hash() -> str:
