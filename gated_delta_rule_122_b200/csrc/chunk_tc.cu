@@ -340,14 +340,15 @@ __device__ __forceinline__ void issue_m2(uint8_t *sm, uint32_t tmem, const Bars 
 
 // The issuer takes the groups in a fixed order, waiting on each group's readiness
 // mbarriers (the warp sleeps in the wait and wakes when the phase completes):
-//   M1(0), M1(1), M2(0), then for each chunk c: M3(c), M4(c), M2(c+1), M1(c+2).
+//   M1(0), M1(1), M2(0), then for each chunk c: M3(c), M4(c), M2(c+1), M1(c+2)
+// (with R staged after the state rewrite: M1(0), M2(0), then M3(c), M1(c+1), M4(c), M2(c+1)).
 // M1(n) needs Lk, Lq, R of chunk n (rc) and A(n-1) read by the prep warps (ra, since
 // A(n) overwrites it); M2(n) needs T' and A_qk (rg, which the prep warps signal after
 // reading W'(n-1)) and the E readout of chunk n-1 (U(n) overwrites E in TMEM; implied
 // by M4(n-1) having been issued); M3(n) needs S'(n) (rs) and -W'(n) (rj); M4(n) needs
 // E^T(n) (re).  Each producer is at most one phase ahead of this order: every arrival
 // for chunk n+1 depends on a group of chunk n that is issued after the wait for chunk n.
-template <int kGate, bool kRaw>
+template <int kGate, bool kRaw, bool kLateB>
 __device__ void issuer(uint8_t *sm, uint32_t tmem, const Bars &bars, int nchunks, volatile int *err_flag)
 {
     MmaIds id;
@@ -370,15 +371,18 @@ __device__ void issuer(uint8_t *sm, uint32_t tmem, const Bars &bars, int nchunks
     auto m2 = [&](int n) {
         if (wait(bars.rg, n)) issue_m2<kGate, kRaw>(sm, tmem, bars, id, n);
     };
+    // kLateB (R staged after the state rewrite, so that rc(c+2) arrives after rs(c+1)):
+    // M3(c), M1(c+1), M4(c), M2(c+1), so that M3(c+1) does not queue behind M1(c+2)
     m1(0);
-    if (nchunks > 1) m1(1);
+    if (!kLateB && nchunks > 1) m1(1);
     m2(0);
     for (int c = 0; c < nchunks && ok; ++c) {
         wait(bars.rs, c);
         if (wait(bars.rj, c)) issue_m3(sm, tmem, bars, id, c);
+        if (kLateB && c + 1 < nchunks) m1(c + 1);
         if (wait(bars.re, c)) issue_m4(sm, tmem, bars, id, c);
         if (c + 1 < nchunks) m2(c + 1);
-        if (c + 2 < nchunks) m1(c + 2);
+        if (!kLateB && c + 2 < nchunks) m1(c + 2);
         if (*err_flag) ok = false;
     }
     if (!ok) *err_flag = 1;
@@ -1362,7 +1366,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(ChunkArgs pa, const
     const uint32_t tmem = *tmem_slot;
 
     if (warp == kIssuerWarp) {
-        if (lane == 0) issuer<kGate, kRaw>(sm, tmem, bars, nchunks, err_flag);
+        if (lane == 0) issuer<kGate, kRaw, kLateB>(sm, tmem, bars, nchunks, err_flag);
     } else if (warp >= NCW) {
         prep_role<kGate, kRaw>(p, maps, sm, tmem, bars, tp, sp, h, nchunks, err_flag);
     } else {
