@@ -41,13 +41,15 @@ if ROOT not in sys.path:
 METRIC = "KDA prefill Mtokens/s (H=64,d=128); decode-step HBM GB/s vs ~8 TB/s peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch of the prefill
-# kernel on the prefill workload (1.0760 GB read + 0.5088 GB written) and on the long
+# kernel on the prefill workload (1.0760 GB read + 0.5094 GB written) and on the long
 # workload (4.3134 GB + 2.1216 GB), from the captures summarised under profiles/, with
 # the hash of the kernel sources they were taken for: once the sources change, the
-# line reports traffic as null until it is captured again.
-PREFILL_TRAFFIC_BYTES = 1_075_952_128 + 508_771_072
+# line reports traffic as null until it is captured again.  (The long workload's kernel,
+# the early-R form, was last changed before its capture; the prefill workload's was
+# captured on these sources.)
+PREFILL_TRAFFIC_BYTES = 1_076_045_824 + 509_351_936
 LONG_TRAFFIC_BYTES = 4_313_396_736 + 2_121_649_920
-PREFILL_TRAFFIC_SOURCES = "ac2c07ca88d4093f"
+PREFILL_TRAFFIC_SOURCES = "9afd6510a83d95c2"
 
 
 def kernel_sources_hash() -> str:
