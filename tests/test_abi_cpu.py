@@ -241,3 +241,16 @@ def test_schedule_setting_round_trip_and_rejection(lib):
             kda.set_schedule("fastest")
     finally:
         lib.kda_set_schedule(prev)
+
+
+def test_schedule_context_restores_after_an_exception(lib):
+    prev = kda.get_schedule()
+    try:
+        kda.set_schedule("scan")
+        with pytest.raises(RuntimeError):
+            with kda.schedule("chunked"):
+                assert kda.get_schedule() == "chunked"
+                raise RuntimeError("inside the block")
+        assert kda.get_schedule() == "scan"
+    finally:
+        kda.set_schedule(prev)
